@@ -1,0 +1,205 @@
+"""fp64 CPU oracle for grouped-KV scaled-dot-product attention (forward).
+
+TEST INFRASTRUCTURE. Only the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package. The product path (the
+CUDA library and its binding) never imports it, and this package never
+imports the product.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module only marshals arrays. Inputs of any float dtype are widened to
+float64 exactly (bf16 -> fp64 is exact), so the oracle sees the very values
+handed to the GPU.
+
+Functions:
+  sdpa(q, k, v, causal, scale, seqlens=None)      -> (o, lse)   full forward
+  sdpa_rows(q_rows, rows, k, v, ...)             -> (o, lse)   sampled rows
+  row_weights(q_row, b, h, i, k, v, ...)         -> (o, lse, w) one row + softmax weights
+  online(q, k, v, causal, scale, block_r, block_c) -> (o, lse) FlashAttention-2 recurrence
+
+Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
+d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
+latent cache row of 576 can serve as key (all 576) and value (first 512)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle with gcc (-O2 -fopenmp, no fast-math)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def _declare(lib):
+    common = [_int] * 7 + [_i64] * 6 + [_i32p, _int, ctypes.c_double]
+    lib.oracle_sdpa_fp64.argtypes = [_f64p] * 5 + common + [_int]
+    lib.oracle_sdpa_fp64.restype = _int
+    lib.oracle_sdpa_rows_fp64.argtypes = [_f64p] * 5 + [_i32p] * 3 + [_int] + common + [_int]
+    lib.oracle_sdpa_rows_fp64.restype = _int
+    lib.oracle_row_weights_fp64.argtypes = [_f64p] * 6 + [_int] * 3 + common
+    lib.oracle_row_weights_fp64.restype = _i64
+    lib.oracle_online_fp64.argtypes = [_f64p] * 5 + common + [_int, _int, _int]
+    lib.oracle_online_fp64.restype = _int
+    return lib
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the oracle library. A non-default
+    ``path`` loads another build of the same source (used by the mutation
+    tests that plant mistakes in a copy of the oracle)."""
+    global _lib
+    if path is not None:
+        return _declare(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = _declare(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact widening to a C-contiguous float64 array (torch or numpy in)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float64).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _kv_strides(t: np.ndarray):
+    if t.ndim != 4:
+        raise ValueError("k and v must be 4-D [B, n_kv, S, row]")
+    es = t.itemsize
+    return tuple(s // es for s in t.strides[:3])
+
+
+def _ptr(a: np.ndarray, ty=_f64p):
+    return a.ctypes.data_as(ty)
+
+
+def _seq(seqlens):
+    if seqlens is None:
+        return None, None
+    s = np.ascontiguousarray(np.asarray(
+        seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int32))
+    return s, _ptr(s, _i32p)
+
+
+def _nthreads(n):
+    return int(n) if n else 0
+
+
+def sdpa(q, k, v, causal: bool, scale: float, seqlens=None, d_qk=None, d_v=None,
+         nthreads=None, lib=None):
+    """Plain-definition forward. Returns (o [B,n_q,Sq,d_v], lse [B,n_q,Sq]) in fp64."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, n_q, Sq, dq = q.shape
+    _, n_kv, Skv, _ = k.shape
+    d_qk = d_qk or dq
+    d_v = d_v or v.shape[3]
+    if d_qk != dq or d_qk > k.shape[3] or d_v > v.shape[3]:
+        raise ValueError("head dims do not fit the given rows")
+    o = np.zeros((B, n_q, Sq, d_v))
+    lse = np.zeros((B, n_q, Sq))
+    s_arr, s_ptr = _seq(seqlens)
+    rc = lib.oracle_sdpa_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                              B, n_q, n_kv, Sq, Skv, d_qk, d_v,
+                              *_kv_strides(k), *_kv_strides(v), s_ptr,
+                              int(bool(causal)), float(scale), _nthreads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return o, lse
+
+
+def sdpa_rows(q_rows, rows, k, v, B, n_q, Sq, causal: bool, scale: float,
+              seqlens=None, d_v=None, nthreads=None, lib=None):
+    """Sampled rows. ``rows`` is an int array [n, 3] of (b, h, i); ``q_rows``
+    is [n, d_qk] (the query vectors of those rows). Returns (o [n, d_v], lse [n])."""
+    lib = lib or load()
+    q_rows, k, v = _f64(q_rows), _f64(k), _f64(v)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    n, d_qk = q_rows.shape
+    _, n_kv, Skv, _ = k.shape
+    d_v = d_v or v.shape[3]
+    rb = np.ascontiguousarray(rows[:, 0])
+    rh = np.ascontiguousarray(rows[:, 1])
+    ri = np.ascontiguousarray(rows[:, 2])
+    o = np.zeros((n, d_v))
+    lse = np.zeros((n,))
+    s_arr, s_ptr = _seq(seqlens)
+    rc = lib.oracle_sdpa_rows_fp64(_ptr(q_rows), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                   _ptr(rb, _i32p), _ptr(rh, _i32p), _ptr(ri, _i32p), n,
+                                   B, n_q, n_kv, Sq, Skv, d_qk, d_v,
+                                   *_kv_strides(k), *_kv_strides(v), s_ptr,
+                                   int(bool(causal)), float(scale), _nthreads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return o, lse
+
+
+def row_weights(q_row, b, h, i, k, v, B, n_q, Sq, causal: bool, scale: float,
+                seqlens=None, d_v=None, lib=None):
+    """One row: (o [d_v], lse, weights [Skv], n_visible)."""
+    lib = lib or load()
+    q_row, k, v = _f64(q_row).reshape(-1), _f64(k), _f64(v)
+    _, n_kv, Skv, _ = k.shape
+    d_qk = q_row.shape[0]
+    d_v = d_v or v.shape[3]
+    o = np.zeros((d_v,))
+    lse = np.zeros((1,))
+    w = np.zeros((max(Skv, 1),))
+    s_arr, s_ptr = _seq(seqlens)
+    nv = lib.oracle_row_weights_fp64(_ptr(q_row), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(w),
+                                     int(b), int(h), int(i),
+                                     B, n_q, n_kv, Sq, Skv, d_qk, d_v,
+                                     *_kv_strides(k), *_kv_strides(v), s_ptr,
+                                     int(bool(causal)), float(scale))
+    if nv < 0:
+        raise ValueError("oracle rejected the arguments")
+    return o, float(lse[0]), w[:Skv], int(nv)
+
+
+def online(q, k, v, causal: bool, scale: float, block_r: int, block_c: int,
+           seqlens=None, d_v=None, nthreads=None, lib=None):
+    """FlashAttention-2 tiled recurrence in fp64. Returns (o, lse)."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, n_q, Sq, d_qk = q.shape
+    _, n_kv, Skv, _ = k.shape
+    d_v = d_v or v.shape[3]
+    o = np.zeros((B, n_q, Sq, d_v))
+    lse = np.zeros((B, n_q, Sq))
+    s_arr, s_ptr = _seq(seqlens)
+    rc = lib.oracle_online_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                B, n_q, n_kv, Sq, Skv, d_qk, d_v,
+                                *_kv_strides(k), *_kv_strides(v), s_ptr,
+                                int(bool(causal)), float(scale),
+                                int(block_r), int(block_c), _nthreads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return o, lse
