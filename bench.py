@@ -1,0 +1,424 @@
+"""Benchmark of the fused grouped-KV attention forward on B200.
+
+One step = one pass of the hot path over synthetic inputs resident in HBM:
+  * prefill: attn_fwd on the Llama-3-8B-shaped causal GQA workload
+    (B=1, S=4096, 32 query / 8 KV heads, head dim 128) -- the headline;
+  * decode: attn_decode on the GQA decode workload (B=32, cache lengths
+    ~U[1024, 32768], 32/8 heads, head dim 128), split-KV + combine.
+`value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
+decode regime is reported in HBM GB/s (algorithmic bytes: the K/V rows below
+each sequence's length, plus q, o and lse) under "regimes". Each kernel is
+timed with CUDA events on its launching stream; L2 (126 MB) is flushed by
+writing a 512 MB buffer before every timed launch.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU: launched by torchrun, one rank per GPU; every rank runs its own
+replica of the workload (independent problems, weak scaling), time is the max
+over ranks, value the sum of all ranks' work over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill TFLOP/s & decode HBM GB/s (fraction of B200 peak), 1 GPU"
+HEADLINE = "llama3_8b_prefill"
+DECODE = "gqa_decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work
+# ----------------------------------------------------------------------------
+def prefill_flops(w) -> float:
+    """4 * d per visible (query, key) pair per head: 2d for Q.K^T, 2d for P.V."""
+    if w.causal:
+        off = w.Skv - w.Sq
+        pairs = sum(min(w.Skv, i + off + 1) for i in range(w.Sq))
+    else:
+        pairs = w.Sq * w.Skv
+    return float(w.B * w.n_q * pairs * 2 * (w.d_qk + w.d_v))
+
+
+def prefill_bytes(w) -> float:
+    return float(2 * (w.B * w.n_q * w.Sq * (w.d_qk + w.d_v) + w.B * w.n_kv * w.Skv * (w.d_qk + w.d_v))
+                 + 4 * w.B * w.n_q * w.Sq)
+
+
+def decode_bytes(w, seqlens) -> float:
+    """K and V rows below each sequence's length, q, o (bf16) and lse (fp32)."""
+    total_keys = float(sum(int(x) for x in seqlens))
+    kv = total_keys * w.n_kv * (w.d_qk + w.d_v) * 2
+    return kv + w.B * w.n_q * (w.d_qk * 2 + w.d_v * 2 + 4)
+
+
+def decode_flops(w, seqlens) -> float:
+    return float(sum(int(x) for x in seqlens)) * w.n_q * 2 * (w.d_qk + w.d_v)
+
+
+# ----------------------------------------------------------------------------
+# measurement helpers
+# ----------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(values: dict, world_size: int):
+    """Reduce per-rank numbers: max of times, sum of work. `values` holds
+    'time_s' (max-reduced) and 'work' (sum-reduced)."""
+    if world_size <= 1:
+        return dict(values)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([values["time_s"]], dtype=torch.float64, device=dev)
+    w = torch.tensor([values["work"]], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return {"time_s": float(t.item()), "work": float(w.item())}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle leg (reported baseline; also the --impl reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(w, q, k, v, n_rows, seed):
+    """Time the fp64 oracle on a seeded sample of query rows of the workload.
+    Returns (seconds, algorithmic FLOPs of those rows, threads)."""
+    import numpy as np
+    import oracle
+    from mqa_attention_attn_b200 import inputs
+    rows = inputs.sample_rows(n_rows, w.B, w.n_q, w.Sq, seed)[:n_rows]
+    rb, rh, ri = rows[:, 0].long(), rows[:, 1].long(), rows[:, 2].long()
+    q_rows = q[rb, rh, ri]
+    threads = os.cpu_count() or 1
+    kd = oracle._f64(k)
+    vd = oracle._f64(v)
+    off = w.Skv - w.Sq
+    flops = float(sum((min(w.Skv, int(i) + off + 1) if w.causal else w.Skv) for i in ri)) * 2 * (w.d_qk + w.d_v)
+    t0 = time.perf_counter()
+    oracle.sdpa_rows(q_rows, rows.numpy(), kd, vd, w.B, w.n_q, w.Sq, w.causal, w.scale, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return dt, flops, threads
+
+
+def oracle_full(w, q, k, v):
+    """Time the fp64 oracle on the whole workload (every query row).
+    Returns (seconds, algorithmic FLOPs, threads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    qd, kd, vd = oracle._f64(q), oracle._f64(k), oracle._f64(v)
+    t0 = time.perf_counter()
+    oracle.sdpa(qd, kd, vd, w.causal, w.scale, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return dt, prefill_flops(w), threads
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import torch
+    from mqa_attention_attn_b200 import inputs
+    w = inputs.WORKLOADS[HEADLINE]
+    q, k, v = inputs.make(w, device="cpu")
+    n_rows = args.ref_rows
+    for i in range(args.warmup):
+        oracle_sample(w, q, k, v, n_rows, 1000 + i)
+    times, flops = [], []
+    threads = os.cpu_count() or 1
+    for i in range(args.steps):
+        dt, fl, threads = oracle_sample(w, q, k, v, n_rows, 2000 + i)
+        times.append(dt)
+        flops.append(fl)
+    value = sum(flops) / sum(times) / 1e12
+    ms = 1e3 * sum(times) / len(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "S": w.Sq, "n_q": w.n_q, "n_kv": w.n_kv, "d": w.d_qk,
+                   "causal": w.causal, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n_rows} seeded query rows of {w.name} per step (fp64 plain "
+                                   f"definition, OpenMP over rows)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# the CUDA arm
+# ----------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    ws, rank, local = _dist()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    from mqa_attention_attn_b200 import binding, build, inputs
+    build.build_library()
+    binding.lib()
+
+    w = inputs.WORKLOADS[HEADLINE]
+    wd = inputs.WORKLOADS[DECODE]
+    gen_seed_shift = 1000 * rank
+    q, k, v = inputs.prefill_inputs(w.B, w.Sq, w.Skv, w.n_q, w.n_kv, w.d_qk, w.d_v, w.seed + gen_seed_shift,
+                                    device=dev)
+    o = torch.empty((w.B, w.n_q, w.Sq, w.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.n_q, w.Sq), dtype=torch.float32, device=dev)
+    seqlens, qd, kc, vc = inputs.decode_inputs(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv, wd.seqlen_range,
+                                               wd.seed + gen_seed_shift, device=dev)
+    sl_dev = seqlens.to(dev)
+    od = torch.empty((wd.B, wd.n_q, wd.d_v), dtype=torch.bfloat16, device=dev)
+    ld = torch.empty((wd.B, wd.n_q), dtype=torch.float32, device=dev)
+    wsz = binding.decode_workspace_bytes(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv)
+    work = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    stream = torch.cuda.current_stream(dev)
+    fl_p = prefill_flops(w)
+    by_p = prefill_bytes(w)
+    by_d = decode_bytes(wd, seqlens)
+    fl_d = decode_flops(wd, seqlens)
+
+    def step(times_p, times_d):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        binding.attn_fwd(q, k, v, w.causal, w.scale, o=o, lse=lse, stream=stream)
+        e1.record(stream)
+        flush.fill_(2.0)
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        binding.attn_decode(qd, kc, vc, sl_dev, wd.scale, o=od, lse=ld, workspace=work, stream=stream)
+        e3.record(stream)
+        if times_p is not None:
+            times_p.append((e0, e1))
+            times_d.append((e2, e3))
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step(None, None)
+    barrier()
+    assert binding.device_status(stream) == 0, "device status not clean after warm-up"
+
+    tp, td = [], []
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        barrier()
+        t_wall0 = time.perf_counter()
+        for _ in range(args.steps):
+            step(tp, td)
+        barrier()
+        t_wall = time.perf_counter() - t_wall0
+    st = binding.device_status(stream)
+    assert st == 0, f"device status {st}"
+    ms_p = [a.elapsed_time(b) for a, b in tp]
+    ms_d = [a.elapsed_time(b) for a, b in td]
+    mean_p = sum(ms_p) / len(ms_p)
+    mean_d = sum(ms_d) / len(ms_d)
+
+    agg_p = aggregate({"time_s": sum(ms_p) / 1e3, "work": fl_p * args.steps}, ws)
+    agg_d = aggregate({"time_s": sum(ms_d) / 1e3, "work": by_d * args.steps}, ws)
+    value = agg_p["work"] / agg_p["time_s"] / 1e12
+    dec_gbs = agg_d["work"] / agg_d["time_s"] / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        qx, kx, vx = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+        def e2e_step():
+            qx.copy_(qh, non_blocking=True)
+            kx.copy_(kh, non_blocking=True)
+            vx.copy_(vh, non_blocking=True)
+            binding.attn_fwd(qx, kx, vx, w.causal, w.scale, o=o, lse=lse, stream=stream)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record(stream)
+        barrier()
+        e2e_ms = s0.elapsed_time(s1) / args.steps
+        agg_e = aggregate({"time_s": e2e_ms / 1e3, "work": fl_p}, ws)
+        e2e = {"value": agg_e["work"] / agg_e["time_s"] / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    peaks, peak_src = load_peaks()
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_bw = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    achieved_tf = fl_p / (mean_p / 1e3) / 1e12
+    traffic = load_traffic()
+    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved_tf / peak_tf, "traffic": traffic.get("prefill_kernel_128"),
+                "kernel": "attn::pf::prefill_kernel<128>", "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "algorithmic_flops_per_launch": fl_p}
+    dec_achieved = by_d / (mean_d / 1e3) / 1e9
+    regimes = {
+        "prefill": {"workload": w.name, "ms": mean_p, "tflops": achieved_tf,
+                    "frac_of_peak": achieved_tf / peak_tf, "frac_of_nominal_2250": achieved_tf / 2250.0,
+                    "algorithmic_flops": fl_p, "algorithmic_bytes": by_p},
+        "decode": {"workload": wd.name, "ms": mean_d, "gbs": dec_achieved, "aggregate_gbs": dec_gbs,
+                   "frac_of_peak": dec_achieved / peak_bw, "frac_of_nominal_8000": dec_achieved / 8000.0,
+                   "algorithmic_bytes": by_d, "algorithmic_flops": fl_d,
+                   "kernels": "attn::dec::decode_split_kernel<4> + decode_combine_kernel",
+                   "peak": peak_bw, "peak_source": f"{peak_src} hbm_gbs"},
+    }
+
+    cpu_baseline = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        qc, kc_, vc_ = q.cpu(), k.cpu(), v.cpu()
+        dt, fl, threads = oracle_full(w, qc, kc_, vc_)
+        cpu_baseline = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                        "sample": f"the whole {w.name} workload, all {w.B * w.n_q * w.Sq} query rows "
+                                  f"(fp64 plain definition, OpenMP over rows), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": mean_p + mean_d, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "S": w.Sq, "n_q": w.n_q, "n_kv": w.n_kv, "d": w.d_qk,
+                       "causal": w.causal, "decode_workload": wd.name,
+                       "l2": "flushed (512 MB write) before every timed launch",
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+            "roofline": roofline,
+            "regimes": regimes,
+            "cpu_baseline": cpu_baseline,
+            "e2e": e2e,
+            "clocks": clocks.summary(),
+            "gpu_launches": 3 * args.steps,
+            "wall_s_timed_region": t_wall,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the kernels, from the committed ncu summary."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f)
+    return {}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=16384,
+                    help="query rows of the headline workload per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,145 @@
+/*
+ * attn.h -- C ABI of libattn_b200.so: fused grouped-KV scaled-dot-product
+ * attention forward on NVIDIA B200 (sm_100a).
+ *
+ * The operation (all entry points):
+ *   For batch b, query head h, query row i, with G = n_q / n_kv and the
+ *   key/value head g = floor(h / G):
+ *     s_j = scale * <q[b,h,i,:], k[b,g,j,:]>   for the visible keys j
+ *     O[b,h,i,:] = sum_j softmax_j(s) v[b,g,j,:]
+ *     LSE[b,h,i] = ln sum_j exp(s_j)          (natural log, scaled scores)
+ *   Sources: "Attention, Worked Out by Hand (Part 2)" (j33.ai), "The recap"
+ *   (score, scale, mask, softmax, mix); "Attention Engineering: From MHA to
+ *   GQA, MLA & FlashAttention" (arman1o1.github.io), section 2 (Grouped-Query
+ *   Attention Formulation: G query heads share one K/V head) and section 4
+ *   (the online-softmax recurrence and the per-row log-sum-exp L = m + log l);
+ *   "2.4 Multi-Head Attention, MQA, GQA & MLA" (llm-stack-book), "Implementing
+ *   the MHA -> GQA conversion" (query head j reads KV head j // n_rep).
+ *   MQA is n_kv = 1; MHA is n_kv = n_q.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers of the current CUDA device; the caller
+ *     owns and allocates every buffer (the library never allocates, frees or
+ *     keeps a pointer after the call returns).
+ *   - bf16 tensors are IEEE bfloat16 stored as 16-bit words; LSE is fp32.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; 0 is
+ *     the legacy default stream). Nothing on the hot path synchronises.
+ *   - Argument errors are returned synchronously and nothing is launched.
+ *     Errors found on the device (a bounded wait that expired, a seqlen out
+ *     of range) are recorded in a per-device status word that
+ *     attn_device_status() reads.
+ *   - Every base pointer must be 16-byte aligned and every row stride a
+ *     multiple of 8 elements (16 bytes): the kernels move tiles with the
+ *     Tensor Memory Accelerator, which requires it.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared here without the CUDA headers. */
+typedef struct CUstream_st *attn_stream_t;
+
+/* Status codes. */
+enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = -1,   /* null pointer, bad size, n_q % n_kv != 0, bad scale/causal */
+    ATTN_ERR_UNSUPPORTED = -2,   /* head dims outside the compiled set; causal with Sq > Skv */
+    ATTN_ERR_MISALIGNED = -3,    /* pointer not 16-byte aligned or stride not a multiple of 8 */
+    ATTN_ERR_WORKSPACE = -4,     /* workspace missing or smaller than attn_decode_workspace_bytes */
+    ATTN_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed (e.g. launch error) */
+    ATTN_ERR_DEVICE_TIMEOUT = -6,/* a kernel's bounded wait expired (reported by attn_device_status) */
+    ATTN_ERR_DEVICE_RANGE = -7   /* a device-side value (seqlens[b]) was out of range and clamped */
+};
+
+/*
+ * attn_fwd -- prefill / full forward.
+ *
+ *   q   [B, n_q,  Sq,  d_qk] bf16, contiguous (BHSD)
+ *   k   [B, n_kv, Skv, d_qk] bf16, contiguous
+ *   v   [B, n_kv, Skv, d_v ] bf16, contiguous
+ *   o   [B, n_q,  Sq,  d_v ] bf16, contiguous (written)
+ *   lse [B, n_q,  Sq]        fp32, contiguous (written; may be NULL to skip)
+ *   causal: 0 = every key visible; 1 = key j visible to query row i iff
+ *     j <= i + (Skv - Sq) (the query rows are the last Sq positions; for
+ *     Sq == Skv this is the usual lower-triangular mask).
+ *   scale: multiplies q.k before the softmax (finite, > 0; 1/sqrt(d_qk) is
+ *     the usual choice).
+ * Supported: d_qk == d_v in {32, 64, 128}; any B >= 0, Sq >= 0, Skv >= 1,
+ * any n_kv dividing n_q with n_q / n_kv a power of two <= 128; causal needs
+ * Sq <= Skv. Output rows are bf16 rounded to nearest even.
+ * Returns ATTN_OK or an error code (nothing launched on error).
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int Sq, int Skv, int n_q, int n_kv, int d_qk, int d_v,
+             int causal, float scale, attn_stream_t stream);
+
+/*
+ * attn_decode_workspace_bytes -- scratch size attn_decode needs for these
+ * sizes (split-KV partial outputs and their softmax statistics). Writes the
+ * byte count to *bytes. The same sizes always give the same answer.
+ */
+int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
+                                size_t *bytes);
+
+/*
+ * attn_decode -- one query token per sequence against a KV cache.
+ * Source: "Attention deep dive" (askaiml.pages.dev), section 5 (the KV cache:
+ * the new token's query against every cached key and value); "2.4 Multi-Head
+ * Attention, MQA, GQA & MLA", exercise decode_step (is_causal=False for the
+ * lone query: every cached key is visible).
+ *
+ *   q       [B, n_q, d_qk] bf16, contiguous
+ *   kcache  element (b, g, j, c) at kcache[b*k_stride_b + g*k_stride_h + j*k_stride_s + c]
+ *   vcache  element (b, g, j, c) at vcache[b*v_stride_b + g*v_stride_h + j*v_stride_s + c]
+ *           (strides in ELEMENTS; kcache and vcache may alias: the MLA latent
+ *           cache passes the same pointer, the 576-wide row as key and its
+ *           first 512 columns as value)
+ *   seqlens [B] int32: keys 0 .. seqlens[b]-1 of sequence b are visible
+ *           (values above S_max are clamped and reported as
+ *           ATTN_ERR_DEVICE_RANGE; 0 gives O = 0 and LSE = -inf)
+ *   o       [B, n_q, d_v] bf16 (written); lse [B, n_q] fp32 (written; may be NULL)
+ *   workspace: device scratch of at least attn_decode_workspace_bytes(...)
+ *           bytes, 256-byte aligned; its contents on entry do not matter.
+ *           Calls that share a workspace must be ordered on one stream.
+ * Supported: (d_qk, d_v) = (128, 128) with n_q / n_kv in {1, 2, 4, 8, 16, ...}
+ * (any power of two); (576, 512) with n_kv = 1 (MLA absorbed decode, the
+ * scale usually 1/sqrt(128 + 64)).
+ */
+int attn_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                void *o, float *lse,
+                int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
+                int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
+                float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/* Human-readable text of a status code (static storage). */
+const char *attn_status_string(int status);
+
+/*
+ * attn_device_status -- synchronise `stream`, then read and clear the status
+ * word of the current device. Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a
+ * kernel's bounded wait expired; its outputs are invalid), ATTN_ERR_DEVICE_RANGE,
+ * or ATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+int attn_device_status(attn_stream_t stream);
+
+/*
+ * attn_selftest_timeout -- launch one small kernel that waits, with the
+ * library's bounded-wait routine, on a barrier nothing will complete, giving
+ * up after `timeout_us` microseconds (1 .. 1000000). It must end with the
+ * status word set to ATTN_ERR_DEVICE_TIMEOUT: a test of the failure path that
+ * faults and hangs nothing.
+ */
+int attn_selftest_timeout(int timeout_us, attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -6,14 +6,12 @@ absorbed-latent decode), as sm_100a CUDA kernels behind a C ABI.
 The kernels are reached through ``mqa_attention_attn_b200.binding`` (loaded
 lazily; it raises if the CUDA library has not been built).
 """
-__all__ = ["inputs", "binding"]
+import importlib
+
+__all__ = ["inputs", "binding", "build"]
 
 
 def __getattr__(name):
-    if name == "binding":
-        from . import binding
-        return binding
-    if name == "inputs":
-        from . import inputs
-        return inputs
+    if name in __all__:
+        return importlib.import_module(f"{__name__}.{name}")
     raise AttributeError(name)

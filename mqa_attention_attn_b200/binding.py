@@ -1,0 +1,157 @@
+"""Python binding of libattn_b200.so (argument marshalling only).
+
+Every function here forwards torch tensors' device pointers and sizes to the
+C ABI declared in include/attn.h; all arithmetic runs in the library's CUDA
+kernels. There is no fallback: if the library is missing or a call fails, a
+RuntimeError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn_b200.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "attn.h")
+
+ATTN_OK = 0
+STATUS = {
+    0: "ATTN_OK", -1: "ATTN_ERR_INVALID_ARG", -2: "ATTN_ERR_UNSUPPORTED", -3: "ATTN_ERR_MISALIGNED",
+    -4: "ATTN_ERR_WORKSPACE", -5: "ATTN_ERR_CUDA", -6: "ATTN_ERR_DEVICE_TIMEOUT", -7: "ATTN_ERR_DEVICE_RANGE",
+}
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/attn.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(attn_\w+)\s*\(", text, flags=re.M)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library. Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} not built: run `python -m mqa_attention_attn_b200.build` "
+                               "(no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.attn_fwd.argtypes = [_vp] * 5 + [_i] * 8 + [ctypes.c_float, _vp]
+        L.attn_fwd.restype = _i
+        L.attn_decode_workspace_bytes.argtypes = [_i] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
+        L.attn_decode_workspace_bytes.restype = _i
+        L.attn_decode.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 +
+                                  [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_decode.restype = _i
+        L.attn_status_string.argtypes = [_i]
+        L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_device_status.argtypes = [_vp]
+        L.attn_device_status.restype = _i
+        L.attn_selftest_timeout.argtypes = [_i, _vp]
+        L.attn_selftest_timeout.restype = _i
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().attn_status_string(int(code)).decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(code: int, what: str):
+    if code != ATTN_OK:
+        raise AttnError(code, what)
+
+
+def attn_fwd(q, k, v, causal: bool, scale: float, o=None, lse=None, stream=None, want_lse=True):
+    """Prefill forward. q [B,n_q,Sq,d], k/v [B,n_kv,Skv,d] bf16 CUDA tensors
+    (contiguous). Returns (o [B,n_q,Sq,d] bf16, lse [B,n_q,Sq] fp32 or None)."""
+    B, n_q, Sq, d_qk = q.shape
+    _, n_kv, Skv, _ = k.shape
+    d_v = v.shape[3]
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if o is None:
+        o = torch.empty((B, n_q, Sq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Sq), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, n_q, n_kv, d_qk, d_v,
+                        int(bool(causal)), float(scale), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_fwd")
+    return o, lse
+
+
+def decode_workspace_bytes(B, n_q, n_kv, d_qk, d_v, S_max) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().attn_decode_workspace_bytes(B, n_q, n_kv, d_qk, d_v, S_max, ctypes.byref(out)),
+           "attn_decode_workspace_bytes")
+    return int(out.value)
+
+
+def _elem_strides(t):
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("cache must be 4-D [B, n_kv, S_max, row] with unit inner stride")
+    return t.stride(0), t.stride(1), t.stride(2)
+
+
+def attn_decode(q, kcache, vcache, seqlens, scale: float, d_v=None, o=None, lse=None, workspace=None,
+                stream=None, want_lse=True):
+    """Decode one query token per sequence. q [B,n_q,d_qk]; kcache/vcache
+    [B,n_kv,S_max,row] (any strides with a unit inner stride; they may be the
+    same tensor); seqlens int32 [B] on the device. Returns (o, lse)."""
+    B, n_q, d_qk = q.shape
+    _, n_kv, S_max, _ = kcache.shape
+    d_v = d_v or vcache.shape[3]
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    if seqlens.dtype != torch.int32 or not seqlens.is_cuda:
+        raise ValueError("seqlens must be an int32 CUDA tensor")
+    ks, vs = _elem_strides(kcache), _elem_strides(vcache)
+    if o is None:
+        o = torch.empty((B, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, n_q, n_kv, d_qk, d_v, S_max)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse),
+                           B, n_q, n_kv, d_qk, d_v, S_max, *ks, *vs, float(scale),
+                           _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_decode")
+    return o, lse
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream, read and clear the device status word."""
+    return int(lib().attn_device_status(ctypes.c_void_p(_stream(stream))))
+
+
+def selftest_timeout(timeout_us: int, stream=None):
+    _check(lib().attn_selftest_timeout(int(timeout_us), ctypes.c_void_p(_stream(stream))),
+           "attn_selftest_timeout")

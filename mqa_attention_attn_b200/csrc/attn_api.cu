@@ -1,0 +1,300 @@
+// attn_api.cu -- the C ABI of libattn_b200.so (declared in include/attn.h):
+// argument validation, TMA descriptor encoding and kernel launches.
+//
+// The library allocates nothing: every buffer (including the decode
+// workspace) belongs to the caller. Validation errors return before any
+// launch; device-side errors land in the status word that
+// attn_device_status() reads.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "decode_gqa.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using attn::g_status;
+
+// ---------------------------------------------------------------------------
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+CUtensorMapSwizzle swizzle_for(int row_bytes) {
+    return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                            : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// bf16 tensor map of rank `rank`: dims[0] is the contiguous one; strides in
+// bytes for dims 1..rank-1.
+bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
+              const uint32_t *box, int row_bytes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[5], gstr[4];
+    cuuint32_t bdim[5], estr[5];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+        estr[i] = 1;
+    }
+    for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr,
+                    bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(row_bytes),
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
+template <typename K>
+bool ensure_smem_attr(K kernel, size_t bytes, uint64_t &done_mask) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done_mask & bit) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    done_mask |= bit;
+    return true;
+}
+inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// ---------------------------------------------------------------------------
+// prefill
+// ---------------------------------------------------------------------------
+template <int D>
+int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,
+                   int n_q, int n_kv, int causal, float scale, cudaStream_t stream) {
+    using C = attn::pf::Cfg<D>;
+    const int G = n_q / n_kv;
+    attn::pf::Params p;
+    p.B = B;
+    p.Sq = Sq;
+    p.Skv = Skv;
+    p.n_q = n_q;
+    p.n_kv = n_kv;
+    p.G = G;
+    p.causal = causal;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.lse = lse;
+    if (G >= 2) {
+        p.Ht = G / 2;
+        p.Pt = 256 / G;
+        p.pair_by_heads = 1;
+        p.n_pb = (Sq + p.Pt - 1) / p.Pt;
+    } else {
+        p.Ht = 1;
+        p.Pt = 128;
+        p.pair_by_heads = 0;
+        p.n_pb = (Sq + 255) / 256;
+    }
+    CUtensorMap tq, tk, tv, to;
+    {
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * n_q};
+        const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
+        const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)p.Pt, (uint32_t)p.Ht};
+        if (!make_map(&tq, q, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+        if (!make_map(&to, o, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Skv, (uint64_t)B * n_kv};
+        const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Skv * D * 2};
+        const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)attn::pf::BN, 1u};
+        if (!make_map(&tk, k, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+        if (!make_map(&tv, v, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+    }
+    const size_t smem = attn::pf::smem_bytes<D>();
+    static uint64_t attr_done = 0;  // per template instance, one bit per device
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D>, smem, attr_done)) return ATTN_ERR_CUDA;
+    const long long grid = (long long)p.n_pb * B * n_kv;
+    if (grid <= 0) return ATTN_OK;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    attn::pf::prefill_kernel<D><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to, p);
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// decode (GQA, head dim 128)
+// ---------------------------------------------------------------------------
+inline int decode_n_splits(int S_max) { return (S_max + attn::dec::CH - 1) / attn::dec::CH; }
+
+size_t decode_ws_bytes(int B, int n_q, int d_v, int n_splits) {
+    const size_t rows = (size_t)B * n_q * n_splits;
+    size_t o_bytes = rows * d_v * sizeof(float);
+    o_bytes = (o_bytes + 255) & ~size_t(255);
+    return o_bytes + rows * sizeof(float2);
+}
+
+template <int GT>
+int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *o, float *lse,
+                      int B, int n_q, int n_kv, int S_max, const int64_t *ks, const int64_t *vs, float scale,
+                      void *ws, cudaStream_t stream) {
+    using namespace attn::dec;
+    const int G = n_q / n_kv;
+    const int n_hb = G / GT;
+    const int n_splits = decode_n_splits(S_max);
+    CUtensorMap tk, tv;
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S_max, (uint64_t)n_kv, (uint64_t)B};
+    const uint32_t box[4] = {64u, (uint32_t)KT, 1u, 1u};
+    const uint64_t kstr[3] = {(uint64_t)ks[2] * 2, (uint64_t)ks[1] * 2, (uint64_t)ks[0] * 2};
+    const uint64_t vstr[3] = {(uint64_t)vs[2] * 2, (uint64_t)vs[1] * 2, (uint64_t)vs[0] * 2};
+    if (!make_map(&tk, kc, 4, dims, kstr, box, 128)) return ATTN_ERR_CUDA;
+    if (!make_map(&tv, vc, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
+    const size_t smem = smem_bytes<GT>();
+    static uint64_t attr_done = 0;
+    if (!ensure_smem_attr(decode_split_kernel<GT>, smem, attr_done)) return ATTN_ERR_CUDA;
+    float *ws_o = reinterpret_cast<float *>(ws);
+    size_t o_bytes = (size_t)B * n_q * n_splits * D * sizeof(float);
+    o_bytes = (o_bytes + 255) & ~size_t(255);
+    float2 *ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(ws) + o_bytes);
+    const float scale_log2 = (float)((double)scale * 1.4426950408889634);
+    dim3 grid(n_splits, n_kv * n_hb, B);
+    decode_split_kernel<GT><<<grid, THREADS, smem, stream>>>(tk, tv, reinterpret_cast<const __nv_bfloat16 *>(q),
+                                                             seqlens, ws_o, ws_ml, n_q, G, n_hb, S_max, n_splits,
+                                                             scale_log2);
+    if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    decode_combine_kernel<<<dim3(n_q, B), 128, 0, stream>>>(ws_o, ws_ml, seqlens,
+                                                              reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q,
+                                                              n_splits, S_max, CH, D);
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        attn::mbar_init(attn::smem_u32(&bar), 1);
+        abort_flag = 0;
+        attn::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)  // nothing ever arrives on `bar`
+        attn::mbar_wait_slow(attn::smem_u32(&bar), 0, &abort_flag, 0x7e57, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv, int n_q,
+             int n_kv, int d_qk, int d_v, int causal, float scale, attn_stream_t stream) {
+    if (B < 0 || Sq < 0 || Skv < 1 || n_q < 1 || n_kv < 1 || d_qk < 1 || d_v < 1) return ATTN_ERR_INVALID_ARG;
+    if (n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || Sq == 0) return ATTN_OK;
+    if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+    if (d_qk != d_v || (d_qk != 32 && d_qk != 64 && d_qk != 128)) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G) || G > 256) return ATTN_ERR_UNSUPPORTED;
+    if (causal && Sq > Skv) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)B * n_q > 0x7fffffffLL || (long long)B * n_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (d_qk) {
+        case 32: return launch_prefill<32>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
+        case 64: return launch_prefill<64>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
+        default: return launch_prefill<128>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
+    }
+}
+
+int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, size_t *bytes) {
+    if (!bytes || B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!((d_qk == 128 && d_v == 128) || (d_qk == 576 && d_v == 512 && n_kv == 1))) return ATTN_ERR_UNSUPPORTED;
+    *bytes = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
+    return ATTN_OK;
+}
+
+int attn_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o, float *lse,
+                int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b, int64_t k_stride_h,
+                int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale,
+                void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+    if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0) return ATTN_OK;
+    if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (k_stride_b < 0 || k_stride_h < 0 || k_stride_s < 0 || v_stride_b < 0 || v_stride_h < 0 || v_stride_s < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (d_qk == 128 && d_v == 128) {
+        if (!is_pow2(G)) return ATTN_ERR_UNSUPPORTED;
+        if (k_stride_s < 128 || v_stride_s < 128) return ATTN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+        if ((k_stride_b | k_stride_h | k_stride_s | v_stride_b | v_stride_h | v_stride_s) & 7)
+            return ATTN_ERR_MISALIGNED;
+        const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
+        if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+        const int64_t ks[3] = {k_stride_b, k_stride_h, k_stride_s};
+        const int64_t vs[3] = {v_stride_b, v_stride_h, v_stride_s};
+        const int GT = G >= 8 ? 8 : G;
+        if ((long long)n_kv * (G / GT) > 65535) return ATTN_ERR_UNSUPPORTED;
+        switch (GT) {
+            case 1: return launch_decode_gqa<1>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
+            case 2: return launch_decode_gqa<2>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
+            case 4: return launch_decode_gqa<4>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
+            default: return launch_decode_gqa<8>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
+        }
+    }
+    if (d_qk == 576 && d_v == 512 && n_kv == 1) {
+        return ATTN_ERR_UNSUPPORTED;  // MLA decode kernel: not built yet
+    }
+    return ATTN_ERR_UNSUPPORTED;
+}
+
+const char *attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ATTN_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+        case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case ATTN_ERR_CUDA: return "CUDA error";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired on the device";
+        case ATTN_ERR_DEVICE_RANGE: return "a device-side value was out of range and clamped";
+        default: return "unknown status";
+    }
+}
+
+int attn_device_status(attn_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    unsigned int st = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&st, g_status, sizeof(st)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (st == 0) return ATTN_OK;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemcpyToSymbol(attn::g_timeout_site, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (st & attn::kStatusTimeout) return ATTN_ERR_DEVICE_TIMEOUT;
+    return ATTN_ERR_DEVICE_RANGE;
+}
+
+int attn_selftest_timeout(int timeout_us, attn_stream_t stream) {
+    if (timeout_us < 1 || timeout_us > 1000000) return ATTN_ERR_INVALID_ARG;
+    selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)timeout_us * 1000ull);
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

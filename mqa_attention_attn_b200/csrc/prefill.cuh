@@ -1,0 +1,411 @@
+// prefill.cuh -- fused tiled online-softmax attention forward (prefill) for
+// sm_100a: TMA-staged Q/K/V tiles, tcgen05 MMAs with TMEM accumulators.
+//
+// Work split. A CTA owns two 128-row query tiles of one (batch b, KV head g):
+//   * G = n_q/n_kv >= 2: each tile packs G/2 query heads x 256/G positions of
+//     the group, the two tiles being the two halves of the group's heads at
+//     the same positions. Every K/V tile is loaded once into shared memory and
+//     multiplied against all G heads of the group: the grouped broadcast of
+//     "Attention Engineering: From MHA to GQA, MLA & FlashAttention",
+//     section 2 (no repeat_interleave, K/V read once per group).
+//   * G = 1 (MHA): the two tiles are consecutive blocks of 128 positions.
+// Both tiles stream the same K/V tiles (128 keys each) through a 2-stage ring.
+//
+// Per K/V tile j and query tile t the recurrence of the same page, section 4
+// (FlashAttention-2 tiled rescaling) runs as:
+//   MMA warp:      S_t = Q_t K_j^T        (tcgen05, fp32 in TMEM)
+//   softmax WG t:  m' = max(m, rowmax S_t * scale*log2e)  (causal mask and
+//                  the key-count bound applied only on tiles that cross them)
+//                  P = 2^(S*scale*log2e - m') -> bf16 into TMEM over S_t
+//                  l' = l * 2^(m - m') + rowsum P ; O_t *= 2^(m - m')
+//   MMA warp:      O_t += P_t V_j         (A operand from TMEM)
+// with two refinements that keep the result exact:
+//   * the running maximum is only moved (and O rescaled) when the new tile
+//     raises it by more than 2^8; otherwise the stale maximum is kept, which
+//     bounds P by 256 and leaves O / l unchanged;
+//   * key tiles right of a tile's last causal row are never visited
+//     (causal tile skipping, "Attention, Worked Out by Hand (Part 2)",
+//     section 2).
+// The two query tiles ping-pong: while one softmax warpgroup exponentiates,
+// the tensor core runs the other tile's MMAs. Epilogue: O / l -> bf16 ->
+// swizzled shared memory -> TMA store; LSE = (m + log2 l) * ln 2.
+//
+// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 4-7 and 8-11 the softmax / epilogue warpgroups of tiles 0 and 1
+// (warp w reads TMEM lanes 32*(w%4) .. +31, so each warpgroup covers 128 rows).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+namespace pf {
+
+constexpr int BM = 128;        // query rows per tile (MMA M)
+constexpr int BN = 128;        // keys per K/V tile (MMA N of Q K^T)
+constexpr int NSTAGE = 2;
+constexpr int THREADS = 384;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only past a 256x growth
+
+template <int D>
+struct Cfg {
+    static constexpr int ROWB = (2 * D < 128) ? 2 * D : 128;   // bytes per shared row of one box
+    static constexpr int BOXD = ROWB / 2;                        // elements per box row
+    static constexpr int NBOX = D / BOXD;
+    static constexpr int SWB = ROWB == 128 ? 3 : (ROWB == 64 ? 2 : 1);
+    static constexpr uint32_t LAYOUT = ROWB == 128 ? 2u : (ROWB == 64 ? 4u : 6u);
+    static constexpr int QBYTES = BM * D * 2;
+    static constexpr int KBYTES = BN * D * 2;
+    static constexpr int QBOX = BM * ROWB;
+    static constexpr int KBOX = BN * ROWB;
+    static constexpr int ATOM = 8 * ROWB;                        // 8-row swizzle atom
+    static constexpr uint32_t TMEM_COLS = 512;
+    // TMEM columns: S (and P over its first half) of tile t, then O of tile t
+    __device__ static constexpr uint32_t col_s(int t) { return (uint32_t)t * 128u; }
+    __device__ static constexpr uint32_t col_o(int t) { return 256u + (uint32_t)t * (uint32_t)D; }
+    static_assert(D == 32 || D == 64 || D == 128, "head dim");
+};
+
+template <int D>
+struct Smem {
+    uint8_t q[2][Cfg<D>::QBYTES];          // Q tiles; reused as O staging in the epilogue
+    uint8_t k[NSTAGE][Cfg<D>::KBYTES];
+    uint8_t v[NSTAGE][Cfg<D>::KBYTES];
+    uint64_t q_full;
+    uint64_t kv_full[NSTAGE];
+    uint64_t kv_empty[NSTAGE];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_done[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+constexpr size_t smem_bytes() {
+    // at least ~116 KB so that one CTA (which takes all 512 TMEM columns)
+    // owns an SM
+    size_t s = sizeof(Smem<D>) + 1024;
+    return s < 118784 ? 118784 : s;
+}
+
+struct Params {
+    int B, Sq, Skv, n_q, n_kv, G;
+    int Ht, Pt;            // heads and positions per query tile (Ht * Pt = 128)
+    int pair_by_heads;     // 1: tiles = two head halves at one position block
+    int n_pb;              // position blocks per (b, kv head)
+    int causal;
+    float scale_log2;      // scale * log2(e)
+    float *lse;            // may be null
+};
+
+// All 32 lanes wait; the outcome is made warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t site) {
+    bool ok = mbar_wait(bar, parity, abort_flag, site);
+    ok = __all_sync(0xffffffffu, ok);
+    return ok;
+}
+
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    Smem<D> &sm = *reinterpret_cast<Smem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+
+    // ---- work unit: (b, kv head, position block), heaviest causal blocks first
+    const int nbh = p.B * p.n_kv;
+    const int bh = blockIdx.x % nbh;
+    const int pb = p.n_pb - 1 - (int)(blockIdx.x / nbh);
+    const int b = bh / p.n_kv, kvh = bh % p.n_kv;
+    int h0[2], p0[2], nt[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        if (p.pair_by_heads) {
+            h0[t] = kvh * p.G + t * p.Ht;
+            p0[t] = pb * p.Pt;
+        } else {
+            h0[t] = kvh;  // G == 1: query head == KV head
+            p0[t] = pb * 2 * p.Pt + t * p.Pt;
+        }
+        if (p0[t] >= p.Sq) {
+            nt[t] = 0;
+        } else {
+            const int last = min(p0[t] + p.Pt, p.Sq) - 1;
+            const int keys = p.causal ? min(p.Skv, last + (p.Skv - p.Sq) + 1) : p.Skv;
+            nt[t] = (keys + BN - 1) / BN;
+        }
+    }
+    const int nmax = max(nt[0], nt[1]);
+
+    // ---- setup: barriers (warp 0), TMEM (warp 1)
+    if (warp == 0 && lane == 0) {
+        mbar_init(smem_u32(&sm.q_full), 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(smem_u32(&sm.kv_full[s]), 1);
+            mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(smem_u32(&sm.s_full[t]), 1);
+            mbar_init(smem_u32(&sm.p_full[t]), 128);
+            mbar_init(smem_u32(&sm.o_done[t]), 1);
+        }
+        mbar_init(smem_u32(&sm.mma_done), 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&sm.tmem_base), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+
+    if (warp == 0) {
+        // ======================= TMA producer =======================
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_o);
+            uint32_t qbytes = 0;
+            for (int t = 0; t < 2; ++t)
+                if (nt[t] > 0) qbytes += C::QBYTES;
+            const uint32_t qbar = smem_u32(&sm.q_full);
+            mbar_arrive_expect_tx(qbar, qbytes);
+            for (int t = 0; t < 2; ++t) {
+                if (nt[t] == 0) continue;
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
+                                b * p.n_q + h0[t]);
+            }
+            int issued = 0;
+            for (int j = 0; j < nmax; ++j) {
+                const int s = j % NSTAGE;
+                if (j >= NSTAGE &&
+                    !mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / NSTAGE) + 1) & 1, abort_flag, 0x11))
+                    break;
+                const uint32_t fb = smem_u32(&sm.kv_full[s]);
+                mbar_arrive_expect_tx(fb, 2 * C::KBYTES);
+                for (int bx = 0; bx < C::NBOX; ++bx) {
+                    tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, j * BN,
+                                b * p.n_kv + kvh);
+                    tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, j * BN,
+                                b * p.n_kv + kvh);
+                }
+                ++issued;
+            }
+            // never leave copies in flight into this CTA's shared memory
+            mbar_wait(qbar, 0, nullptr, 0x12);
+            for (int j = issued - 1; j >= 0 && j >= issued - NSTAGE; --j)
+                mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x13);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ======================= MMA issuer =======================
+        if (lane == 0) {
+            const uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0, 0);
+            const uint32_t idesc_o = umma_idesc_bf16(BM, D, 0, 1);
+            bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x21);
+            auto issue_s = [&](int t, int j) {
+                const int s = j % NSTAGE;
+                const uint32_t qa = smem_u32(sm.q[t]);
+                const uint32_t ka = smem_u32(sm.k[s]);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int kel = ks * 16;
+                    const uint32_t off_q = (kel / C::BOXD) * C::QBOX + (kel % C::BOXD) * 2;
+                    const uint32_t off_k = (kel / C::BOXD) * C::KBOX + (kel % C::BOXD) * 2;
+                    const uint64_t ad = umma_smem_desc(qa + off_q, 16, C::ATOM, C::LAYOUT);
+                    const uint64_t bd = umma_smem_desc(ka + off_k, 16, C::ATOM, C::LAYOUT);
+                    umma_ss(tmem + C::col_s(t), ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&sm.s_full[t]));
+            };
+            auto issue_pv = [&](int t, int j) {
+                const int s = j % NSTAGE;
+                const uint32_t va = smem_u32(sm.v[s]);
+#pragma unroll
+                for (int ks = 0; ks < BN / 16; ++ks) {
+                    const uint64_t bd = umma_smem_desc(va + ks * 16 * C::ROWB, C::KBOX, C::ATOM, C::LAYOUT);
+                    umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + ks * 8, bd, idesc_o,
+                            (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&sm.o_done[t]));
+            };
+            if (ok && nmax > 0) {
+                ok = mbar_wait(smem_u32(&sm.kv_full[0]), 0, abort_flag, 0x22);
+                if (ok) {
+                    tc_fence_after();
+                    for (int t = 0; t < 2; ++t)
+                        if (nt[t] > 0) issue_s(t, 0);
+                }
+            }
+            for (int j = 0; ok && j < nmax; ++j) {
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j >= nt[t]) continue;
+                    ok = mbar_wait(smem_u32(&sm.p_full[t]), j & 1, abort_flag, 0x23);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(t, j);
+                    if (j + 1 < nt[t]) {
+                        ok = mbar_wait(smem_u32(&sm.kv_full[(j + 1) % NSTAGE]), ((j + 1) / NSTAGE) & 1,
+                                       abort_flag, 0x24);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(t, j + 1);
+                    }
+                }
+                umma_commit(smem_u32(&sm.kv_empty[j % NSTAGE]));
+            }
+            // all MMAs of this CTA done before TMEM can be released
+            umma_commit(smem_u32(&sm.mma_done));
+            mbar_wait(smem_u32(&sm.mma_done), 0, nullptr, 0x25);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ================== softmax + epilogue warpgroups ==================
+        const int t = (int)(warp - 4) / 4;
+        const uint32_t quad = warp & 3u;
+        const int r = (int)(quad * 32 + lane);          // row of the tile = TMEM lane
+        if (nt[t] > 0) {
+            const int hl = r / p.Pt, pl = r % p.Pt;
+            const int pos = p0[t] + pl;
+            const int head = h0[t] + hl;
+            int lim = p.causal ? pos + (p.Skv - p.Sq) : p.Skv - 1;   // last visible key
+            lim = min(lim, p.Skv - 1);
+            const uint32_t trow = tmem + ((quad * 32u) << 16);
+            const uint32_t colS = C::col_s(t), colO = C::col_o(t);
+            const float sl = p.scale_log2;
+            float m_run = -INFINITY, l_run = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nt[t]; ++j) {
+                ok = warp_wait(smem_u32(&sm.s_full[t]), j & 1, abort_flag, 0x31);
+                if (!ok) break;
+                __syncwarp();
+                tc_fence_after();
+                const int kbase = j * BN;
+                const bool need_mask = (kbase + BN - 1 > lim);
+                // pass 1: row maximum of this tile
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t x[32];
+                    tmem_ld32(trow + colS + 32 * c, x);
+                    tmem_wait_ld();
+                    const int rem = lim - (kbase + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float f = (need_mask && e > rem) ? -INFINITY : __uint_as_float(x[e]);
+                        mx = fmaxf(mx, f);
+                    }
+                }
+                const float m_new = fmaxf(m_run, mx * sl);
+                if (j == 0) {
+                    m_run = m_new;
+                } else {
+                    const bool need = m_new > m_run + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float alpha = ex2(m_run - m_new);
+                        ok = warp_wait(smem_u32(&sm.o_done[t]), (j - 1) & 1, abort_flag, 0x32);
+                        if (!ok) break;
+                        __syncwarp();
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(trow + colO + 32 * c, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st32(trow + colO + 32 * c, o);
+                        }
+                        tmem_wait_st();
+                        l_run *= alpha;
+                        m_run = m_new;
+                    }
+                }
+                // pass 2: P = 2^(s*scale*log2e - m) as bf16 over the first half of S
+                float rowsum = 0.f;
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t x[32];
+                    tmem_ld32(trow + colS + 32 * c, x);
+                    tmem_wait_ld();
+                    const int rem = lim - (kbase + 32 * c);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float s0 = __uint_as_float(x[2 * e]), s1 = __uint_as_float(x[2 * e + 1]);
+                        float p0v = ex2(fmaf(s0, sl, -m_run));
+                        float p1v = ex2(fmaf(s1, sl, -m_run));
+                        if (need_mask) {
+                            if (2 * e > rem) p0v = 0.f;
+                            if (2 * e + 1 > rem) p1v = 0.f;
+                        }
+                        rowsum += p0v + p1v;
+                        pk[e] = f2_to_bf2(p0v, p1v);
+                    }
+                    tmem_st16(trow + colS + 16 * c, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sm.p_full[t]));
+                l_run += rowsum;
+            }
+            // ---- epilogue: O / l -> bf16 -> swizzled smem -> TMA store; LSE
+            if (ok) ok = warp_wait(smem_u32(&sm.o_done[t]), (nt[t] - 1) & 1, abort_flag, 0x33);
+            __syncwarp();
+            tc_fence_after();
+            const float inv_l = 1.f / l_run;
+            const uint32_t stage = smem_u32(sm.q[t]);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(trow + colO + 32 * c, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {       // four 16-byte chunks of 8 values
+                    const int e0 = 32 * c + 8 * q4;     // first element of the chunk
+                    const int bx = e0 / C::BOXD;
+                    const int ci = (e0 % C::BOXD) / 8;
+                    uint4 w;
+                    w.x = f2_to_bf2(__uint_as_float(o[8 * q4 + 0]) * inv_l, __uint_as_float(o[8 * q4 + 1]) * inv_l);
+                    w.y = f2_to_bf2(__uint_as_float(o[8 * q4 + 2]) * inv_l, __uint_as_float(o[8 * q4 + 3]) * inv_l);
+                    w.z = f2_to_bf2(__uint_as_float(o[8 * q4 + 4]) * inv_l, __uint_as_float(o[8 * q4 + 5]) * inv_l);
+                    w.w = f2_to_bf2(__uint_as_float(o[8 * q4 + 6]) * inv_l, __uint_as_float(o[8 * q4 + 7]) * inv_l);
+                    sts128(stage + bx * C::QBOX + swz<C::SWB>((uint32_t)(r * C::ROWB + ci * 16)), w);
+                }
+            }
+            if (p.lse != nullptr && pos < p.Sq)
+                p.lse[((size_t)b * p.n_q + head) * p.Sq + pos] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+            fence_proxy_async_smem();
+            named_bar_sync(2 + t, 128);
+            if (r == 0 && ok) {
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_store_3d(&tm_o, stage + bx * C::QBOX, bx * C::BOXD, p0[t], b * p.n_q + h0[t]);
+                tma_store_commit();
+                tma_store_wait_read0();
+            }
+        }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace pf
+}  // namespace attn

@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every symbol include/attn.h declares;
+argument validation answers without a GPU (no compute call is made here)."""
+import ctypes
+
+import pytest
+
+from mqa_attention_attn_b200 import binding, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return binding.lib()
+
+
+def test_header_declares_the_boundary():
+    names = binding.header_functions()
+    for required in ("attn_fwd", "attn_decode", "attn_decode_workspace_bytes", "attn_status_string",
+                     "attn_device_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in binding.header_functions():
+        assert hasattr(lib, name), f"{name} declared in include/attn.h but not exported"
+
+
+def test_status_strings(lib):
+    for code in range(0, -8, -1):
+        assert binding.status_string(code) not in ("", "unknown status")
+    assert binding.status_string(-99) == "unknown status"
+
+
+def test_validation_rejects_before_any_launch(lib):
+    vp = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    # n_q % n_kv != 0
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 6, 4, 64, 64, 1, 0.1, None) == -1
+    # causal must be 0 or 1
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 2, 0.1, None) == -1
+    # non-finite / non-positive scale
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 1, float("inf"), None) == -1
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 1, -1.0, None) == -1
+    # Skv = 0
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 0, 4, 2, 64, 64, 0, 0.1, None) == -1
+    # null pointers
+    assert lib.attn_fwd(None, vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 1, 0.1, None) == -1
+    # head dim outside the compiled set, d_qk != d_v
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 96, 96, 1, 0.1, None) == -2
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 128, 64, 1, 0.1, None) == -2
+    # group size not a power of two
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 8, 8, 6, 2, 64, 64, 1, 0.1, None) == -2
+    # causal with Sq > Skv
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 9, 8, 4, 2, 64, 64, 1, 0.1, None) == -2
+    # misaligned pointer
+    assert lib.attn_fwd(ctypes.c_void_p(18), vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 1, 0.1, None) == -3
+    # empty batch / no query rows: nothing to do
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 0, 8, 8, 4, 2, 64, 64, 1, 0.1, None) == 0
+    assert lib.attn_fwd(vp, vp, vp, vp, None, 1, 0, 8, 4, 2, 64, 64, 1, 0.1, None) == 0
+
+
+def test_decode_validation(lib):
+    vp = ctypes.c_void_p(256)
+    out = ctypes.c_size_t(0)
+    assert lib.attn_decode_workspace_bytes(32, 32, 8, 128, 128, 32768, ctypes.byref(out)) == 0
+    # partial outputs (fp32, 128 wide) + (m, l) per (b, h, chunk of 512 keys)
+    assert out.value == 32 * 32 * 64 * 128 * 4 + 32 * 32 * 64 * 8
+    assert lib.attn_decode_workspace_bytes(32, 32, 8, 96, 96, 4096, ctypes.byref(out)) == -2
+    args = dict(B=2, n_q=8, n_kv=2, d_qk=128, d_v=128, S_max=1024)
+    need = ctypes.c_size_t(0)
+    lib.attn_decode_workspace_bytes(2, 8, 2, 128, 128, 1024, ctypes.byref(need))
+
+    def call(ws_bytes=need.value, ws=vp, n_q=8, n_kv=2, d_qk=128, d_v=128, k_s=(8 * 1024 * 128, 1024 * 128, 128)):
+        return lib.attn_decode(vp, vp, vp, vp, vp, vp, 2, n_q, n_kv, d_qk, d_v, 1024, *k_s, *k_s, 0.1, ws,
+                               ws_bytes, None)
+    assert call(ws_bytes=need.value - 1) == -4          # workspace too small
+    assert call(ws=None) == -4                          # no workspace
+    assert call(ws=ctypes.c_void_p(272)) == -3          # workspace not 256-byte aligned
+    assert call(n_q=7) == -1                            # n_q % n_kv != 0
+    assert call(d_qk=64, d_v=64) == -2                  # not a compiled decode shape
+    assert call(k_s=(8 * 1024 * 128, 1024 * 128, 130)) == -3   # row stride not a multiple of 8

@@ -1,0 +1,138 @@
+"""attn_decode (single-token decode against a KV cache) on the GPU against the
+fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import check_parity, need_gpu
+from mqa_attention_attn_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode_and_check(seqlens, q, kc, vc, scale, what, d_v=None):
+    binding = need_gpu()
+    sl = seqlens.to("cuda")
+    o, lse = binding.attn_decode(q, kc, vc, sl, scale, d_v=d_v)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    B, n_q, d_qk = q.shape
+    o_ref, lse_ref = oracle.sdpa(q[:, :, None, :], kc, vc, False, scale, seqlens=seqlens.numpy(),
+                                 d_v=d_v)
+    check_parity(o, lse, o_ref[:, :, 0], lse_ref[:, :, 0], what)
+    return o, lse
+
+
+@pytest.mark.parametrize("B,n_q,n_kv,S_max,seqlens", [
+    (3, 8, 2, 1100, [1, 700, 1100]),        # G=4, ragged, 1..3 chunks
+    (2, 32, 8, 2048, [2048, 1537]),         # Llama-3-8B heads
+    (2, 4, 4, 600, [513, 64]),              # MHA (G=1)
+    (1, 16, 8, 300, [300]),                 # G=2
+    (2, 64, 8, 900, [899, 1]),              # G=8
+    (1, 32, 2, 1030, [1030]),               # G=16 (two head blocks)
+    (2, 32, 1, 700, [700, 65]),             # MQA, G=32 (four head blocks)
+])
+def test_decode_shapes(B, n_q, n_kv, S_max, seqlens):
+    seq = torch.tensor(seqlens, dtype=torch.int32)
+    g = torch.Generator(device="cuda").manual_seed(B * 1000 + n_q + S_max)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    _decode_and_check(seq, q, kc, vc, 1 / math.sqrt(128), f"decode {B} {n_q}/{n_kv} {S_max}")
+
+
+def test_decode_strided_cache():
+    """A cache stored [B, S_max, n_kv, d] (token-major) passed through strides."""
+    B, n_q, n_kv, S_max = 2, 16, 4, 1500
+    seq = torch.tensor([1500, 999], dtype=torch.int32)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kb = torch.randn(B, S_max, n_kv, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vb = torch.randn(B, S_max, n_kv, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc, vc = kb.permute(0, 2, 1, 3), vb.permute(0, 2, 1, 3)      # views, not copies
+    _decode_and_check(seq, q, kc, vc, 0.1, "strided cache")
+
+
+def test_gqa_decode_workload_full():
+    """The GQA decode workload at full size (B=32, cache lengths ~U[1024, 32768],
+    32/8 heads): every (b, h) output row against the oracle."""
+    binding = need_gpu()
+    w = inputs.WORKLOADS["gqa_decode"]
+    seqlens, q, kc, vc = inputs.make(w, device="cuda")
+    o, lse = binding.attn_decode(q, kc, vc, seqlens.cuda(), w.scale)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    o_ref = np.zeros((w.B, w.n_q, w.d_v))
+    l_ref = np.zeros((w.B, w.n_q))
+    for b in range(w.B):
+        L = int(seqlens[b])
+        ob, lb = oracle.sdpa(q[b:b + 1, :, None, :], kc[b:b + 1, :, :L], vc[b:b + 1, :, :L], False, w.scale)
+        o_ref[b], l_ref[b] = ob[0, :, 0], lb[0, :, 0]
+    check_parity(o, lse, o_ref, l_ref, "gqa_decode")
+
+
+def test_decode_equals_last_prefill_row():
+    """Decode of token L-1 against a cache of L tokens == row L-1 of causal prefill."""
+    binding = need_gpu()
+    n_q, n_kv, L = 32, 8, 1234
+    q, k, v = inputs.prefill_inputs(1, L, L, n_q, n_kv, 128, 128, 21, device="cuda")
+    o_p, l_p = binding.attn_fwd(q, k, v, True, 0.08)
+    o_d, l_d = binding.attn_decode(q[:, :, L - 1].contiguous(), k, v,
+                                   torch.tensor([L], dtype=torch.int32, device="cuda"), 0.08)
+    assert (o_p[:, :, L - 1].float() - o_d.float()).abs().max() <= 2e-2
+    assert (l_p[:, :, L - 1] - l_d).abs().max() <= 1e-3
+
+
+def test_decode_zero_length_and_range_status():
+    binding = need_gpu()
+    B, n_q, n_kv, S_max = 3, 8, 2, 256
+    g = torch.Generator(device="cuda").manual_seed(6)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    seq = torch.tensor([0, 100, 1000], dtype=torch.int32, device="cuda")   # 1000 > S_max: clamped
+    o, lse = binding.attn_decode(q, kc, vc, seq, 0.1)
+    assert binding.device_status() == -7                                     # ATTN_ERR_DEVICE_RANGE
+    assert binding.device_status() == 0                                      # cleared by the read
+    assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    o_ref, l_ref = oracle.sdpa(q[:, :, None, :], kc, vc, False, 0.1,
+                               seqlens=np.array([0, 100, 256], np.int32))
+    check_parity(o, lse, o_ref[:, :, 0], l_ref[:, :, 0], "zero/clamped lengths")
+
+
+def test_decode_workspace_checks():
+    binding = need_gpu()
+    B, n_q, n_kv, S_max = 2, 8, 2, 1024
+    q = torch.zeros(B, n_q, 128, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(B, n_kv, S_max, 128, dtype=torch.bfloat16, device="cuda")
+    seq = torch.tensor([5, 6], dtype=torch.int32, device="cuda")
+    need = binding.decode_workspace_bytes(B, n_q, n_kv, 128, 128, S_max)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(binding.AttnError) as e:
+        binding.attn_decode(q, kc, kc, seq, 0.1, workspace=ws)
+    assert e.value.code == -4
+
+
+def test_decode_deterministic():
+    binding = need_gpu()
+    w = inputs.WORKLOADS["gqa_decode"]
+    seqlens, q, kc, vc = inputs.decode_inputs(4, 32, 8, 128, 128, 8192, (1, 8192), 31, device="cuda")
+    sl = seqlens.cuda()
+    o1, l1 = binding.attn_decode(q, kc, vc, sl, w.scale)
+    for _ in range(5):
+        o2, l2 = binding.attn_decode(q, kc, vc, sl, w.scale)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_timeout_path_reports_status():
+    """A bounded wait that nothing completes ends with ATTN_ERR_DEVICE_TIMEOUT
+    and leaves the context usable."""
+    binding = need_gpu()
+    binding.selftest_timeout(20000)
+    assert binding.device_status() == -6
+    assert binding.device_status() == 0
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum()) == 8.0
