@@ -262,20 +262,26 @@ def run_ours(args):
     by_d = decode_bytes(wd, seqlens)
     fl_d = decode_flops(wd, seqlens)
 
+    do_p = args.only in ("all", "prefill")
+    do_d = args.only in ("all", "decode")
+
     def step(times_p, times_d):
-        flush.fill_(1.0)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        binding.attn_fwd(q, k, v, w.causal, w.scale, o=o, lse=lse, stream=stream)
-        e1.record(stream)
-        flush.fill_(2.0)
-        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e2.record(stream)
-        binding.attn_decode(qd, kc, vc, sl_dev, wd.scale, o=od, lse=ld, workspace=work, stream=stream)
-        e3.record(stream)
-        if times_p is not None:
-            times_p.append((e0, e1))
-            times_d.append((e2, e3))
+        if do_p:
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binding.attn_fwd(q, k, v, w.causal, w.scale, o=o, lse=lse, stream=stream)
+            e1.record(stream)
+            if times_p is not None:
+                times_p.append((e0, e1))
+        if do_d:
+            flush.fill_(2.0)
+            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e2.record(stream)
+            binding.attn_decode(qd, kc, vc, sl_dev, wd.scale, o=od, lse=ld, workspace=work, stream=stream)
+            e3.record(stream)
+            if times_d is not None:
+                times_d.append((e2, e3))
 
     def barrier():
         if ws > 1:
@@ -298,8 +304,8 @@ def run_ours(args):
         t_wall = time.perf_counter() - t_wall0
     st = binding.device_status(stream)
     assert st == 0, f"device status {st}"
-    ms_p = [a.elapsed_time(b) for a, b in tp]
-    ms_d = [a.elapsed_time(b) for a, b in td]
+    ms_p = [a.elapsed_time(b) for a, b in tp] or [float("nan")]
+    ms_d = [a.elapsed_time(b) for a, b in td] or [float("nan")]
     mean_p = sum(ms_p) / len(ms_p)
     mean_d = sum(ms_d) / len(ms_d)
 
@@ -310,7 +316,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and do_p:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
@@ -362,7 +368,7 @@ def run_ours(args):
     }
 
     cpu_baseline = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and do_p:
         qc, kc_, vc_ = q.cpu(), k.cpu(), v.cpu()
         dt, fl, threads = oracle_full(w, qc, kc_, vc_)
         cpu_baseline = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -383,7 +389,7 @@ def run_ours(args):
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
             "clocks": clocks.summary(),
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (int(do_p) + 2 * int(do_d)) * args.steps,
             "wall_s_timed_region": t_wall,
         }
         print(json.dumps(line), flush=True)
@@ -412,6 +418,8 @@ def main():
                     help="query rows of the headline workload per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+                    help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
