@@ -118,6 +118,44 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
                 int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
                 float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
+/*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
+ * memory.
+ *
+ * This entry point has no counterpart in the pages the method comes from; it
+ * exists for the library's users. Some callers of a decode step cannot call
+ * cudaMalloc or any allocator: a plugin running inside another framework that
+ * owns every device allocation, a real-time serving loop that must not take
+ * the allocator's locks or implicit synchronisation, or host code that has no
+ * device allocator at all. They cannot provide attn_decode's workspace, so this
+ * variant uses a scratch array that the library itself holds in device memory
+ * (a file-scope __device__ array of ATTN_NOALLOC_SCRATCH_BYTES bytes, present
+ * on every GPU that loads the library until the process exits).
+ *
+ * Arguments and results are those of attn_decode without the workspace.
+ * Sizes whose scratch need (attn_decode_workspace_bytes) exceeds
+ * ATTN_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_WORKSPACE, before
+ * anything is launched. Supported shapes: the (128, 128) head dims of
+ * attn_decode.
+ *
+ * The first call on a device looks up that device's address of the scratch
+ * array (cudaGetSymbolAddress); make that first call before any stream
+ * capture on the device. Nothing is allocated or freed, then or later.
+ * All calls share the one array and it keeps the previous call's contents;
+ * no part of it needs to start at zero (every value read is written earlier
+ * in the same call). Calls that overlap on the GPU (on different streams, or
+ * from several host threads without ordering) race on the array: order them
+ * on one stream.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (36u * 1024u * 1024u)
+
+int attn_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                        void *o, float *lse,
+                        int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
+                        int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                        int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
+                        float scale, attn_stream_t stream);
+
 /* Human-readable text of a status code (static storage). */
 const char *attn_status_string(int status);
 

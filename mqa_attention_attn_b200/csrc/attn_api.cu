@@ -298,3 +298,51 @@ int attn_selftest_timeout(int timeout_us, attn_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_decode_noalloc: the decode step for callers that cannot allocate.
+//
+// Its split-KV scratch (partial outputs and their softmax statistics) lives
+// in the file-scope array below instead of a caller-provided workspace. In
+// host code `g_noalloc_scratch` names only a host-side stand-in, so the
+// device address is looked up once per device with cudaGetSymbolAddress
+// (with that device current) and passed to the kernels.
+// ---------------------------------------------------------------------------
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device (first call on
+// a device does the lookup). Returns nullptr on failure.
+void *noalloc_scratch_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int attn_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                                   void *o, float *lse, int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
+                                   int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                                   int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale,
+                                   attn_stream_t stream) {
+    if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (B == 0) return ATTN_OK;
+    if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
+    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
+    if (need > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;  // beyond the static maximum
+    void *scratch = noalloc_scratch_ptr();
+    if (scratch == nullptr) return ATTN_ERR_CUDA;
+    return attn_decode(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, d_qk, d_v, S_max, k_stride_b, k_stride_h,
+                       k_stride_s, v_stride_b, v_stride_h, v_stride_s, scale, scratch, need, stream);
+}
