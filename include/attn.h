@@ -176,6 +176,15 @@ int attn_device_status(attn_stream_t stream);
  */
 int attn_selftest_timeout(int timeout_us, attn_stream_t stream);
 
+/*
+ * attn_selftest_ex2 -- evaluate, for n device floats x, the two base-2
+ * exponentials the prefill softmax uses: y_poly = the FMA-pipe evaluation
+ * (range reduction + a cubic fitted for relative error, inputs clamped at
+ * -125) and y_sfu = the special-function unit's ex2.approx. For tests of the
+ * kernels' exponential accuracy.
+ */
+int attn_selftest_ex2(const float *x, float *y_poly, float *y_sfu, int n, attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.attn_device_status.restype = _i
         L.attn_selftest_timeout.argtypes = [_i, _vp]
         L.attn_selftest_timeout.restype = _i
+        L.attn_selftest_ex2.argtypes = [_vp, _vp, _vp, _i, _vp]
+        L.attn_selftest_ex2.restype = _i
         _lib = L
     return _lib
 
@@ -155,3 +157,13 @@ def device_status(stream=None) -> int:
 def selftest_timeout(timeout_us: int, stream=None):
     _check(lib().attn_selftest_timeout(int(timeout_us), ctypes.c_void_p(_stream(stream))),
            "attn_selftest_timeout")
+
+
+def selftest_ex2(x, stream=None):
+    """(poly, sfu) base-2 exponentials of a float32 CUDA tensor x, as the
+    prefill softmax evaluates them."""
+    x = x.contiguous()
+    yp, ys = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().attn_selftest_ex2(_ptr(x), _ptr(yp), _ptr(ys), x.numel(), ctypes.c_void_p(_stream(stream))),
+           "attn_selftest_ex2")
+    return yp, ys

@@ -127,6 +127,16 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     const size_t smem = attn::pf::smem_bytes<D>();
     static uint64_t attr_done = 0;  // per template instance, one bit per device
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D>, smem, attr_done)) return ATTN_ERR_CUDA;
+    // The kernel rebalances registers between warpgroups (setmaxnreg); that is
+    // only safe if it was built with exactly the register count the split
+    // assumes, otherwise the increase could never be granted.
+    static int regs_checked = 0;
+    if (regs_checked == 0) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D>) != cudaSuccess) return ATTN_ERR_CUDA;
+        regs_checked = (fa.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
+    }
+    if (regs_checked < 0) return ATTN_ERR_UNSUPPORTED;
     const long long grid = (long long)p.n_pb * B * n_kv;
     if (grid <= 0) return ATTN_OK;
     if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
@@ -191,6 +201,19 @@ __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
     __syncthreads();
     if (threadIdx.x == 0)  // nothing ever arrives on `bar`
         attn::mbar_wait_slow(attn::smem_u32(&bar), 0, &abort_flag, 0x7e57, limit_ns);
+}
+
+__global__ void selftest_ex2_kernel(const float *x, float *y_poly, float *y_sfu, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+    const float2 p = attn::ex2_poly2(make_float2(a, b));
+    y_poly[i] = p.x;
+    y_sfu[i] = attn::ex2(a);
+    if (i + 1 < n) {
+        y_poly[i + 1] = p.y;
+        y_sfu[i + 1] = attn::ex2(b);
+    }
 }
 
 }  // namespace
@@ -288,6 +311,15 @@ int attn_device_status(attn_stream_t stream) {
     if (cudaMemcpyToSymbol(attn::g_timeout_site, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
     if (st & attn::kStatusTimeout) return ATTN_ERR_DEVICE_TIMEOUT;
     return ATTN_ERR_DEVICE_RANGE;
+}
+
+int attn_selftest_ex2(const float *x, float *y_poly, float *y_sfu, int n, attn_stream_t stream) {
+    if (n < 0 || (n > 0 && (!x || !y_poly || !y_sfu))) return ATTN_ERR_INVALID_ARG;
+    if (n == 0) return ATTN_OK;
+    const int pairs = (n + 1) / 2;
+    selftest_ex2_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y_poly, y_sfu,
+                                                                                                n);
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_selftest_timeout(int timeout_us, attn_stream_t stream) {

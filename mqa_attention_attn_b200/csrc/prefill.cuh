@@ -45,6 +45,22 @@ constexpr int BN = 128;        // keys per K/V tile (MMA N of Q K^T)
 constexpr int NSTAGE = 2;
 constexpr int THREADS = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only past a 256x growth
+#ifndef ATTN_PF_P_CHUNKS
+#define ATTN_PF_P_CHUNKS 2
+#endif
+#ifndef ATTN_PF_POLY_EVERY
+#define ATTN_PF_POLY_EVERY 0
+#endif
+// P is handed to the MMA warp in kPChunks pieces of the 128 keys; every
+// kPolyEvery-th exponential pair runs on the FMA pipe (0: none).
+constexpr int kPChunks = ATTN_PF_P_CHUNKS;
+constexpr int kPolyEvery = ATTN_PF_POLY_EVERY;
+constexpr int kChunkKeys = BN / kPChunks;
+static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P hand-off chunks");
+constexpr int kLaunchRegs = 168;            // registers per thread the kernel must be built with
+constexpr int kRegsLow = 56;               // producer / MMA warpgroup after setmaxnreg.dec
+constexpr int kRegsHigh = 224;              // softmax warpgroups after setmaxnreg.inc
+static_assert(kRegsLow * 128 + kRegsHigh * 256 <= kLaunchRegs * THREADS, "register split exceeds the block");
 
 template <int D>
 struct Cfg {
@@ -74,7 +90,7 @@ struct Smem {
     uint64_t kv_full[NSTAGE];
     uint64_t kv_empty[NSTAGE];
     uint64_t s_full[2];
-    uint64_t p_full[2];
+    uint64_t p_full[2][kPChunks];  // one per hand-off chunk of P
     uint64_t o_done[2];
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -152,7 +168,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&sm.s_full[t]), 1);
-            mbar_init(smem_u32(&sm.p_full[t]), 128);
+            for (int c = 0; c < kPChunks; ++c) mbar_init(smem_u32(&sm.p_full[t][c]), 128);
             mbar_init(smem_u32(&sm.o_done[t]), 1);
         }
         mbar_init(smem_u32(&sm.mma_done), 1);
@@ -169,6 +185,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
 
+    // Register split: the producer / MMA warpgroup needs few registers, the
+    // softmax warpgroups hold a 128-key row of S each. 56*128 + 224*256 =
+    // 168*384, the block's registers at launch (the host refuses to launch
+    // unless the kernel was built with exactly kLaunchRegs per thread).
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
         // ======================= TMA producer =======================
         if (lane == 0) {
@@ -230,16 +252,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 umma_commit(smem_u32(&sm.s_full[t]));
             };
-            auto issue_pv = [&](int t, int j) {
+            // O_t += P_t V_j, 32 keys at a time as soon as the softmax
+            // warpgroup has written that chunk of P
+            auto issue_pv = [&](int t, int j) -> bool {
                 const int s = j % NSTAGE;
                 const uint32_t va = smem_u32(sm.v[s]);
 #pragma unroll
-                for (int ks = 0; ks < BN / 16; ++ks) {
-                    const uint64_t bd = umma_smem_desc(va + ks * 16 * C::ROWB, C::KBOX, C::ATOM, C::LAYOUT);
-                    umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + ks * 8, bd, idesc_o,
-                            (j > 0 || ks > 0) ? 1u : 0u);
+                for (int c = 0; c < kPChunks; ++c) {
+                    if (!mbar_wait(smem_u32(&sm.p_full[t][c]), j & 1, abort_flag, 0x23)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kChunkKeys / 16; ++kk) {
+                        const int ks = c * (kChunkKeys / 16) + kk;
+                        const uint64_t bd = umma_smem_desc(va + ks * 16 * C::ROWB, C::KBOX, C::ATOM, C::LAYOUT);
+                        umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + ks * 8, bd, idesc_o,
+                                (j > 0 || ks > 0) ? 1u : 0u);
+                    }
                 }
                 umma_commit(smem_u32(&sm.o_done[t]));
+                return true;
             };
             if (ok && nmax > 0) {
                 ok = mbar_wait(smem_u32(&sm.kv_full[0]), 0, abort_flag, 0x22);
@@ -252,10 +283,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int j = 0; ok && j < nmax; ++j) {
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j >= nt[t]) continue;
-                    ok = mbar_wait(smem_u32(&sm.p_full[t]), j & 1, abort_flag, 0x23);
+                    ok = issue_pv(t, j);
                     if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(t, j);
                     if (j + 1 < nt[t]) {
                         ok = mbar_wait(smem_u32(&sm.kv_full[(j + 1) % NSTAGE]), ((j + 1) / NSTAGE) & 1,
                                        abort_flag, 0x24);
@@ -271,7 +300,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_wait(smem_u32(&sm.mma_done), 0, nullptr, 0x25);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
         // ================== softmax + epilogue warpgroups ==================
         const int t = (int)(warp - 4) / 4;
         const uint32_t quad = warp & 3u;
@@ -287,79 +318,95 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float sl = p.scale_log2;
             float m_run = -INFINITY, l_run = 0.f;
             bool ok = true;
-            for (int j = 0; j < nt[t]; ++j) {
+            const int ntt = nt[t];
+            const float2 sl2 = make_float2(sl, sl);
+            for (int j = 0; j < ntt; ++j) {
                 ok = warp_wait(smem_u32(&sm.s_full[t]), j & 1, abort_flag, 0x31);
                 if (!ok) break;
                 __syncwarp();
                 tc_fence_after();
+                // the whole 128-key row of S in registers (four loads, one wait)
+                uint32_t x[BN];
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c)
+                    tmem_ld32(trow + colS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
+                tmem_wait_ld();
                 const int kbase = j * BN;
-                const bool need_mask = (kbase + BN - 1 > lim);
-                // pass 1: row maximum of this tile
-                float mx = -INFINITY;
+                // causal / key-count mask: only on tiles that cross some row's limit
+                const bool masked = __any_sync(0xffffffffu, kbase + BN - 1 > lim);
+                if (masked) {
+                    const int rem = lim - kbase;
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t x[32];
-                    tmem_ld32(trow + colS + 32 * c, x);
-                    tmem_wait_ld();
-                    const int rem = lim - (kbase + 32 * c);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float f = (need_mask && e > rem) ? -INFINITY : __uint_as_float(x[e]);
-                        mx = fmaxf(mx, f);
-                    }
+                    for (int e = 0; e < BN; ++e)
+                        if (e > rem) x[e] = 0xff800000u;   // -inf
                 }
+                // row maximum (four independent 3-input max chains)
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < BN; e += 8) {
+                    mx0 = fmax3(mx0, __uint_as_float(x[e + 0]), __uint_as_float(x[e + 1]));
+                    mx1 = fmax3(mx1, __uint_as_float(x[e + 2]), __uint_as_float(x[e + 3]));
+                    mx2 = fmax3(mx2, __uint_as_float(x[e + 4]), __uint_as_float(x[e + 5]));
+                    mx3 = fmax3(mx3, __uint_as_float(x[e + 6]), __uint_as_float(x[e + 7]));
+                }
+                const float mx = fmaxf(fmax3(mx0, mx1, mx2), mx3);
                 const float m_new = fmaxf(m_run, mx * sl);
                 if (j == 0) {
                     m_run = m_new;
-                } else {
-                    const bool need = m_new > m_run + kRescaleThreshold;
-                    if (__any_sync(0xffffffffu, need)) {
-                        const float alpha = ex2(m_run - m_new);
-                        ok = warp_wait(smem_u32(&sm.o_done[t]), (j - 1) & 1, abort_flag, 0x32);
-                        if (!ok) break;
-                        __syncwarp();
-                        tc_fence_after();
+                } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold)) {
+                    // move the running maximum: rescale this row's O and l
+                    // O is stable here: s_full for tile j was committed after
+                    // the P.V MMA of tile j-1, and a commit tracks every MMA
+                    // issued before it.
+                    const float alpha = ex2(m_run - m_new);
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(trow + colO + 32 * c, o);
-                            tmem_wait_ld();
+                    for (int c = 0; c < D / 32; ++c) {   // 32 columns at a time: S stays in registers
+                        uint32_t o[32];
+                        tmem_ld32(trow + colO + 32 * c, o);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                            tmem_st32(trow + colO + 32 * c, o);
-                        }
-                        tmem_wait_st();
-                        l_run *= alpha;
-                        m_run = m_new;
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(trow + colO + 32 * c, o);
                     }
+                    tmem_wait_st();
+                    l_run *= alpha;
+                    m_run = m_new;
                 }
-                // pass 2: P = 2^(s*scale*log2e - m) as bf16 over the first half of S
-                float rowsum = 0.f;
+                // P = 2^(s*scale*log2e - m) -> bf16 pairs over the first half of S,
+                // handed to the MMA warp in kPChunks pieces so that P.V starts on
+                // the first keys while later ones are still exponentiated.
+                // Optionally (kPolyEvery > 0) part of the exponentials run on the
+                // FMA pipe (ex2_poly2) beside the special-function unit; measured
+                // on B200 this is slower for head dim 128 (the softmax is bound
+                // by issue and latency, not by the special-function unit), so it
+                // is off by default.
+                const float2 nm2 = make_float2(-m_run, -m_run);
+                float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t x[32];
-                    tmem_ld32(trow + colS + 32 * c, x);
-                    tmem_wait_ld();
-                    const int rem = lim - (kbase + 32 * c);
-                    uint32_t pk[16];
+                for (int c = 0; c < kPChunks; ++c) {
+                    uint32_t pk[kChunkKeys / 2];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float s0 = __uint_as_float(x[2 * e]), s1 = __uint_as_float(x[2 * e + 1]);
-                        float p0v = ex2(fmaf(s0, sl, -m_run));
-                        float p1v = ex2(fmaf(s1, sl, -m_run));
-                        if (need_mask) {
-                            if (2 * e > rem) p0v = 0.f;
-                            if (2 * e + 1 > rem) p1v = 0.f;
-                        }
-                        rowsum += p0v + p1v;
-                        pk[e] = f2_to_bf2(p0v, p1v);
+                    for (int e = 0; e < kChunkKeys / 2; ++e) {
+                        const int i0 = c * kChunkKeys + 2 * e;
+                        const float2 t2 = ffma2(make_float2(__uint_as_float(x[i0]), __uint_as_float(x[i0 + 1])),
+                                                sl2, nm2);
+                        const bool poly = kPolyEvery > 0 && !masked && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) ==
+                                                                         (kPolyEvery > 0 ? kPolyEvery - 1 : 0);
+                        const float2 pe = poly ? ex2_poly2(t2) : make_float2(ex2(t2.x), ex2(t2.y));
+                        rs = fadd2(rs, pe);
+                        pk[e] = f2_to_bf2(pe.x, pe.y);
                     }
-                    tmem_st16(trow + colS + 16 * c, pk);
+#pragma unroll
+                    for (int q = 0; q < kChunkKeys / 64; ++q)
+                        tmem_st32(trow + colS + c * (kChunkKeys / 2) + 32 * q,
+                                  *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * q]));
+                    if constexpr (kChunkKeys == 32)
+                        tmem_st16(trow + colS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(smem_u32(&sm.p_full[t][c]));
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(smem_u32(&sm.p_full[t]));
-                l_run += rowsum;
+                l_run += rs.x + rs.y;
             }
             // ---- epilogue: O / l -> bf16 -> swizzled smem -> TMA store; LSE
             if (ok) ok = warp_wait(smem_u32(&sm.o_done[t]), (nt[t] - 1) & 1, abort_flag, 0x33);
@@ -367,21 +414,22 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc_fence_after();
             const float inv_l = 1.f / l_run;
             const uint32_t stage = smem_u32(sm.q[t]);
+            {
+                uint32_t o[D];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(trow + colO + 32 * c, o);
+                for (int c = 0; c < D / 32; ++c)
+                    tmem_ld32(trow + colO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
                 tmem_wait_ld();
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {       // four 16-byte chunks of 8 values
-                    const int e0 = 32 * c + 8 * q4;     // first element of the chunk
+                for (int q8 = 0; q8 < D / 8; ++q8) {     // 16-byte chunks of 8 values
+                    const int e0 = 8 * q8;
                     const int bx = e0 / C::BOXD;
                     const int ci = (e0 % C::BOXD) / 8;
                     uint4 w;
-                    w.x = f2_to_bf2(__uint_as_float(o[8 * q4 + 0]) * inv_l, __uint_as_float(o[8 * q4 + 1]) * inv_l);
-                    w.y = f2_to_bf2(__uint_as_float(o[8 * q4 + 2]) * inv_l, __uint_as_float(o[8 * q4 + 3]) * inv_l);
-                    w.z = f2_to_bf2(__uint_as_float(o[8 * q4 + 4]) * inv_l, __uint_as_float(o[8 * q4 + 5]) * inv_l);
-                    w.w = f2_to_bf2(__uint_as_float(o[8 * q4 + 6]) * inv_l, __uint_as_float(o[8 * q4 + 7]) * inv_l);
+                    w.x = f2_to_bf2(__uint_as_float(o[e0 + 0]) * inv_l, __uint_as_float(o[e0 + 1]) * inv_l);
+                    w.y = f2_to_bf2(__uint_as_float(o[e0 + 2]) * inv_l, __uint_as_float(o[e0 + 3]) * inv_l);
+                    w.z = f2_to_bf2(__uint_as_float(o[e0 + 4]) * inv_l, __uint_as_float(o[e0 + 5]) * inv_l);
+                    w.w = f2_to_bf2(__uint_as_float(o[e0 + 6]) * inv_l, __uint_as_float(o[e0 + 7]) * inv_l);
                     sts128(stage + bx * C::QBOX + swz<C::SWB>((uint32_t)(r * C::ROWB + ci * 16)), w);
                 }
             }

@@ -74,7 +74,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Slow path of a bounded wait: spin on try_wait, watch the CTA's abort flag
 // and the wall clock. On expiry: record the site, raise the status word and
 // the CTA's abort flag, and return false so the caller can unwind.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                             uint32_t site, unsigned long long limit_ns) {
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
@@ -226,6 +226,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -281,20 +290,71 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
     __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&t);
 }
-// d = a * b + c on fp32 pairs (one FFMA2)
+// Packed fp32 pair arithmetic (one FFMA2 / FADD2 / FMUL2 instruction each).
+// The pairs are assembled inside the asm block so no value goes through memory.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    unsigned long long ra = *reinterpret_cast<unsigned long long *>(&a);
-    unsigned long long rb = *reinterpret_cast<unsigned long long *>(&b);
-    unsigned long long rc = *reinterpret_cast<unsigned long long *>(&c);
-    unsigned long long rd;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
-    return *reinterpret_cast<float2 *>(&rd);
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// max of three fp32 values (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for a pair of values on the FMA pipe, used beside the special-function
+// unit so that both units produce exponentials at the same time.
+// Method: range reduction x = n + f with n the nearest integer (adding
+// 1.5 * 2^23 rounds x to an integer held in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f by a cubic whose coefficients minimise the maximum
+// relative error on that interval (Remez exchange, derived for this library:
+// max relative error 7.5e-5, far below the bf16 rounding P goes through);
+// 2^n applied by adding n to the exponent field. Inputs are clamped to
+// >= -125 so the result stays a normal number (2^-125 stands in for 0).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+    constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+    constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+    const float2 n = fadd2(t, make_float2(-kMagic, -kMagic));
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+    float2 p = ffma2(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+    p = ffma2(p, f, make_float2(kC1, kC1));
+    p = ffma2(p, f, make_float2(kC0, kC0));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {

@@ -185,3 +185,20 @@ def test_empty_batch_is_noop():
     q, k, v = inputs.prefill_inputs(0, 64, 64, 4, 2, 64, 64, 1, device="cuda")
     o, lse = binding.attn_fwd(q, k, v, True, 0.1)
     assert o.numel() == 0 and lse.numel() == 0
+
+
+def test_exponential_accuracy():
+    """The FMA-pipe 2^x (range reduction + fitted cubic) against float64 2^x:
+    relative error below 1e-4 on the softmax's input range; clamped at -125
+    (2^-125 stands in for 0); the special-function unit's ex2 as a control."""
+    binding = need_gpu()
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_003), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0])])
+    yp, ys = binding.selftest_ex2(x.cuda())
+    ref = torch.exp2(x.double())
+    rel_p = ((yp.double().cpu() - ref) / ref).abs().max().item()
+    rel_s = ((ys.double().cpu() - ref) / ref).abs().max().item()
+    assert rel_p < 1e-4, rel_p
+    assert rel_s < 1e-5, rel_s
+    yp2, _ = binding.selftest_ex2(torch.tensor([-1e4, -200.0, float("-inf")], device="cuda"))
+    y2 = yp2.double().cpu()
+    assert torch.all((y2 - 2.0 ** -125).abs() <= 1e-4 * 2.0 ** -125), y2
