@@ -4,7 +4,9 @@ One step = one pass of the hot path over synthetic inputs resident in HBM:
   * prefill: attn_fwd on the Llama-3-8B-shaped causal GQA workload
     (B=1, S=4096, 32 query / 8 KV heads, head dim 128) -- the headline;
   * decode: attn_decode on the GQA decode workload (B=32, cache lengths
-    ~U[1024, 32768], 32/8 heads, head dim 128), split-KV + combine.
+    ~U[1024, 32768], 32/8 heads, head dim 128), split-KV + combine;
+  * MLA decode: attn_decode on the latent cache (B=64, 4096 rows of 576,
+    128 heads, value = first 512 columns).
 `value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
 decode regime is reported in HBM GB/s (algorithmic bytes: the K/V rows below
 each sequence's length, plus q, o and lse) under "regimes". Each kernel is
@@ -35,6 +37,7 @@ if ROOT not in sys.path:
 METRIC = "prefill TFLOP/s & decode HBM GB/s (fraction of B200 peak), 1 GPU"
 HEADLINE = "llama3_8b_prefill"
 DECODE = "gqa_decode"
+MLA = "mla_decode"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -65,6 +68,12 @@ def decode_bytes(w, seqlens) -> float:
 
 def decode_flops(w, seqlens) -> float:
     return float(sum(int(x) for x in seqlens)) * w.n_q * 2 * (w.d_qk + w.d_v)
+
+
+def mla_bytes(w, seqlens) -> float:
+    """Each latent row is read once (it is both key and value), plus q, o, lse."""
+    rows = float(sum(int(x) for x in seqlens))
+    return rows * w.d_qk * 2 + w.B * w.n_q * (w.d_qk * 2 + w.d_v * 2 + 4)
 
 
 # ----------------------------------------------------------------------------
@@ -255,6 +264,15 @@ def run_ours(args):
     wsz = binding.decode_workspace_bytes(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv)
     work = torch.empty(wsz, dtype=torch.uint8, device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    wm = inputs.WORKLOADS[MLA]
+    slm, qm, cm = inputs.mla_inputs(wm.B, wm.n_q, wm.d_qk, wm.Skv, wm.seqlen_range, wm.seed + gen_seed_shift,
+                                    device=dev)
+    cm4 = cm[:, None]
+    slm_dev = slm.to(dev)
+    om = torch.empty((wm.B, wm.n_q, wm.d_v), dtype=torch.bfloat16, device=dev)
+    lm = torch.empty((wm.B, wm.n_q), dtype=torch.float32, device=dev)
+    by_m = mla_bytes(wm, slm)
+    fl_m = decode_flops(wm, slm)
 
     stream = torch.cuda.current_stream(dev)
     fl_p = prefill_flops(w)
@@ -264,8 +282,9 @@ def run_ours(args):
 
     do_p = args.only in ("all", "prefill")
     do_d = args.only in ("all", "decode")
+    do_m = args.only in ("all", "mla")
 
-    def step(times_p, times_d):
+    def step(times_p, times_d, times_m=None):
         if do_p:
             flush.fill_(1.0)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -282,6 +301,14 @@ def run_ours(args):
             e3.record(stream)
             if times_d is not None:
                 times_d.append((e2, e3))
+        if do_m:
+            flush.fill_(3.0)
+            e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e4.record(stream)
+            binding.attn_decode(qm, cm4, cm4, slm_dev, wm.scale, d_v=wm.d_v, o=om, lse=lm, stream=stream)
+            e5.record(stream)
+            if times_m is not None:
+                times_m.append((e4, e5))
 
     def barrier():
         if ws > 1:
@@ -294,18 +321,20 @@ def run_ours(args):
     barrier()
     assert binding.device_status(stream) == 0, "device status not clean after warm-up"
 
-    tp, td = [], []
+    tp, td, tm = [], [], []
     with ClockSampler(torch.cuda.current_device()) as clocks:
         barrier()
         t_wall0 = time.perf_counter()
         for _ in range(args.steps):
-            step(tp, td)
+            step(tp, td, tm)
         barrier()
         t_wall = time.perf_counter() - t_wall0
     st = binding.device_status(stream)
     assert st == 0, f"device status {st}"
     ms_p = [a.elapsed_time(b) for a, b in tp] or [float("nan")]
     ms_d = [a.elapsed_time(b) for a, b in td] or [float("nan")]
+    ms_m = [a.elapsed_time(b) for a, b in tm] or [float("nan")]
+    mean_m = sum(ms_m) / len(ms_m)
     mean_p = sum(ms_p) / len(ms_p)
     mean_d = sum(ms_d) / len(ms_d)
 
@@ -365,6 +394,12 @@ def run_ours(args):
                    "algorithmic_bytes": by_d, "algorithmic_flops": fl_d,
                    "kernels": "attn::dec::decode_split_kernel<4> + decode_combine_kernel",
                    "peak": peak_bw, "peak_source": f"{peak_src} hbm_gbs"},
+        "mla_decode": {"workload": wm.name, "ms": mean_m, "gbs": by_m / (mean_m / 1e3) / 1e9,
+                       "tflops": fl_m / (mean_m / 1e3) / 1e12,
+                       "frac_of_peak_hbm": by_m / (mean_m / 1e3) / 1e9 / peak_bw,
+                       "roofline_frac": max(by_m / (peak_bw * 1e9), fl_m / (peak_tf * 1e12)) / (mean_m / 1e3),
+                       "algorithmic_bytes": by_m, "algorithmic_flops": fl_m,
+                       "kernel": "attn::mla::mla_decode_kernel (2-CTA cluster)"},
     }
 
     cpu_baseline = None
@@ -389,7 +424,7 @@ def run_ours(args):
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
             "clocks": clocks.summary(),
-            "gpu_launches": (int(do_p) + 2 * int(do_d)) * args.steps,
+            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m)) * args.steps,
             "wall_s_timed_region": t_wall,
         }
         print(json.dumps(line), flush=True)
@@ -418,7 +453,7 @@ def main():
                     help="query rows of the headline workload per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla"],
                     help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
     if args.impl == "reference":

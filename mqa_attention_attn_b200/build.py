@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn_b200.so")
 SOURCES = ["attn_api.cu"]
-DEPS = ["attn_api.cu", "sm100.cuh", "prefill.cuh", "decode_gqa.cuh"]
+DEPS = ["attn_api.cu", "sm100.cuh", "prefill.cuh", "decode_gqa.cuh", "decode_mla.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -12,6 +12,7 @@
 
 #include "../../include/attn.h"
 #include "decode_gqa.cuh"
+#include "decode_mla.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -190,6 +191,52 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// MLA decode (latent row of 576 = key, its first 512 columns = value)
+// ---------------------------------------------------------------------------
+int launch_decode_mla(const void *q, const void *cache, const int32_t *seqlens, void *o, float *lse, int B, int n_q,
+                      int S_max, int64_t stride_b, int64_t stride_s, float scale, cudaStream_t stream) {
+    using namespace attn::mla;
+    CUtensorMap tq, tc;
+    {
+        const uint64_t dims[3] = {(uint64_t)DL, (uint64_t)n_q, (uint64_t)B};
+        const uint64_t str[2] = {(uint64_t)DL * 2, (uint64_t)n_q * DL * 2};
+        const uint32_t box[3] = {64u, (uint32_t)M, 1u};
+        if (!make_map(&tq, q, 3, dims, str, box, 128)) return ATTN_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)DL, (uint64_t)S_max, (uint64_t)B};
+        const uint64_t str[2] = {(uint64_t)stride_s * 2, (uint64_t)stride_b * 2};
+        const uint32_t box[3] = {64u, (uint32_t)KT, 1u};
+        if (!make_map(&tc, cache, 3, dims, str, box, 128)) return ATTN_ERR_CUDA;
+    }
+    const size_t smem = smem_bytes();
+    static uint64_t attr_done = 0;
+    if (!ensure_smem_attr(mla_decode_kernel, smem, attr_done)) return ATTN_ERR_CUDA;
+    Params p;
+    p.B = B;
+    p.n_q = n_q;
+    p.S_max = S_max;
+    p.seqlens = seqlens;
+    p.o = reinterpret_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * B, n_q / M, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mla_decode_kernel, tq, tc, p) != cudaSuccess) return ATTN_ERR_CUDA;
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
@@ -244,7 +291,11 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
 
 int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, size_t *bytes) {
     if (!bytes || B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
-    if (!((d_qk == 128 && d_v == 128) || (d_qk == 576 && d_v == 512 && n_kv == 1))) return ATTN_ERR_UNSUPPORTED;
+    if (d_qk == 576 && d_v == 512 && n_kv == 1) {  // the MLA kernel keeps everything on chip
+        *bytes = 0;
+        return ATTN_OK;
+    }
+    if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
     *bytes = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
     return ATTN_OK;
 }
@@ -283,7 +334,14 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         }
     }
     if (d_qk == 576 && d_v == 512 && n_kv == 1) {
-        return ATTN_ERR_UNSUPPORTED;  // MLA decode kernel: not built yet
+        // the value rows must be the first 512 columns of the key rows
+        if (vcache != kcache || v_stride_b != k_stride_b || v_stride_s != k_stride_s) return ATTN_ERR_UNSUPPORTED;
+        if (n_q % attn::mla::M != 0 || n_q / attn::mla::M > 65535) return ATTN_ERR_UNSUPPORTED;
+        if (k_stride_s < 576) return ATTN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(kcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+        if ((k_stride_b | k_stride_s) & 7) return ATTN_ERR_MISALIGNED;
+        if (B > 32767) return ATTN_ERR_UNSUPPORTED;
+        return launch_decode_mla(q, kcache, seqlens, o, lse, B, n_q, S_max, k_stride_b, k_stride_s, scale, s);
     }
     return ATTN_ERR_UNSUPPORTED;
 }
