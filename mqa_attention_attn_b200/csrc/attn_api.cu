@@ -81,6 +81,19 @@ bool ensure_smem_attr(K kernel, size_t bytes, uint64_t &done_mask) {
 }
 inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
+// Number of SMs of the current device (cached per device).
+int sm_count() {
+    static int counts[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
 // ---------------------------------------------------------------------------
 // prefill
 // ---------------------------------------------------------------------------
@@ -162,10 +175,18 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
                       int B, int n_q, int n_kv, int S_max, const int64_t *ks, const int64_t *vs, float scale,
                       void *ws, cudaStream_t stream) {
     using namespace attn::dec;
+    using C = Cfg<GT>;
     const int G = n_q / n_kv;
     const int n_hb = G / GT;
     const int n_splits = decode_n_splits(S_max);
-    CUtensorMap tk, tv;
+    CUtensorMap tq, tk, tv;
+    {
+        // the group's query rows: [B][n_q][128], box = 64 dims x NH heads
+        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)n_q, (uint64_t)B};
+        const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)n_q * D * 2};
+        const uint32_t box[3] = {64u, (uint32_t)C::NH, 1u};
+        if (!make_map(&tq, q, 3, dims, str, box, 128)) return ATTN_ERR_CUDA;
+    }
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S_max, (uint64_t)n_kv, (uint64_t)B};
     const uint32_t box[4] = {64u, (uint32_t)KT, 1u, 1u};
     const uint64_t kstr[3] = {(uint64_t)ks[2] * 2, (uint64_t)ks[1] * 2, (uint64_t)ks[0] * 2};
@@ -180,10 +201,13 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
     o_bytes = (o_bytes + 255) & ~size_t(255);
     float2 *ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(ws) + o_bytes);
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
-    dim3 grid(n_splits, n_kv * n_hb, B);
-    decode_split_kernel<GT><<<grid, THREADS, smem, stream>>>(tk, tv, reinterpret_cast<const __nv_bfloat16 *>(q),
-                                                             seqlens, ws_o, ws_ml, n_q, G, n_hb, S_max, n_splits,
-                                                             scale_log2);
+    // persistent: two CTAs per SM, never more than the largest possible unit count
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return ATTN_ERR_CUDA;
+    const long long max_units = (long long)B * n_kv * n_hb * n_splits;
+    const int grid = (int)(max_units < 2LL * n_sm ? max_units : 2LL * n_sm);
+    decode_split_kernel<GT><<<grid, THREADS, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q, n_kv, G,
+                                                             n_hb, S_max, n_splits, scale_log2);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     decode_combine_kernel<<<dim3(n_q, B), 128, 0, stream>>>(ws_o, ws_ml, seqlens,
                                                               reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q,
@@ -324,13 +348,13 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
         const int64_t ks[3] = {k_stride_b, k_stride_h, k_stride_s};
         const int64_t vs[3] = {v_stride_b, v_stride_h, v_stride_s};
-        const int GT = G >= 8 ? 8 : G;
-        if ((long long)n_kv * (G / GT) > 65535) return ATTN_ERR_UNSUPPORTED;
+        const int GT = G >= 16 ? 16 : G;
         switch (GT) {
             case 1: return launch_decode_gqa<1>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
             case 2: return launch_decode_gqa<2>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
             case 4: return launch_decode_gqa<4>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
-            default: return launch_decode_gqa<8>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
+            case 8: return launch_decode_gqa<8>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
+            default: return launch_decode_gqa<16>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
         }
     }
     if (d_qk == 576 && d_v == 512 && n_kv == 1) {

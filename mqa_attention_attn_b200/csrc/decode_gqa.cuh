@@ -1,48 +1,76 @@
 // decode_gqa.cuh -- single-token GQA decode against a KV cache, split-KV.
 //
-// One CTA owns (sequence b, KV head g, a block of GT query heads of that
-// group, one chunk of CH consecutive cached keys). The chunk's keys and
-// values are streamed HBM -> shared memory by TMA (tile = 64 keys x 128
-// dims, 128-byte swizzle) through a 4-stage ring fed by a producer warp; four
-// compute warps consume it on the CUDA cores (fp32, packed FFMA2):
-//   phase A  scores s[key][h] = <q_h, k_key> * scale * log2(e), all chunk keys
-//   phase B  per head: m = max over the chunk, p = 2^(s - m), l = sum p
-//   phase C  o[h][:] = sum_key p[key][h] * v_key[:]
-// and the partial (o, m, l) goes to the workspace. A second kernel merges the
-// chunks of each (b, h) by their log-sum-exp weights.
+// A work unit is (sequence b, KV head g, a block of GT query heads of that
+// group, one chunk of CH = 512 consecutive cached keys). The grid is
+// persistent (two CTAs per SM); each CTA walks its share of the units.
 //
-// Each K/V tile is read from HBM once and used by all GT heads of the group
-// (the grouped broadcast of "Attention Engineering: From MHA to GQA, MLA &
-// FlashAttention", section 2, done in registers); the chunk merge is the
-// online-softmax rescaling of section 4 applied across chunks instead of
-// tiles. Decode arithmetic intensity is about n_q / n_kv FLOPs per byte
-// (same page, section 0), so this kernel is bound by HBM bandwidth: the
-// design goal is to keep the ring full and the CUDA-core work per byte small.
+// Per unit, with the group's GT query rows as the narrow operand of the
+// 5th-generation tensor core (padded to NH = max(8, GT) columns):
+//   S^T[key][h] = K_tile . Q^T        M = 128 keys, N = NH, K = 128 dims
+//   (softmax over the chunk on the CUDA cores, reading S^T from TMEM)
+//   O^T[d][h]  += V_tile^T . P^T      M = 128 dims, N = NH, K = 128 keys
+// K and V tiles (128 keys x 128 dims, two 64-dim boxes with the 128-byte
+// swizzle) stream HBM -> shared memory by TMA through a ring that a producer
+// warp keeps full across units; one thread issues the MMAs; four warps
+// (one TMEM lane quarter each) do the softmax and write the partial
+// (o, m, l) of the chunk to the workspace. A second kernel merges the chunks
+// of each (b, h) by their log-sum-exp weights.
+//
+// Each K/V element is read from HBM once and used by all GT heads of its
+// group (the grouped sharing of "Attention Engineering: From MHA to GQA, MLA
+// & FlashAttention", section 2); the chunk merge is the online-softmax
+// rescaling of section 4 applied across chunks instead of tiles. Decode
+// arithmetic intensity is about n_q / n_kv FLOPs per byte (same page,
+// section 0), so the kernel is bound by HBM bandwidth; the tensor core is
+// used because it retires the G-fold reuse of every loaded element in a few
+// instructions, leaving the issue slots of the SM to the data movement and
+// the softmax.
 #pragma once
 
 #include "sm100.cuh"
+
+#ifndef ATTN_DEC_STAGES
+#define ATTN_DEC_STAGES 2
+#endif
 
 namespace attn {
 namespace dec {
 
 constexpr int D = 128;            // head dim (keys and values)
-constexpr int KT = 64;            // keys per tile
-constexpr int CH = 512;           // keys per chunk (one CTA)
-constexpr int NSTAGE = 4;         // ring depth
-constexpr int TILE_BYTES = KT * D * 2;      // 16 KB: two 64-dim boxes of 64 rows x 128 B
-constexpr int BOX_BYTES = KT * 128;         // one 64-dim box
-constexpr int NCW = 4;            // compute warps
-constexpr int THREADS = (NCW + 1) * 32;
+constexpr int KT = 128;           // keys per tile (the MMA's M for S^T)
+constexpr int CH = 512;           // keys per chunk (one work unit)
+constexpr int TPC = CH / KT;      // tiles per chunk
+constexpr int NSTAGE = ATTN_DEC_STAGES;
+constexpr int BOX_BYTES = KT * 128;         // one 64-dim box: 128 rows x 128 B
+constexpr int TILE_BYTES = 2 * BOX_BYTES;   // 32 KB
+constexpr int NSW = 4;            // softmax warps (TMEM lane quarters)
+constexpr int PRODUCER_WARP = 4;
+constexpr int MMA_WARP = 5;
+constexpr int THREADS = 6 * 32;
+
+template <int GT>
+struct Cfg {
+    static constexpr int NH = GT < 8 ? 8 : GT;             // MMA N (query-head columns)
+    static constexpr int QBOX = NH * 128;                   // one 64-dim half of the Q rows
+    static constexpr int COL_S = 0;                         // S^T: TPC tiles x NH columns
+    static constexpr int COL_O = TPC * NH;                  // O^T: NH columns
+    static constexpr int NEED = COL_O + NH;
+    static constexpr int TMEM_COLS = NEED <= 32 ? 32 : NEED <= 64 ? 64 : NEED <= 128 ? 128 : 256;
+    static_assert(GT == 1 || GT == 2 || GT == 4 || GT == 8 || GT == 16 || GT == 32, "head block");
+};
 
 template <int GT>
 struct Smem {
+    using C = Cfg<GT>;
     uint8_t ring[NSTAGE][TILE_BYTES];       // 1024-byte aligned (swizzle atoms)
-    float scores[CH * GT];                  // [key][head], log2 units, then p
-    float opart[NCW][GT][D];                // per-warp partial outputs
-    float red_m[NCW][GT];
-    float red_l[NCW][GT];
+    uint8_t q[2][C::QBOX];                  // Q rows, two 64-dim boxes, 128-byte swizzle
+    uint8_t p[C::NH / 8][CH * 16];          // P^T: [8-head block][key][8 heads] bf16
+    float red_m[2][NSW][GT];                // double-buffered by unit parity
+    float red_l[2][NSW][GT];
     uint64_t full[NSTAGE];
     uint64_t empty[NSTAGE];
+    uint64_t q_full, q_empty, s_full, p_full, o_full, mma_done;
+    uint32_t tmem_base;
     int abort_flag;
 };
 
@@ -51,254 +79,318 @@ constexpr size_t smem_bytes() {
     return sizeof(Smem<GT>) + 1024;  // + alignment slack
 }
 
-// Mapping of compute warps in phase A: each thread holds a quarter of the
-// head dim (32 values) of HPT heads; warps split into HS head sets x KS key
-// sets.
-template <int GT>
-struct QkMap {
-    static constexpr int HPT = GT < 2 ? GT : 2;
-    static constexpr int HS = GT / HPT;
-    static constexpr int KS = NCW / HS;
-    static_assert(HS * KS == NCW, "head block must map onto 4 warps");
+// Work units are the non-empty (b, kv head, head block, chunk) slots, in order
+// b-major, then kv head and head block, then chunk; sequence b contributes
+// n_kv * n_hb * ceil(seqlen_b / CH) units. The CTA walks units c, c + G, ...
+// (G = gridDim.x) and every role derives the same unit from its index.
+struct UnitCursor {
+    int b = 0;          // sequence of the current range
+    long long base = 0; // first unit index of sequence b
+    int ns = 0;         // chunks of sequence b
+    int seqlen = 0;
 };
+
+struct Unit {
+    int b, kvh, hb, split, key0, nkeys, ntiles;
+};
+
+__device__ __forceinline__ int clamp_seqlen(const int32_t *seqlens, int b, int S_max) {
+    int L = seqlens[b];
+    return L < 0 ? 0 : (L > S_max ? S_max : L);
+}
+
+// Advance the cursor to the sequence holding unit i (i never decreases) and
+// decode the unit. Returns false when i is past the last unit.
+__device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const int32_t *seqlens, int B, int S_max,
+                                          int n_hb, int units_per_chunk, Unit &u) {
+    while (cur.b < B) {
+        const long long n = (long long)units_per_chunk * cur.ns;
+        if (i < cur.base + n) {
+            const long long local = i - cur.base;
+            const int y = (int)(local / cur.ns);
+            u.b = cur.b;
+            u.split = (int)(local % cur.ns);
+            u.kvh = y / n_hb;
+            u.hb = y % n_hb;
+            u.key0 = u.split * CH;
+            u.nkeys = min(CH, cur.seqlen - u.key0);
+            u.ntiles = (u.nkeys + KT - 1) / KT;
+            return true;
+        }
+        cur.base += n;
+        ++cur.b;
+        if (cur.b < B) {
+            cur.seqlen = clamp_seqlen(seqlens, cur.b, S_max);
+            cur.ns = (cur.seqlen + CH - 1) / CH;
+        }
+    }
+    return false;
+}
 
 template <int GT>
 __global__ void __launch_bounds__(THREADS, 2)
-decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ seqlens,
-                    float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int n_q, int G, int n_hb,
+decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
+                    float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
                     int S_max, int n_splits, float scale_log2) {
-    using Map = QkMap<GT>;
+    using C = Cfg<GT>;
+    constexpr int NH = C::NH;
     extern __shared__ uint8_t smem_raw[];
     Smem<GT> &sm = *reinterpret_cast<Smem<GT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-    const int split = blockIdx.x;
-    const int kvh = blockIdx.y / n_hb;
-    const int hb = blockIdx.y % n_hb;
-    const int b = blockIdx.z;
-    int seqlen = seqlens[b];
-    if (seqlen > S_max) {
-        if (threadIdx.x == 0 && split == 0 && blockIdx.y == 0) atomicOr(&g_status, kStatusRange);
-        seqlen = S_max;
-    }
-    if (seqlen < 0) seqlen = 0;
-    const int key0 = split * CH;
-    if (key0 >= seqlen) return;  // uniform for the CTA
-    const int nkeys = min(CH, seqlen - key0);
-    const int ntiles = (nkeys + KT - 1) / KT;
-    const int h0 = kvh * G + hb * GT;  // first query head of this CTA
-
     const uint32_t warp = warp_id(), lane = lane_id();
+    const int units_per_chunk = n_kv * n_hb;   // units of one chunk index of one sequence
+
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(smem_u32(&sm.full[s]), 1);
-            mbar_init(smem_u32(&sm.empty[s]), NCW);
+            mbar_init(smem_u32(&sm.empty[s]), 1);
         }
+        mbar_init(smem_u32(&sm.q_full), 1);
+        mbar_init(smem_u32(&sm.q_empty), 1);
+        mbar_init(smem_u32(&sm.s_full), 1);
+        mbar_init(smem_u32(&sm.p_full), NSW * 32);
+        mbar_init(smem_u32(&sm.o_full), 1);
+        mbar_init(smem_u32(&sm.mma_done), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
+        // values above S_max are clamped; report it once per launch
+        if (blockIdx.x == 0)
+            for (int b = 0; b < B; ++b)
+                if (seqlens[b] > S_max) {
+                    atomicOr(&g_status, kStatusRange);
+                    break;
+                }
     }
+    if (warp == MMA_WARP) {
+        tmem_alloc(smem_u32(&sm.tmem_base), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
 
-    if (warp == NCW) {
-        // ---------------- producer warp ----------------
+    UnitCursor cur;
+    cur.seqlen = B > 0 ? clamp_seqlen(seqlens, 0, S_max) : 0;
+    cur.ns = (cur.seqlen + CH - 1) / CH;
+    Unit u;
+
+    if (warp == PRODUCER_WARP) {
+        // ---------------- TMA producer: Q rows, then K tiles, then V tiles ----------------
         if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            int issued = 0;
-            for (int t = 0; t < 2 * ntiles; ++t) {
-                const int s = t % NSTAGE;
-                const uint32_t ph = (t / NSTAGE) & 1;
-                if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1, abort_flag, 0x101)) break;
-                const uint32_t full = smem_u32(&sm.full[s]);
-                mbar_arrive_expect_tx(full, TILE_BYTES);
-                const CUtensorMap *tm = (t < ntiles) ? &tm_k : &tm_v;
-                const int krow = key0 + (t < ntiles ? t : t - ntiles) * KT;
-                const uint32_t dst = smem_u32(sm.ring[s]);
-                tma_load_4d(dst, tm, full, 0, krow, kvh, b);
-                tma_load_4d(dst + BOX_BYTES, tm, full, 64, krow, kvh, b);
-                ++issued;
+            int t = 0, n = 0;   // ring tiles issued, units started
+            bool ok = true;
+            for (long long i = blockIdx.x; ok && next_unit(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+                 i += gridDim.x, ++n) {
+                // the single Q buffer is free once the previous unit's S^T MMAs completed
+                if (n > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n - 1) & 1, abort_flag, 0x101)) break;
+                const int h0 = u.kvh * G + u.hb * GT;
+                mbar_arrive_expect_tx(smem_u32(&sm.q_full), 2 * C::QBOX);
+                tma_load_3d(smem_u32(sm.q[0]), &tm_q, smem_u32(&sm.q_full), 0, h0, u.b);
+                tma_load_3d(smem_u32(sm.q[1]), &tm_q, smem_u32(&sm.q_full), 64, h0, u.b);
+                for (int j = 0; j < 2 * u.ntiles; ++j, ++t) {
+                    const int s = t % NSTAGE;
+                    if (!mbar_wait(smem_u32(&sm.empty[s]), ((t / NSTAGE) & 1) ^ 1, abort_flag, 0x102)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full = smem_u32(&sm.full[s]);
+                    mbar_arrive_expect_tx(full, TILE_BYTES);
+                    const CUtensorMap *tm = (j < u.ntiles) ? &tm_k : &tm_v;
+                    const int krow = u.key0 + (j < u.ntiles ? j : j - u.ntiles) * KT;
+                    const uint32_t dst = smem_u32(sm.ring[s]);
+                    tma_load_4d(dst, tm, full, 0, krow, u.kvh, u.b);
+                    tma_load_4d(dst + BOX_BYTES, tm, full, 64, krow, u.kvh, u.b);
+                }
             }
             // Do not leave while copies into this CTA's shared memory are in
-            // flight: wait (bounded) for the last issued tile of each stage.
-            for (int t = issued - 1; t >= 0 && t >= issued - NSTAGE; --t)
-                mbar_wait(smem_u32(&sm.full[t % NSTAGE]), (t / NSTAGE) & 1, nullptr, 0x102);
+            // flight: wait (bounded) for the last issued tile of each stage
+            // and the last Q load.
+            for (int j = t - 1; j >= 0 && j >= t - NSTAGE; --j)
+                mbar_wait(smem_u32(&sm.full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x103);
+            if (n > 0) mbar_wait(smem_u32(&sm.q_full), (n - 1) & 1, nullptr, 0x104);
         }
-        return;
-    }
-
-    // ---------------- compute warps (128 threads) ----------------
-    const int tid = threadIdx.x;  // 0..127
-
-    // phase A: scores ------------------------------------------------------
-    {
-        const int hs = warp / Map::KS;        // head set
-        const int ks = warp % Map::KS;        // key set
-        const int quarter = lane >> 3;        // which 32 dims
-        const int kl = lane & 7;              // key within the warp's 8
-        float2 qr[Map::HPT][16];
-#pragma unroll
-        for (int hh = 0; hh < Map::HPT; ++hh) {
-            const int h = h0 + hs * Map::HPT + hh;
-            const uint4 *src = reinterpret_cast<const uint4 *>(q + ((size_t)b * n_q + h) * D + quarter * 32);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 w = __ldg(src + c);
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 f = bf2_to_f2(ws[e]);
-                    qr[hh][c * 4 + e] = make_float2(f.x * scale_log2, f.y * scale_log2);
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ---------------- MMA issue (one thread), ring bookkeeping (whole warp) ----------------
+        constexpr uint32_t idesc_s = umma_idesc_bf16(KT, NH, 0, 0);   // K tile (K-major) x Q rows (K-major)
+        constexpr uint32_t idesc_o = umma_idesc_bf16(D, NH, 1, 1);    // V^T (MN-major) x P^T (MN-major)
+        int t = 0, n = 0;
+        for (long long i = blockIdx.x; next_unit(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+             i += gridDim.x, ++n) {
+            if (!mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x201)) break;
+            bool ok = true;
+            for (int j = 0; j < u.ntiles; ++j) {
+                const int g = t + j, s = g % NSTAGE;
+                if (!mbar_wait(smem_u32(&sm.full[s]), (g / NSTAGE) & 1, abort_flag, 0x202)) {
+                    ok = false;
+                    break;
                 }
-            }
-        }
-        for (int t = 0; t < ntiles; ++t) {
-            const int s = t % NSTAGE;
-            if (!mbar_wait(smem_u32(&sm.full[s]), (t / NSTAGE) & 1, abort_flag, 0x201)) break;
-            const uint32_t base = smem_u32(sm.ring[s]);
-#pragma unroll 2
-            for (int p = 0; p < KT / (8 * Map::KS); ++p) {
-                const int key = p * 8 * Map::KS + ks * 8 + kl;  // key within the tile
-                float2 acc[Map::HPT];
+                tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
-                for (int hh = 0; hh < Map::HPT; ++hh) acc[hh] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int c = quarter * 4 + i;  // 16-byte chunk of the 256-byte row
-                    const uint32_t off = (uint32_t)((c >> 3) * BOX_BYTES) + swz<3>((uint32_t)(key * 128 + (c & 7) * 16));
-                    const uint4 w = lds128(base + off);
-                    const float2 k0 = bf2_to_f2(w.x), k1 = bf2_to_f2(w.y), k2 = bf2_to_f2(w.z), k3 = bf2_to_f2(w.w);
-#pragma unroll
-                    for (int hh = 0; hh < Map::HPT; ++hh) {
-                        acc[hh] = ffma2(qr[hh][i * 4 + 0], k0, acc[hh]);
-                        acc[hh] = ffma2(qr[hh][i * 4 + 1], k1, acc[hh]);
-                        acc[hh] = ffma2(qr[hh][i * 4 + 2], k2, acc[hh]);
-                        acc[hh] = ffma2(qr[hh][i * 4 + 3], k3, acc[hh]);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = (uint32_t)((kk >> 2) * BOX_BYTES + (kk & 3) * 32);
+                        const uint32_t qoff = (uint32_t)((kk >> 2) * C::QBOX + (kk & 3) * 32);
+                        const uint64_t ad = umma_smem_desc(smem_u32(sm.ring[s]) + koff, 16, 1024, 2);
+                        const uint64_t bd = umma_smem_desc(smem_u32(sm.q[0]) + qoff, 16, 1024, 2);
+                        umma_ss(tmem + C::COL_S + j * NH, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                     }
+                    umma_commit(smem_u32(&sm.empty[s]));
                 }
-#pragma unroll
-                for (int hh = 0; hh < Map::HPT; ++hh) {
-                    float sc = acc[hh].x + acc[hh].y;
-                    sc += __shfl_xor_sync(0xffffffffu, sc, 8);
-                    sc += __shfl_xor_sync(0xffffffffu, sc, 16);
-                    if (quarter == hh) sm.scores[(t * KT + key) * GT + hs * Map::HPT + hh] = sc;
-                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) {
+                umma_commit(smem_u32(&sm.q_empty));
+                umma_commit(smem_u32(&sm.s_full));
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+            t += u.ntiles;
+            if (!mbar_wait(smem_u32(&sm.p_full), n & 1, abort_flag, 0x203)) break;
+            tc_fence_after();
+            for (int j = 0; j < u.ntiles; ++j) {
+                const int g = t + j, s = g % NSTAGE;
+                if (!mbar_wait(smem_u32(&sm.full[s]), (g / NSTAGE) & 1, abort_flag, 0x204)) {
+                    ok = false;
+                    break;
+                }
+                const int rows = u.nkeys - j * KT;   // valid value rows of this tile
+                if (rows < KT) {
+                    // Rows past the sequence end get weight 0, but 0 * (NaN or
+                    // Inf) is not 0: clear them so that whatever the cache holds
+                    // beyond the length cannot reach the output.
+                    const uint32_t base = smem_u32(sm.ring[s]);
+                    for (int e = rows * 8 + (int)lane; e < KT * 8; e += 32) {
+                        const uint32_t off = (uint32_t)(e >> 3) * 128u + (uint32_t)(e & 7) * 16u;
+                        sts128(base + off, make_uint4(0u, 0u, 0u, 0u));
+                        sts128(base + BOX_BYTES + off, make_uint4(0u, 0u, 0u, 0u));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int ks = 0; ks < KT / 16; ++ks) {
+                        // A = V^T: 16 keys x 128 dims of the tile; B = P^T rows of the same 16 keys
+                        const uint64_t ad = umma_smem_desc(smem_u32(sm.ring[s]) + ks * 16 * 128, BOX_BYTES, 1024, 2);
+                        const uint64_t bd = umma_smem_desc(smem_u32(sm.p[0]) + (j * KT + ks * 16) * 16, 128, CH * 16, 0);
+                        umma_ss(tmem + C::COL_O, ad, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&sm.empty[s]));
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(smem_u32(&sm.o_full));
+            __syncwarp();
+            t += u.ntiles;
         }
-    }
-    if (named_bar_or(1, NCW * 32, *abort_flag != 0)) return;
-
-    // phase B: softmax statistics over the chunk ------------------------------
-    float m[GT], l[GT];
-    {
-        float mloc[GT];
+        // every MMA issued by this warp has completed before TMEM is released
+        if (lane == 0) umma_commit(smem_u32(&sm.mma_done));
+        __syncwarp();
+        mbar_wait(smem_u32(&sm.mma_done), 0, nullptr, 0x205);
+    } else if (warp < NSW) {
+        // ---------------- softmax + partial output (128 threads, thread = TMEM lane) ----------------
+        const int tid = threadIdx.x;                       // key row of each tile; dim row of O^T
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        int n = 0;
+        for (long long i = blockIdx.x; next_unit(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+             i += gridDim.x, ++n) {
+            const int h0 = u.kvh * G + u.hb * GT;
+            bool ok = mbar_wait(smem_u32(&sm.s_full), n & 1, abort_flag, 0x301);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            uint32_t sv[TPC][NH];
 #pragma unroll
-        for (int h = 0; h < GT; ++h) mloc[h] = -INFINITY;
-        for (int key = tid; key < nkeys; key += NCW * 32) {
-#pragma unroll
-            for (int h = 0; h < GT; ++h) mloc[h] = fmaxf(mloc[h], sm.scores[key * GT + h]);
-        }
-#pragma unroll
-        for (int h = 0; h < GT; ++h) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], o));
-            if (lane == 0) sm.red_m[warp][h] = mloc[h];
-        }
-        named_bar_sync(1, NCW * 32);
-#pragma unroll
-        for (int h = 0; h < GT; ++h) {
-            m[h] = sm.red_m[0][h];
-#pragma unroll
-            for (int w = 1; w < NCW; ++w) m[h] = fmaxf(m[h], sm.red_m[w][h]);
-        }
-        float lloc[GT];
-#pragma unroll
-        for (int h = 0; h < GT; ++h) lloc[h] = 0.f;
-        for (int key = tid; key < ntiles * KT; key += NCW * 32) {
+            for (int j = 0; j < TPC; ++j)
+                if (j < u.ntiles) tmem_ld<NH>(lane_base + C::COL_S + j * NH, sv[j]);
+            tmem_wait_ld();
+            // chunk maximum per head
+            float m[GT];
 #pragma unroll
             for (int h = 0; h < GT; ++h) {
-                float pv = 0.f;
-                if (key < nkeys) pv = ex2(sm.scores[key * GT + h] - m[h]);
-                sm.scores[key * GT + h] = pv;
-                lloc[h] += pv;
+                m[h] = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < TPC; ++j)
+                    if (j < u.ntiles && j * KT + tid < u.nkeys) m[h] = fmaxf(m[h], __uint_as_float(sv[j][h]));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], o));
+                if (lane == 0) sm.red_m[n & 1][warp][h] = m[h];
             }
-        }
+            if (named_bar_or(1, NSW * 32, !ok)) break;
+            float mc[GT], l[GT];
 #pragma unroll
-        for (int h = 0; h < GT; ++h) {
+            for (int h = 0; h < GT; ++h) {
+                float mm = sm.red_m[n & 1][0][h];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) lloc[h] += __shfl_xor_sync(0xffffffffu, lloc[h], o);
-            if (lane == 0) sm.red_l[warp][h] = lloc[h];
-        }
-        named_bar_sync(1, NCW * 32);
+                for (int w = 1; w < NSW; ++w) mm = fmaxf(mm, sm.red_m[n & 1][w][h]);
+                mc[h] = mm * scale_log2;     // finite: every unit holds at least one key
+                l[h] = 0.f;
+            }
+            // p = 2^(s * scale * log2 e - m), written as P^T rows of bf16 [key][8 heads]
 #pragma unroll
-        for (int h = 0; h < GT; ++h) {
-            l[h] = 0.f;
+            for (int j = 0; j < TPC; ++j) {
+                if (j >= u.ntiles) break;
+                const bool valid = j * KT + tid < u.nkeys;
+                uint32_t pk[NH / 2];
 #pragma unroll
-            for (int w = 0; w < NCW; ++w) l[h] += sm.red_l[w][h];
-        }
-    }
-
-    // phase C: p . V ------------------------------------------------------------
-    float2 oacc[GT][2];
-#pragma unroll
-    for (int h = 0; h < GT; ++h) oacc[h][0] = oacc[h][1] = make_float2(0.f, 0.f);
-    {
-        const int c = lane >> 1;       // 16-byte chunk holding this lane's 4 dims
-        const int half = lane & 1;
-        const uint32_t box_off = (uint32_t)((c >> 3) * BOX_BYTES);
-        for (int t = 0; t < ntiles; ++t) {
-            const int tt = ntiles + t;
-            const int s = tt % NSTAGE;
-            if (!mbar_wait(smem_u32(&sm.full[s]), (tt / NSTAGE) & 1, abort_flag, 0x301)) break;
-            const uint32_t base = smem_u32(sm.ring[s]) + box_off;
-            const float *ps = sm.scores + (size_t)t * KT * GT;
-#pragma unroll 4
-            for (int kk = warp; kk < KT; kk += NCW) {
-                const uint2 w = lds64(base + swz<3>((uint32_t)(kk * 128 + (c & 7) * 16)) + half * 8);
-                const float2 v0 = bf2_to_f2(w.x), v1 = bf2_to_f2(w.y);
-                float pk[GT];
-                if constexpr (GT % 4 == 0) {
-#pragma unroll
-                    for (int h4 = 0; h4 < GT / 4; ++h4) {
-                        const float4 t4 = *reinterpret_cast<const float4 *>(ps + kk * GT + h4 * 4);
-                        pk[h4 * 4 + 0] = t4.x;
-                        pk[h4 * 4 + 1] = t4.y;
-                        pk[h4 * 4 + 2] = t4.z;
-                        pk[h4 * 4 + 3] = t4.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < GT; ++h) pk[h] = ps[kk * GT + h];
+                for (int h2 = 0; h2 < NH / 2; ++h2) {
+                    float p0 = 0.f, p1 = 0.f;
+                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[j][2 * h2]), scale_log2, -mc[2 * h2]));
+                    if (2 * h2 + 1 < GT && valid)
+                        p1 = ex2(fmaf(__uint_as_float(sv[j][2 * h2 + 1]), scale_log2, -mc[2 * h2 + 1]));
+                    if (2 * h2 < GT) l[2 * h2] += p0;
+                    if (2 * h2 + 1 < GT) l[2 * h2 + 1] += p1;
+                    pk[h2] = f2_to_bf2(p0, p1);
                 }
 #pragma unroll
-                for (int h = 0; h < GT; ++h) {
-                    const float2 pp = make_float2(pk[h], pk[h]);
-                    oacc[h][0] = ffma2(pp, v0, oacc[h][0]);
-                    oacc[h][1] = ffma2(pp, v1, oacc[h][1]);
-                }
+                for (int hb8 = 0; hb8 < NH / 8; ++hb8)
+                    sts128(smem_u32(sm.p[hb8]) + (uint32_t)(j * KT + tid) * 16u,
+                           make_uint4(pk[hb8 * 4 + 0], pk[hb8 * 4 + 1], pk[hb8 * 4 + 2], pk[hb8 * 4 + 3]));
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.p_full));
+#pragma unroll
+            for (int h = 0; h < GT; ++h) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
+                if (lane == 0) sm.red_l[n & 1][warp][h] = l[h];
+            }
+            ok = mbar_wait(smem_u32(&sm.o_full), n & 1, abort_flag, 0x302);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            uint32_t ov[NH];
+            tmem_ld<NH>(lane_base + C::COL_O, ov);
+            tmem_wait_ld();
+            tc_fence_before();
+            if (named_bar_or(1, NSW * 32, !ok)) break;
+            const size_t row0 = (size_t)u.b * n_q + h0;
+#pragma unroll
+            for (int h = 0; h < GT; ++h)
+                ws_o[((row0 + h) * n_splits + u.split) * D + tid] = __uint_as_float(ov[h]);
+#pragma unroll
+            for (int h = 0; h < GT; ++h)
+                if (tid == h) {
+                    float lt = 0.f;
+#pragma unroll
+                    for (int w = 0; w < NSW; ++w) lt += sm.red_l[n & 1][w][h];
+                    ws_ml[(row0 + h) * n_splits + u.split] = make_float2(mc[h], lt);
+                }
         }
     }
-    // combine the four warps' partial sums, write (o, m, l) of this chunk
-#pragma unroll
-    for (int h = 0; h < GT; ++h)
-        *reinterpret_cast<float4 *>(&sm.opart[warp][h][lane * 4]) =
-            make_float4(oacc[h][0].x, oacc[h][0].y, oacc[h][1].x, oacc[h][1].y);
-    if (named_bar_or(1, NCW * 32, *abort_flag != 0)) return;
-#pragma unroll
-    for (int j = 0; j < GT; ++j) {
-        const int idx = tid + j * NCW * 32;  // over GT * D outputs
-        const int h = idx / D, d = idx % D;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) acc += sm.opart[w][h][d];
-        ws_o[(((size_t)b * n_q + h0 + h) * n_splits + split) * D + d] = acc;
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    if (tid < GT) ws_ml[((size_t)b * n_q + h0 + tid) * n_splits + split] = make_float2(m[tid], l[tid]);
 }
 
 // Merge the chunks of each (b, h): M = max m_s, w_s = 2^(m_s - M),

@@ -33,7 +33,9 @@ def _decode_and_check(seqlens, q, kc, vc, scale, what, d_v=None):
     (1, 16, 8, 300, [300]),                 # G=2
     (2, 64, 8, 900, [899, 1]),              # G=8
     (1, 32, 2, 1030, [1030]),               # G=16 (two head blocks)
-    (2, 32, 1, 700, [700, 65]),             # MQA, G=32 (four head blocks)
+    (2, 32, 1, 700, [700, 65]),             # MQA, G=32 (two head blocks)
+    (2, 8, 2, 100, [100, 37]),              # cache shorter than one 128-key tile
+    (1, 2, 2, 513, [513]),                  # MHA with fewer heads than the MMA's 8 columns
 ])
 def test_decode_shapes(B, n_q, n_kv, S_max, seqlens):
     seq = torch.tensor(seqlens, dtype=torch.int32)
@@ -101,6 +103,24 @@ def test_decode_zero_length_and_range_status():
     o_ref, l_ref = oracle.sdpa(q[:, :, None, :], kc, vc, False, 0.1,
                                seqlens=np.array([0, 100, 256], np.int32))
     check_parity(o, lse, o_ref[:, :, 0], l_ref[:, :, 0], "zero/clamped lengths")
+
+
+def test_decode_ignores_nonfinite_cache_rows_past_the_length():
+    """Cache rows at or beyond a sequence's length take no part, whatever they
+    hold: they are filled with NaN and +Inf here, inside the same 128-key
+    tile as valid rows, and the result must equal the oracle's on the valid
+    rows."""
+    B, n_q, n_kv, S_max = 3, 32, 8, 1100
+    seq = torch.tensor([1, 700, 1029], dtype=torch.int32)
+    g = torch.Generator(device="cuda").manual_seed(8)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    for b, L in enumerate(seq.tolist()):
+        kc[b, :, L:] = float("nan")
+        vc[b, :, L:] = float("inf")
+    o, lse = _decode_and_check(seq, q, kc, vc, 0.1, "non-finite rows past the length")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
 
 
 def test_decode_workspace_checks():
