@@ -161,7 +161,13 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
 // ---------------------------------------------------------------------------
 // decode (GQA, head dim 128)
 // ---------------------------------------------------------------------------
-inline int decode_n_splits(int S_max) { return (S_max + attn::dec::CH - 1) / attn::dec::CH; }
+// Query heads per decode work unit (a power of two dividing G) and the
+// number of key chunks of S_max at that block size.
+inline int decode_head_block(int G) { return G >= 16 ? 16 : G; }
+inline int decode_n_splits(int G, int S_max) {
+    const int ch = attn::dec::chunk_keys(decode_head_block(G));
+    return (S_max + ch - 1) / ch;
+}
 
 size_t decode_ws_bytes(int B, int n_q, int d_v, int n_splits) {
     const size_t rows = (size_t)B * n_q * n_splits;
@@ -178,7 +184,7 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
     using C = Cfg<GT>;
     const int G = n_q / n_kv;
     const int n_hb = G / GT;
-    const int n_splits = decode_n_splits(S_max);
+    const int n_splits = decode_n_splits(G, S_max);
     CUtensorMap tq, tk, tv;
     {
         // the group's query rows: [B][n_q][128], box = 64 dims x NH heads
@@ -209,9 +215,8 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
     decode_split_kernel<GT><<<grid, THREADS, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q, n_kv, G,
                                                              n_hb, S_max, n_splits, scale_log2);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    decode_combine_kernel<<<dim3(n_q, B), 128, 0, stream>>>(ws_o, ws_ml, seqlens,
-                                                              reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q,
-                                                              n_splits, S_max, CH, D);
+    decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
+        ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH);
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -320,7 +325,7 @@ int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int
         return ATTN_OK;
     }
     if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
-    *bytes = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
+    *bytes = decode_ws_bytes(B, n_q, d_v, decode_n_splits(n_q / n_kv, S_max));
     return ATTN_OK;
 }
 
@@ -343,13 +348,12 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
         if ((k_stride_b | k_stride_h | k_stride_s | v_stride_b | v_stride_h | v_stride_s) & 7)
             return ATTN_ERR_MISALIGNED;
-        const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
+        const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(G, S_max));
         if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
         const int64_t ks[3] = {k_stride_b, k_stride_h, k_stride_s};
         const int64_t vs[3] = {v_stride_b, v_stride_h, v_stride_s};
-        const int GT = G >= 16 ? 16 : G;
-        switch (GT) {
+        switch (decode_head_block(G)) {
             case 1: return launch_decode_gqa<1>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
             case 2: return launch_decode_gqa<2>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
             case 4: return launch_decode_gqa<4>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
@@ -453,7 +457,7 @@ extern "C" int attn_decode_noalloc(const void *q, const void *kcache, const void
     if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
     if (B == 0) return ATTN_OK;
     if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
-    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(S_max));
+    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(n_q / n_kv, S_max));
     if (need > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;  // beyond the static maximum
     void *scratch = noalloc_scratch_ptr();
     if (scratch == nullptr) return ATTN_ERR_CUDA;

@@ -1,7 +1,7 @@
 // decode_gqa.cuh -- single-token GQA decode against a KV cache, split-KV.
 //
 // A work unit is (sequence b, KV head g, a block of GT query heads of that
-// group, one chunk of CH = 512 consecutive cached keys). The grid is
+// group, one chunk of CH consecutive cached keys, CH = 1024 or 512). The grid is
 // persistent (two CTAs per SM); each CTA walks its share of the units.
 //
 // Per unit, with the group's GT query rows as the narrow operand of the
@@ -38,8 +38,9 @@ namespace dec {
 
 constexpr int D = 128;            // head dim (keys and values)
 constexpr int KT = 128;           // keys per tile (the MMA's M for S^T)
-constexpr int CH = 512;           // keys per chunk (one work unit)
-constexpr int TPC = CH / KT;      // tiles per chunk
+// Keys per chunk (one work unit): 1024 while a head block has at most 8
+// heads, 512 for 16 (the chunk's scores then fill the same registers).
+__host__ __device__ constexpr int chunk_keys(int GT) { return GT <= 8 ? 1024 : 512; }
 constexpr int NSTAGE = ATTN_DEC_STAGES;
 constexpr int BOX_BYTES = KT * 128;         // one 64-dim box: 128 rows x 128 B
 constexpr int TILE_BYTES = 2 * BOX_BYTES;   // 32 KB
@@ -51,6 +52,8 @@ constexpr int THREADS = 6 * 32;
 template <int GT>
 struct Cfg {
     static constexpr int NH = GT < 8 ? 8 : GT;             // MMA N (query-head columns)
+    static constexpr int CH = chunk_keys(GT);               // keys per unit
+    static constexpr int TPC = CH / KT;                     // tiles per unit
     static constexpr int QBOX = NH * 128;                   // one 64-dim half of the Q rows
     static constexpr int COL_S = 0;                         // S^T: TPC tiles x NH columns
     static constexpr int COL_O = TPC * NH;                  // O^T: NH columns
@@ -64,7 +67,7 @@ struct Smem {
     using C = Cfg<GT>;
     uint8_t ring[NSTAGE][TILE_BYTES];       // 1024-byte aligned (swizzle atoms)
     uint8_t q[2][C::QBOX];                  // Q rows, two 64-dim boxes, 128-byte swizzle
-    uint8_t p[C::NH / 8][CH * 16];          // P^T: [8-head block][key][8 heads] bf16
+    uint8_t p[C::NH / 8][C::CH * 16];       // P^T: [8-head block][key][8 heads] bf16
     float red_m[2][NSW][GT];                // double-buffered by unit parity
     float red_l[2][NSW][GT];
     uint64_t full[NSTAGE];
@@ -81,7 +84,7 @@ constexpr size_t smem_bytes() {
 
 // Work units are the non-empty (b, kv head, head block, chunk) slots, in order
 // b-major, then kv head and head block, then chunk; sequence b contributes
-// n_kv * n_hb * ceil(seqlen_b / CH) units. The CTA walks units c, c + G, ...
+// n_kv * n_hb * ceil(seqlen_b / CH) units (CH = keys per unit). The CTA walks units c, c + G, ...
 // (G = gridDim.x) and every role derives the same unit from its index.
 struct UnitCursor {
     int b = 0;          // sequence of the current range
@@ -101,6 +104,7 @@ __device__ __forceinline__ int clamp_seqlen(const int32_t *seqlens, int b, int S
 
 // Advance the cursor to the sequence holding unit i (i never decreases) and
 // decode the unit. Returns false when i is past the last unit.
+template <int CH>
 __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const int32_t *seqlens, int B, int S_max,
                                           int n_hb, int units_per_chunk, Unit &u) {
     while (cur.b < B) {
@@ -173,7 +177,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     UnitCursor cur;
     cur.seqlen = B > 0 ? clamp_seqlen(seqlens, 0, S_max) : 0;
-    cur.ns = (cur.seqlen + CH - 1) / CH;
+    cur.ns = (cur.seqlen + C::CH - 1) / C::CH;
     Unit u;
 
     if (warp == PRODUCER_WARP) {
@@ -184,7 +188,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_prefetch_desc(&tm_v);
             int t = 0, n = 0;   // ring tiles issued, units started
             bool ok = true;
-            for (long long i = blockIdx.x; ok && next_unit(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+            for (long long i = blockIdx.x; ok && next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
                  i += gridDim.x, ++n) {
                 // the single Q buffer is free once the previous unit's S^T MMAs completed
                 if (n > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n - 1) & 1, abort_flag, 0x101)) break;
@@ -220,7 +224,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         constexpr uint32_t idesc_s = umma_idesc_bf16(KT, NH, 0, 0);   // K tile (K-major) x Q rows (K-major)
         constexpr uint32_t idesc_o = umma_idesc_bf16(D, NH, 1, 1);    // V^T (MN-major) x P^T (MN-major)
         int t = 0, n = 0;
-        for (long long i = blockIdx.x; next_unit(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
              i += gridDim.x, ++n) {
             if (!mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x201)) break;
             bool ok = true;
@@ -279,7 +283,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int ks = 0; ks < KT / 16; ++ks) {
                         // A = V^T: 16 keys x 128 dims of the tile; B = P^T rows of the same 16 keys
                         const uint64_t ad = umma_smem_desc(smem_u32(sm.ring[s]) + ks * 16 * 128, BOX_BYTES, 1024, 2);
-                        const uint64_t bd = umma_smem_desc(smem_u32(sm.p[0]) + (j * KT + ks * 16) * 16, 128, CH * 16, 0);
+                        const uint64_t bd = umma_smem_desc(smem_u32(sm.p[0]) + (j * KT + ks * 16) * 16, 128, C::CH * 16, 0);
                         umma_ss(tmem + C::COL_O, ad, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(smem_u32(&sm.empty[s]));
@@ -300,15 +304,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int tid = threadIdx.x;                       // key row of each tile; dim row of O^T
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         int n = 0;
-        for (long long i = blockIdx.x; next_unit(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
              i += gridDim.x, ++n) {
             const int h0 = u.kvh * G + u.hb * GT;
             bool ok = mbar_wait(smem_u32(&sm.s_full), n & 1, abort_flag, 0x301);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            uint32_t sv[TPC][NH];
+            uint32_t sv[C::TPC][NH];
 #pragma unroll
-            for (int j = 0; j < TPC; ++j)
+            for (int j = 0; j < C::TPC; ++j)
                 if (j < u.ntiles) tmem_ld<NH>(lane_base + C::COL_S + j * NH, sv[j]);
             tmem_wait_ld();
             // chunk maximum per head
@@ -317,7 +321,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int h = 0; h < GT; ++h) {
                 m[h] = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < TPC; ++j)
+                for (int j = 0; j < C::TPC; ++j)
                     if (j < u.ntiles && j * KT + tid < u.nkeys) m[h] = fmaxf(m[h], __uint_as_float(sv[j][h]));
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], o));
@@ -335,7 +339,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             // p = 2^(s * scale * log2 e - m), written as P^T rows of bf16 [key][8 heads]
 #pragma unroll
-            for (int j = 0; j < TPC; ++j) {
+            for (int j = 0; j < C::TPC; ++j) {
                 if (j >= u.ntiles) break;
                 const bool valid = j * KT + tid < u.nkeys;
                 uint32_t pk[NH / 2];
@@ -393,35 +397,63 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 }
 
-// Merge the chunks of each (b, h): M = max m_s, w_s = 2^(m_s - M),
+// Merge the chunks of each (b, h) (head dim D): M = max m_s, w_s = 2^(m_s - M),
 // O = sum w_s o_s / sum w_s l_s, LSE = (M + log2 sum w_s l_s) * ln 2.
-// One CTA per (h, b); thread i owns output dims i, i + blockDim, ...
-__global__ void __launch_bounds__(128)
+// One CTA per (h, b), 128 threads = 4 groups of 32; a group takes the
+// chunks s = g (mod 4), a lane 4 consecutive output dims per 128 (16-byte
+// loads), and the four groups' sums meet in shared memory.
+constexpr int COMBINE_THREADS = 128;
+
+__global__ void __launch_bounds__(COMBINE_THREADS)
 decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__ ws_ml,
                       const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o,
-                      float *__restrict__ lse, int n_q, int n_splits, int S_max, int chunk, int d_v) {
+                      float *__restrict__ lse, int n_q, int n_splits, int S_max, int chunk) {
+    __shared__ float red[4][D];
+    __shared__ float part[4];
     const int h = blockIdx.x, b = blockIdx.y;
+    const int tid = threadIdx.x, g = tid >> 5, lane = tid & 31;
     int seqlen = seqlens[b];
     seqlen = seqlen < 0 ? 0 : (seqlen > S_max ? S_max : seqlen);
     const int ns = (seqlen + chunk - 1) / chunk;
     const size_t row = (size_t)b * n_q + h;
     const float2 *ml = ws_ml + row * n_splits;
     if (ns == 0) {
-        for (int d = threadIdx.x; d < d_v; d += blockDim.x) o[row * d_v + d] = __float2bfloat16_rn(0.f);
-        if (threadIdx.x == 0 && lse) lse[row] = -INFINITY;
+        for (int d = tid; d < D; d += COMBINE_THREADS) o[row * D + d] = __float2bfloat16_rn(0.f);
+        if (tid == 0 && lse) lse[row] = -INFINITY;
         return;
     }
+    // M = max over chunks
     float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, ml[s].x);
+    for (int s = tid; s < ns; s += COMBINE_THREADS) M = fmaxf(M, ml[s].x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) part[g] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3]));
+    // this group's weighted sum of o_s over its chunks, and of l_s
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float L = 0.f;
-    for (int s = 0; s < ns; ++s) L += ex2(ml[s].x - M) * ml[s].y;
-    const float inv = 1.f / L;
-    for (int d = threadIdx.x; d < d_v; d += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < ns; ++s) acc += ex2(ml[s].x - M) * ws_o[(row * n_splits + s) * d_v + d];
-        o[row * d_v + d] = __float2bfloat16_rn(acc * inv);
+    const float *base = ws_o + row * n_splits * (size_t)D + lane * 4;
+#pragma unroll 4
+    for (int s = g; s < ns; s += 4) {
+        const float2 m_l = ml[s];
+        const float w = ex2(m_l.x - M);
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(base + (size_t)s * D));
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+        L = fmaf(w, m_l.y, L);
     }
-    if (threadIdx.x == 0 && lse) lse[row] = (M + log2f(L)) * 0.6931471805599453f;
+    *reinterpret_cast<float4 *>(&red[g][lane * 4]) = acc;
+    __syncthreads();   // part[] reads above are done before it is reused
+    if (lane == 0) part[g] = L;
+    __syncthreads();
+    const float Lt = part[0] + part[1] + part[2] + part[3];
+    const float inv = 1.f / Lt;
+    for (int d = tid; d < D; d += COMBINE_THREADS)
+        o[row * D + d] = __float2bfloat16_rn((red[0][d] + red[1][d] + red[2][d] + red[3][d]) * inv);
+    if (tid == 0 && lse) lse[row] = (M + log2f(Lt)) * 0.6931471805599453f;
 }
 
 }  // namespace dec

@@ -58,6 +58,7 @@ struct Smem {
     uint64_t qt_ready;                     // Q columns 0-255 copied into TMEM
     uint64_t pv_done;                      // one phase per P.V MMA group
     uint64_t o_done;
+    uint64_t tail_ready;                   // value rows past the length cleared (last tile)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -94,6 +95,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (nkeys < 0) nkeys = 0;
     const int nt = (nkeys + KT - 1) / KT;
+    const int tail = nt > 0 ? nkeys - (nt - 1) * KT : KT;   // valid rows of the last tile
 
     if (warp == 0 && lane == 0) {
         mbar_init(smem_u32(&sm.q_full), 1);
@@ -108,6 +110,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(smem_u32(&sm.qt_ready), 128);
         mbar_init(smem_u32(&sm.pv_done), 1);
         mbar_init(smem_u32(&sm.o_done), 1);
+        mbar_init(smem_u32(&sm.tail_ready), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -152,6 +155,26 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x413);
         }
         __syncwarp();
+        if (tail < KT) {
+            // Rows past the length get weight 0, but 0 * (NaN or Inf) is not
+            // 0: clear this CTA's value columns of those rows so that whatever
+            // the cache holds there cannot reach the output. Done before the
+            // last tile's MMAs are issued (they wait for tail_ready).
+            const int s = (nt - 1) % NSTAGE;
+            bool ok = mbar_wait(smem_u32(&sm.kv_full[s]), ((nt - 1) / NSTAGE) & 1, abort_flag, 0x414);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                for (int e = tail * 8 + (int)lane; e < KT * 8; e += 32) {
+                    const uint32_t off = (uint32_t)(e >> 3) * 128u + (uint32_t)(e & 7) * 16u;
+#pragma unroll
+                    for (int bx = 0; bx < 4; ++bx)
+                        sts128(smem_u32(sm.k[s][4 * rank + bx]) + off, make_uint4(0u, 0u, 0u, 0u));
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.tail_ready));
+        }
     } else if (warp == 1) {
         // ======================= MMA issuer =======================
         if (lane == 0 && nt > 0) {
@@ -206,7 +229,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             while (ok && next_pv < nt) {
                 bool progressed = false;
                 if (next_s < nt && next_s <= next_pv + 1 &&
-                    mbar_try_wait(smem_u32(&sm.kv_full[next_s % NSTAGE]), (next_s / NSTAGE) & 1)) {
+                    mbar_try_wait(smem_u32(&sm.kv_full[next_s % NSTAGE]), (next_s / NSTAGE) & 1) &&
+                    (next_s != nt - 1 || tail == KT || mbar_try_wait(smem_u32(&sm.tail_ready), 0))) {
                     issue_s(next_s);
                     ++next_s;
                     progressed = true;

@@ -9,7 +9,9 @@
 //     "Attention Engineering: From MHA to GQA, MLA & FlashAttention",
 //     section 2 (no repeat_interleave, K/V read once per group).
 //   * G = 1 (MHA): the two tiles are consecutive blocks of 128 positions.
-// Both tiles stream the same K/V tiles (128 keys each) through a 2-stage ring.
+// Both tiles stream the same K/V tiles (128 keys each): K through a 2-stage
+// and V through a 3-stage ring, each fed by its own TMA warp; one MMA commit
+// per iteration releases a V tile and the next K tile together.
 //
 // Per K/V tile j and query tile t the recurrence of the same page, section 4
 // (FlashAttention-2 tiled rescaling) runs as:
@@ -30,9 +32,10 @@
 // the tensor core runs the other tile's MMAs. Epilogue: O / l -> bf16 ->
 // swizzled shared memory -> TMA store; LSE = (m + log2 l) * ln 2.
 //
-// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// warps 4-7 and 8-11 the softmax / epilogue warpgroups of tiles 0 and 1
-// (warp w reads TMEM lanes 32*(w%4) .. +31, so each warpgroup covers 128 rows).
+// Roles (384 threads): warps 0 and 2 TMA producers (Q and K; V), warp 1 MMA
+// issuer and TMEM owner, warps 4-7 and 8-11 the softmax / epilogue
+// warpgroups of tiles 0 and 1 (warp w reads TMEM lanes 32*(w%4) .. +31, so
+// each warpgroup covers 128 rows).
 #pragma once
 
 #include "sm100.cuh"
@@ -42,11 +45,18 @@ namespace pf {
 
 constexpr int BM = 128;        // query rows per tile (MMA M)
 constexpr int BN = 128;        // keys per K/V tile (MMA N of Q K^T)
-constexpr int NSTAGE = 2;
+constexpr int KSTAGE = 2;       // K ring depth
+constexpr int VSTAGE = 3;       // V ring depth
+// One release barrier per K/V iteration i, completed by a single MMA commit
+// once both tiles' P V of tile i and Q K^T of tile i+1 are done (this frees
+// V tile i and K tile i+1). NREL >= max(KSTAGE, VSTAGE) keeps every producer
+// within one phase of the barrier it waits on.
+constexpr int NREL = 3;
+static_assert(NREL >= KSTAGE && NREL >= VSTAGE, "release ring too short");
 constexpr int THREADS = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only past a 256x growth
 #ifndef ATTN_PF_P_CHUNKS
-#define ATTN_PF_P_CHUNKS 2
+#define ATTN_PF_P_CHUNKS 1
 #endif
 #ifndef ATTN_PF_POLY_EVERY
 #define ATTN_PF_POLY_EVERY 0
@@ -84,11 +94,11 @@ struct Cfg {
 template <int D>
 struct Smem {
     uint8_t q[2][Cfg<D>::QBYTES];          // Q tiles; reused as O staging in the epilogue
-    uint8_t k[NSTAGE][Cfg<D>::KBYTES];
-    uint8_t v[NSTAGE][Cfg<D>::KBYTES];
+    uint8_t k[KSTAGE][Cfg<D>::KBYTES];
+    uint8_t v[VSTAGE][Cfg<D>::KBYTES];
     uint64_t q_full;
-    uint64_t kv_full[NSTAGE];
-    uint64_t kv_empty[NSTAGE];
+    uint64_t k_full[KSTAGE], v_full[VSTAGE];
+    uint64_t rel[NREL];
     uint64_t s_full[2];
     uint64_t p_full[2][kPChunks];  // one per hand-off chunk of P
     uint64_t o_done[2];
@@ -113,6 +123,11 @@ struct Params {
     int causal;
     float scale_log2;      // scale * log2(e)
     float *lse;            // may be null
+};
+
+template <bool B>
+struct BoolTag {
+    static constexpr bool value = B;
 };
 
 // All 32 lanes wait; the outcome is made warp-uniform.
@@ -162,9 +177,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ---- setup: barriers (warp 0), TMEM (warp 1)
     if (warp == 0 && lane == 0) {
         mbar_init(smem_u32(&sm.q_full), 1);
-        for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(smem_u32(&sm.kv_full[s]), 1);
-            mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+        for (int s = 0; s < KSTAGE; ++s) mbar_init(smem_u32(&sm.k_full[s]), 1);
+        for (int s = 0; s < VSTAGE; ++s) mbar_init(smem_u32(&sm.v_full[s]), 1);
+        for (int s = 0; s < NREL; ++s) {
+            mbar_init(smem_u32(&sm.rel[s]), 1);
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&sm.s_full[t]), 1);
@@ -209,26 +225,49 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
                                 b * p.n_q + h0[t]);
             }
+            // K tiles (V tiles are loaded by warp 2)
             int issued = 0;
             for (int j = 0; j < nmax; ++j) {
-                const int s = j % NSTAGE;
-                if (j >= NSTAGE &&
-                    !mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / NSTAGE) + 1) & 1, abort_flag, 0x11))
+                const int s = j % KSTAGE;
+                // K tile j - KSTAGE is free once iteration j - KSTAGE - 1 is released
+                // (K tile 0 with iteration 0)
+                const int it = j - KSTAGE - 1 < 0 ? 0 : j - KSTAGE - 1;
+                if (j >= KSTAGE &&
+                    !mbar_wait(smem_u32(&sm.rel[it % NREL]), (it / NREL) & 1, abort_flag, 0x11))
                     break;
-                const uint32_t fb = smem_u32(&sm.kv_full[s]);
-                mbar_arrive_expect_tx(fb, 2 * C::KBYTES);
-                for (int bx = 0; bx < C::NBOX; ++bx) {
+                const uint32_t fb = smem_u32(&sm.k_full[s]);
+                mbar_arrive_expect_tx(fb, C::KBYTES);
+                for (int bx = 0; bx < C::NBOX; ++bx)
                     tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, j * BN,
                                 b * p.n_kv + kvh);
-                    tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, j * BN,
-                                b * p.n_kv + kvh);
-                }
                 ++issued;
             }
             // never leave copies in flight into this CTA's shared memory
             mbar_wait(qbar, 0, nullptr, 0x12);
-            for (int j = issued - 1; j >= 0 && j >= issued - NSTAGE; --j)
-                mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x13);
+            for (int j = issued - 1; j >= 0 && j >= issued - KSTAGE; --j)
+                mbar_wait(smem_u32(&sm.k_full[j % KSTAGE]), (j / KSTAGE) & 1, nullptr, 0x13);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ======================= TMA producer (V tiles) =======================
+        if (lane == 0) {
+            int issued = 0;
+            for (int j = 0; j < nmax; ++j) {
+                const int s = j % VSTAGE;
+                // V tile j - VSTAGE is free once iteration j - VSTAGE is released
+                const int it = j - VSTAGE;
+                if (j >= VSTAGE &&
+                    !mbar_wait(smem_u32(&sm.rel[it % NREL]), (it / NREL) & 1, abort_flag, 0x14))
+                    break;
+                const uint32_t fb = smem_u32(&sm.v_full[s]);
+                mbar_arrive_expect_tx(fb, C::KBYTES);
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, j * BN,
+                                b * p.n_kv + kvh);
+                ++issued;
+            }
+            for (int j = issued - 1; j >= 0 && j >= issued - VSTAGE; --j)
+                mbar_wait(smem_u32(&sm.v_full[j % VSTAGE]), (j / VSTAGE) & 1, nullptr, 0x15);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -238,7 +277,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t idesc_o = umma_idesc_bf16(BM, D, 0, 1);
             bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x21);
             auto issue_s = [&](int t, int j) {
-                const int s = j % NSTAGE;
+                const int s = j % KSTAGE;
                 const uint32_t qa = smem_u32(sm.q[t]);
                 const uint32_t ka = smem_u32(sm.k[s]);
 #pragma unroll
@@ -255,7 +294,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // O_t += P_t V_j, 32 keys at a time as soon as the softmax
             // warpgroup has written that chunk of P
             auto issue_pv = [&](int t, int j) -> bool {
-                const int s = j % NSTAGE;
+                const int s = j % VSTAGE;
                 const uint32_t va = smem_u32(sm.v[s]);
 #pragma unroll
                 for (int c = 0; c < kPChunks; ++c) {
@@ -269,11 +308,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 (j > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
-                umma_commit(smem_u32(&sm.o_done[t]));
+                if (j == nt[t] - 1) umma_commit(smem_u32(&sm.o_done[t]));   // O_t final
                 return true;
             };
             if (ok && nmax > 0) {
-                ok = mbar_wait(smem_u32(&sm.kv_full[0]), 0, abort_flag, 0x22);
+                ok = mbar_wait(smem_u32(&sm.k_full[0]), 0, abort_flag, 0x22);
                 if (ok) {
                     tc_fence_after();
                     for (int t = 0; t < 2; ++t)
@@ -281,19 +320,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             for (int j = 0; ok && j < nmax; ++j) {
+                // operands of this iteration (V tile j, K tile j+1), checked up
+                // front so that no wait sits between the MMA groups below
+                ok = mbar_wait(smem_u32(&sm.v_full[j % VSTAGE]), (j / VSTAGE) & 1, abort_flag, 0x26);
+                if (ok && j + 1 < nmax)
+                    ok = mbar_wait(smem_u32(&sm.k_full[(j + 1) % KSTAGE]), ((j + 1) / KSTAGE) & 1, abort_flag,
+                                   0x24);
+                tc_fence_after();
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j >= nt[t]) continue;
                     ok = issue_pv(t, j);
                     if (!ok) break;
-                    if (j + 1 < nt[t]) {
-                        ok = mbar_wait(smem_u32(&sm.kv_full[(j + 1) % NSTAGE]), ((j + 1) / NSTAGE) & 1,
-                                       abort_flag, 0x24);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_s(t, j + 1);
-                    }
+                    if (j + 1 < nt[t]) issue_s(t, j + 1);
                 }
-                umma_commit(smem_u32(&sm.kv_empty[j % NSTAGE]));
+                // P V of tile j and Q K^T of tile j+1 issued for both tiles
+                umma_commit(smem_u32(&sm.rel[j % NREL]));
             }
             // all MMAs of this CTA done before TMEM can be released
             umma_commit(smem_u32(&sm.mma_done));
@@ -373,8 +414,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     m_run = m_new;
                 }
                 // P = 2^(s*scale*log2e - m) -> bf16 pairs over the first half of S,
-                // handed to the MMA warp in kPChunks pieces so that P.V starts on
-                // the first keys while later ones are still exponentiated.
+                // handed to the MMA warp in kPChunks pieces (kPChunks > 1 lets P.V
+                // start on the first keys while later ones are still
+                // exponentiated; measured on B200 one hand-off is faster, the
+                // extra barrier round trips cost more than the overlap gains).
                 // Optionally (kPolyEvery > 0) part of the exponentials run on the
                 // FMA pipe (ex2_poly2) beside the special-function unit; measured
                 // on B200 this is slower for head dim 128 (the softmax is bound
@@ -382,20 +425,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // is off by default.
                 const float2 nm2 = make_float2(-m_run, -m_run);
                 float2 rs = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int c = 0; c < kPChunks; ++c) {
-                    uint32_t pk[kChunkKeys / 2];
+                // one chunk of exponentials; which pairs take the FMA-pipe
+                // polynomial is fixed at compile time (never on masked tiles)
+                auto exp_chunk = [&](auto poly_on, int c, uint32_t(&pk)[kChunkKeys / 2]) {
 #pragma unroll
                     for (int e = 0; e < kChunkKeys / 2; ++e) {
                         const int i0 = c * kChunkKeys + 2 * e;
                         const float2 t2 = ffma2(make_float2(__uint_as_float(x[i0]), __uint_as_float(x[i0 + 1])),
                                                 sl2, nm2);
-                        const bool poly = kPolyEvery > 0 && !masked && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) ==
-                                                                         (kPolyEvery > 0 ? kPolyEvery - 1 : 0);
-                        const float2 pe = poly ? ex2_poly2(t2) : make_float2(ex2(t2.x), ex2(t2.y));
+                        float2 pe;
+                        if constexpr (decltype(poly_on)::value && kPolyEvery > 0) {
+                            if (e % (kPolyEvery > 0 ? kPolyEvery : 1) == (kPolyEvery > 0 ? kPolyEvery - 1 : 0))
+                                pe = ex2_poly2(t2);
+                            else
+                                pe = make_float2(ex2(t2.x), ex2(t2.y));
+                        } else {
+                            pe = make_float2(ex2(t2.x), ex2(t2.y));
+                        }
                         rs = fadd2(rs, pe);
                         pk[e] = f2_to_bf2(pe.x, pe.y);
                     }
+                };
+#pragma unroll
+                for (int c = 0; c < kPChunks; ++c) {
+                    uint32_t pk[kChunkKeys / 2];
+                    if (masked || kPolyEvery == 0)
+                        exp_chunk(BoolTag<false>{}, c, pk);
+                    else
+                        exp_chunk(BoolTag<true>{}, c, pk);
 #pragma unroll
                     for (int q = 0; q < kChunkKeys / 64; ++q)
                         tmem_st32(trow + colS + c * (kChunkKeys / 2) + 32 * q,
@@ -409,7 +466,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 l_run += rs.x + rs.y;
             }
             // ---- epilogue: O / l -> bf16 -> swizzled smem -> TMA store; LSE
-            if (ok) ok = warp_wait(smem_u32(&sm.o_done[t]), (nt[t] - 1) & 1, abort_flag, 0x33);
+            if (ok) ok = warp_wait(smem_u32(&sm.o_done[t]), 0, abort_flag, 0x33);
             __syncwarp();
             tc_fence_after();
             const float inv_l = 1.f / l_run;

@@ -46,6 +46,23 @@ def test_mla_ragged(seqlens):
             assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
 
 
+def test_mla_ignores_nonfinite_rows_past_the_length():
+    """Latent rows at or beyond a sequence's length hold NaN and +Inf, inside
+    the same 64-row tile as valid rows: the result must equal the oracle's on
+    the valid rows."""
+    seqlens = [1, 100, 4000]
+    B, S_max = len(seqlens), 4096
+    sl = torch.tensor(seqlens, dtype=torch.int32)
+    g = torch.Generator(device="cuda").manual_seed(17)
+    q = torch.randn(B, 128, 576, generator=g, device="cuda").to(torch.bfloat16)
+    cache = torch.randn(B, S_max, 576, generator=g, device="cuda").to(torch.bfloat16)
+    for b, L in enumerate(seqlens):
+        cache[b, L:, :288] = float("nan")
+        cache[b, L:, 288:] = float("inf")
+    o, lse = _run(sl, q, cache, 1 / math.sqrt(192), "mla non-finite rows past the length")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
 def test_mla_two_head_blocks_and_padded_rows():
     """256 heads (two 128-head tiles) and a cache whose rows are padded to 640."""
     binding = need_gpu()
