@@ -404,13 +404,20 @@ def run_ours(args):
                    "frac_of_peak": dec_achieved / peak_bw, "frac_of_nominal_8000": dec_achieved / 8000.0,
                    "algorithmic_bytes": by_d, "algorithmic_flops": fl_d,
                    "kernels": "attn::dec::decode_split_kernel<4> + decode_combine_kernel",
-                   "peak": peak_bw, "peak_source": f"{peak_src} hbm_gbs"},
+                   "peak": peak_bw, "peak_source": f"{peak_src} hbm_gbs",
+                   "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak_bw, "unit": "GB/s",
+                                "frac": dec_achieved / peak_bw, "traffic": traffic.get("decode_split_kernel_4"),
+                                "note": "achieved over split + merge launches; traffic of the split kernel"}},
         "mla_decode": {"workload": wm.name, "ms": mean_m, "gbs": by_m / (mean_m / 1e3) / 1e9,
                        "tflops": fl_m / (mean_m / 1e3) / 1e12,
                        "frac_of_peak_hbm": by_m / (mean_m / 1e3) / 1e9 / peak_bw,
                        "roofline_frac": max(by_m / (peak_bw * 1e9), fl_m / (peak_tf * 1e12)) / (mean_m / 1e3),
                        "algorithmic_bytes": by_m, "algorithmic_flops": fl_m,
-                       "kernel": "attn::mla::mla_decode_kernel (2-CTA cluster)"},
+                       "kernel": "attn::mla::mla_decode_kernel (2-CTA cluster)",
+                       "roofline": {"bound": "hbm", "achieved": by_m / (mean_m / 1e3) / 1e9, "peak": peak_bw,
+                                    "unit": "GB/s", "frac": by_m / (mean_m / 1e3) / 1e9 / peak_bw,
+                                    "traffic": traffic.get("mla_decode_kernel"),
+                                    "tensor_frac": fl_m / (mean_m / 1e3) / 1e12 / peak_tf}},
     }
 
     cpu_baseline = None
