@@ -294,8 +294,32 @@ def run_ours(args):
     do_p = args.only in ("all", "prefill")
     do_d = args.only in ("all", "decode")
     do_m = args.only in ("all", "mla")
+    do_g = args.only in ("all", "paged")
 
-    def step(times_p, times_d, times_m=None):
+    # the GQA decode workload again, its cache cut into 64-token pages placed
+    # in a pool in a seeded random order (the paged-cache serving layout)
+    PAGE = 64
+    if do_g:
+        P = wd.Skv // PAGE
+        npg = (seqlens.long() + PAGE - 1) // PAGE
+        b_idx = torch.repeat_interleave(torch.arange(wd.B), npg)
+        p_idx = torch.cat([torch.arange(int(n)) for n in npg])
+        perm = torch.randperm(len(b_idx), generator=torch.Generator().manual_seed(wd.seed + 77))
+        table = torch.zeros(wd.B, P, dtype=torch.int32)
+        table[b_idx, p_idx] = perm.to(torch.int32)
+        table_dev = table.to(dev)
+        pool_k = torch.empty(len(b_idx), PAGE, wd.n_kv, wd.d_qk, dtype=torch.bfloat16, device=dev)
+        pool_v = torch.empty_like(pool_k)
+        kview = kc.view(wd.B, wd.n_kv, P, PAGE, wd.d_qk).permute(0, 2, 3, 1, 4)
+        vview = vc.view(wd.B, wd.n_kv, P, PAGE, wd.d_v).permute(0, 2, 3, 1, 4)
+        pid_dev, b_dev, p_dev = perm.to(dev), b_idx.to(dev), p_idx.to(dev)
+        pool_k[pid_dev] = kview[b_dev, p_dev]
+        pool_v[pid_dev] = vview[b_dev, p_dev]
+        del pid_dev, b_dev, p_dev
+        og = torch.empty_like(od)
+        lg = torch.empty_like(ld)
+
+    def step(times_p, times_d, times_m=None, times_g=None):
         if do_p:
             cold_l2(1.0)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -320,6 +344,15 @@ def run_ours(args):
             e5.record(stream)
             if times_m is not None:
                 times_m.append((e4, e5))
+        if do_g:
+            cold_l2(4.0)
+            e6, e7 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e6.record(stream)
+            binding.attn_decode_paged(qd, pool_k, pool_v, table_dev, sl_dev, wd.scale, o=og, lse=lg,
+                                      workspace=work, stream=stream)
+            e7.record(stream)
+            if times_g is not None:
+                times_g.append((e6, e7))
 
     def barrier():
         if ws > 1:
@@ -332,12 +365,12 @@ def run_ours(args):
     barrier()
     assert binding.device_status(stream) == 0, "device status not clean after warm-up"
 
-    tp, td, tm = [], [], []
+    tp, td, tm, tg = [], [], [], []
     with ClockSampler(torch.cuda.current_device()) as clocks:
         barrier()
         t_wall0 = time.perf_counter()
         for _ in range(args.steps):
-            step(tp, td, tm)
+            step(tp, td, tm, tg)
         barrier()
         t_wall = time.perf_counter() - t_wall0
     st = binding.device_status(stream)
@@ -345,6 +378,8 @@ def run_ours(args):
     ms_p = [a.elapsed_time(b) for a, b in tp] or [float("nan")]
     ms_d = [a.elapsed_time(b) for a, b in td] or [float("nan")]
     ms_m = [a.elapsed_time(b) for a, b in tm] or [float("nan")]
+    ms_g = [a.elapsed_time(b) for a, b in tg] or [float("nan")]
+    mean_g = sum(ms_g) / len(ms_g)
     mean_m = sum(ms_m) / len(ms_m)
     mean_p = sum(ms_p) / len(ms_p)
     mean_d = sum(ms_d) / len(ms_d)
@@ -418,6 +453,10 @@ def run_ours(args):
                                     "unit": "GB/s", "frac": by_m / (mean_m / 1e3) / 1e9 / peak_bw,
                                     "traffic": traffic.get("mla_decode_kernel"),
                                     "tensor_frac": fl_m / (mean_m / 1e3) / 1e12 / peak_tf}},
+        "paged_decode": {"workload": f"{wd.name}, {PAGE}-token pages in a shuffled pool", "ms": mean_g,
+                         "gbs": by_d / (mean_g / 1e3) / 1e9, "frac_of_peak": by_d / (mean_g / 1e3) / 1e9 / peak_bw,
+                         "algorithmic_bytes": by_d,
+                         "kernels": "attn::dec::decode_split_kernel<4, paged> + decode_combine_kernel"},
     }
 
     cpu_baseline = None
@@ -442,7 +481,7 @@ def run_ours(args):
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
             "clocks": clocks.summary(),
-            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m)) * args.steps,
+            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m) + 2 * int(do_g)) * args.steps,
             "wall_s_timed_region": t_wall,
         }
         print(json.dumps(line), flush=True)
@@ -471,7 +510,7 @@ def main():
                     help="query rows of the headline workload per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla", "paged"],
                     help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -111,7 +111,8 @@ int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int
  *           none is needed (0 bytes; the pointer may be NULL).
  * Supported: (d_qk, d_v) = (128, 128) with n_q / n_kv in {1, 2, 4, 8, 16, ...}
  * (any power of two); (576, 512) with n_kv = 1 (MLA absorbed decode, the
- * scale usually 1/sqrt(128 + 64)).
+ * scale usually 1/sqrt(128 + 64)). Cache rows at or past a sequence's length
+ * may hold anything (NaN and Inf included): they never reach the result.
  */
 int attn_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
                 void *o, float *lse,
@@ -119,6 +120,48 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
                 int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
                 int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
                 float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_decode_paged -- attn_decode against a paged KV cache.
+ * Source: "Attention deep dive" (askaiml.pages.dev), section 5 (production
+ * engines keep the KV cache in fixed-size pages addressed through a page
+ * table, so sequences of different lengths share one pool); "2.4 Multi-Head
+ * Attention, MQA, GQA & MLA", GQA in libraries (serving engines size their
+ * paged KV blocks by the number of KV heads). The attention computed is that
+ * of attn_decode; only where cached token j of sequence b lives changes.
+ *
+ *   q        [B, n_q, 128] bf16, contiguous
+ *   k_pages  element (page p, token t of the page, kv head g, dim c) at
+ *            k_pages[p*k_stride_page + t*k_stride_token + g*k_stride_head + c]
+ *            (strides in ELEMENTS, multiples of 8, token stride >= 128; the
+ *            common pool layout [num_pages][page_size][n_kv][128] has strides
+ *            (page_size*n_kv*128, n_kv*128, 128))
+ *   v_pages  the same for values (may alias k_pages with other strides)
+ *   block_table [B, pages_per_seq] int32, device: logical token j of
+ *            sequence b is token j % page_size of page
+ *            block_table[b*pages_per_seq + j / page_size]. Only the entries
+ *            covering tokens 0 .. seqlens[b]-1 are read. A page id outside
+ *            [0, num_pages) reads as zeros and is reported as
+ *            ATTN_ERR_DEVICE_RANGE (by attn_device_status).
+ *   seqlens  [B] int32, device; values above pages_per_seq*page_size are
+ *            clamped (reported as ATTN_ERR_DEVICE_RANGE); 0 gives O = 0,
+ *            LSE = -inf
+ *   o, lse   as attn_decode
+ *   workspace: at least attn_decode_workspace_bytes(B, n_q, n_kv, 128, 128,
+ *            pages_per_seq * page_size) bytes, 256-byte aligned, caller-owned.
+ * Supported: d_qk = d_v = 128, n_q / n_kv a power of two, page_size in
+ * {16, 32, 64} or a power of two that is a multiple of 128. Cache rows past a
+ * sequence's length may hold anything (NaN and Inf included): they never
+ * reach the result. Returns ATTN_OK or an error code (nothing launched on
+ * error).
+ */
+int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
+                      const int32_t *seqlens, void *o, float *lse,
+                      int B, int n_q, int n_kv, int d_qk, int d_v,
+                      int page_size, int pages_per_seq, int num_pages,
+                      int64_t k_stride_page, int64_t k_stride_token, int64_t k_stride_head,
+                      int64_t v_stride_page, int64_t v_stride_token, int64_t v_stride_head,
+                      float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device

@@ -57,6 +57,9 @@ def lib() -> ctypes.CDLL:
         L.attn_decode.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 +
                                   [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode.restype = _i
+        L.attn_decode_paged.argtypes = ([_vp] * 7 + [_i] * 8 + [_i64] * 6 +
+                                        [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_decode_paged.restype = _i
         L.attn_status_string.argtypes = [_i]
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_device_status.argtypes = [_vp]
@@ -117,8 +120,10 @@ def decode_workspace_bytes(B, n_q, n_kv, d_qk, d_v, S_max) -> int:
 
 
 def _elem_strides(t):
+    """Element strides of the three outer dimensions of a 4-D cache or page
+    pool whose innermost dimension is unit-stride."""
     if t.dim() != 4 or t.stride(3) != 1:
-        raise ValueError("cache must be 4-D [B, n_kv, S_max, row] with unit inner stride")
+        raise ValueError("cache must be 4-D with a unit inner stride")
     return t.stride(0), t.stride(1), t.stride(2)
 
 
@@ -146,6 +151,35 @@ def attn_decode(q, kcache, vcache, seqlens, scale: float, d_v=None, o=None, lse=
                            B, n_q, n_kv, d_qk, d_v, S_max, *ks, *vs, float(scale),
                            _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_decode")
+    return o, lse
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float, o=None, lse=None, workspace=None,
+                      stream=None, want_lse=True):
+    """Decode against a paged cache. q [B,n_q,128]; k_pages/v_pages indexed
+    [page, token in page, kv head, dim] (any strides with a unit inner
+    stride); block_table int32 [B, pages_per_seq] and seqlens int32 [B] on the
+    device. Returns (o, lse)."""
+    B, n_q, d = q.shape
+    num_pages, page_size, n_kv, _ = k_pages.shape
+    pages_per_seq = block_table.shape[1]
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    for t in (block_table, seqlens):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("block_table and seqlens must be contiguous int32 CUDA tensors")
+    ks, vs = _elem_strides(k_pages), _elem_strides(v_pages)
+    if o is None:
+        o = torch.empty((B, n_q, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, n_q, n_kv, d, d, page_size * pages_per_seq)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens), _ptr(o),
+                                 _ptr(lse), B, n_q, n_kv, d, d, page_size, pages_per_seq, num_pages, *ks, *vs,
+                                 float(scale), _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_decode_paged")
     return o, lse
 
 

@@ -176,10 +176,19 @@ size_t decode_ws_bytes(int B, int n_q, int d_v, int n_splits) {
     return o_bytes + rows * sizeof(float2);
 }
 
-template <int GT>
-int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32_t *seqlens, void *o, float *lse,
-                      int B, int n_q, int n_kv, int S_max, const int64_t *ks, const int64_t *vs, float scale,
-                      void *ws, cudaStream_t stream) {
+// Cache addressing of one decode launch: a contiguous cache
+// [B][n_kv][S_max][row] (element strides ks/vs = b, head, token) or a page
+// pool [num_pages][page_size][n_kv][row] (strides = page, token, head).
+struct CacheView {
+    const void *k, *v;
+    int64_t ks[3], vs[3];              // element strides, outermost first
+    attn::dec::PageTable pt;           // pt.table == nullptr: contiguous
+    int page_size;
+};
+
+template <int GT, bool PAGED>
+int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens, void *o, float *lse, int B,
+                      int n_q, int n_kv, int S_max, float scale, void *ws, cudaStream_t stream) {
     using namespace attn::dec;
     using C = Cfg<GT>;
     const int G = n_q / n_kv;
@@ -193,15 +202,26 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
         const uint32_t box[3] = {64u, (uint32_t)C::NH, 1u};
         if (!make_map(&tq, q, 3, dims, str, box, 128)) return ATTN_ERR_CUDA;
     }
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S_max, (uint64_t)n_kv, (uint64_t)B};
-    const uint32_t box[4] = {64u, (uint32_t)KT, 1u, 1u};
-    const uint64_t kstr[3] = {(uint64_t)ks[2] * 2, (uint64_t)ks[1] * 2, (uint64_t)ks[0] * 2};
-    const uint64_t vstr[3] = {(uint64_t)vs[2] * 2, (uint64_t)vs[1] * 2, (uint64_t)vs[0] * 2};
-    if (!make_map(&tk, kc, 4, dims, kstr, box, 128)) return ATTN_ERR_CUDA;
-    if (!make_map(&tv, vc, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
+    if (PAGED) {
+        // [dim][token in page][kv head][page]
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)cv.page_size, (uint64_t)n_kv, (uint64_t)cv.pt.num_pages};
+        const uint32_t box[4] = {64u, (uint32_t)cv.pt.box_rows, 1u, 1u};
+        const uint64_t kstr[3] = {(uint64_t)cv.ks[1] * 2, (uint64_t)cv.ks[2] * 2, (uint64_t)cv.ks[0] * 2};
+        const uint64_t vstr[3] = {(uint64_t)cv.vs[1] * 2, (uint64_t)cv.vs[2] * 2, (uint64_t)cv.vs[0] * 2};
+        if (!make_map(&tk, cv.k, 4, dims, kstr, box, 128)) return ATTN_ERR_CUDA;
+        if (!make_map(&tv, cv.v, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
+    } else {
+        // [dim][token][kv head][sequence]
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S_max, (uint64_t)n_kv, (uint64_t)B};
+        const uint32_t box[4] = {64u, (uint32_t)KT, 1u, 1u};
+        const uint64_t kstr[3] = {(uint64_t)cv.ks[2] * 2, (uint64_t)cv.ks[1] * 2, (uint64_t)cv.ks[0] * 2};
+        const uint64_t vstr[3] = {(uint64_t)cv.vs[2] * 2, (uint64_t)cv.vs[1] * 2, (uint64_t)cv.vs[0] * 2};
+        if (!make_map(&tk, cv.k, 4, dims, kstr, box, 128)) return ATTN_ERR_CUDA;
+        if (!make_map(&tv, cv.v, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
+    }
     const size_t smem = smem_bytes<GT>();
     static uint64_t attr_done = 0;
-    if (!ensure_smem_attr(decode_split_kernel<GT>, smem, attr_done)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(decode_split_kernel<GT, PAGED>, smem, attr_done)) return ATTN_ERR_CUDA;
     float *ws_o = reinterpret_cast<float *>(ws);
     size_t o_bytes = (size_t)B * n_q * n_splits * D * sizeof(float);
     o_bytes = (o_bytes + 255) & ~size_t(255);
@@ -212,12 +232,24 @@ int launch_decode_gqa(const void *q, const void *kc, const void *vc, const int32
     if (n_sm <= 0) return ATTN_ERR_CUDA;
     const long long max_units = (long long)B * n_kv * n_hb * n_splits;
     const int grid = (int)(max_units < 2LL * n_sm ? max_units : 2LL * n_sm);
-    decode_split_kernel<GT><<<grid, THREADS, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q, n_kv, G,
-                                                             n_hb, S_max, n_splits, scale_log2);
+    decode_split_kernel<GT, PAGED><<<grid, THREADS, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q, n_kv,
+                                                                    G, n_hb, S_max, n_splits, scale_log2, cv.pt);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
         ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH);
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <bool PAGED>
+int dispatch_decode_gqa(int G, const void *q, const CacheView &cv, const int32_t *seqlens, void *o, float *lse,
+                        int B, int n_q, int n_kv, int S_max, float scale, void *ws, cudaStream_t s) {
+    switch (decode_head_block(G)) {
+        case 1: return launch_decode_gqa<1, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 2: return launch_decode_gqa<2, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 4: return launch_decode_gqa<4, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 8: return launch_decode_gqa<8, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        default: return launch_decode_gqa<16, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -351,15 +383,12 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(G, S_max));
         if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
-        const int64_t ks[3] = {k_stride_b, k_stride_h, k_stride_s};
-        const int64_t vs[3] = {v_stride_b, v_stride_h, v_stride_s};
-        switch (decode_head_block(G)) {
-            case 1: return launch_decode_gqa<1>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
-            case 2: return launch_decode_gqa<2>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
-            case 4: return launch_decode_gqa<4>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
-            case 8: return launch_decode_gqa<8>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
-            default: return launch_decode_gqa<16>(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, S_max, ks, vs, scale, workspace, s);
-        }
+        CacheView cv{};
+        cv.k = kcache;
+        cv.v = vcache;
+        cv.ks[0] = k_stride_b, cv.ks[1] = k_stride_h, cv.ks[2] = k_stride_s;
+        cv.vs[0] = v_stride_b, cv.vs[1] = v_stride_h, cv.vs[2] = v_stride_s;
+        return dispatch_decode_gqa<false>(G, q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, workspace, s);
     }
     if (d_qk == 576 && d_v == 512 && n_kv == 1) {
         // the value rows must be the first 512 columns of the key rows
@@ -372,6 +401,53 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         return launch_decode_mla(q, kcache, seqlens, o, lse, B, n_q, S_max, k_stride_b, k_stride_s, scale, s);
     }
     return ATTN_ERR_UNSUPPORTED;
+}
+
+int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
+                      const int32_t *seqlens, void *o, float *lse, int B, int n_q, int n_kv, int d_qk, int d_v,
+                      int page_size, int pages_per_seq, int num_pages, int64_t k_stride_page,
+                      int64_t k_stride_token, int64_t k_stride_head, int64_t v_stride_page, int64_t v_stride_token,
+                      int64_t v_stride_head, float scale, void *workspace, size_t workspace_bytes,
+                      attn_stream_t stream) {
+    if (B < 0 || n_q < 1 || n_kv < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (page_size < 1 || pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if ((long long)page_size * pages_per_seq > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    if (B == 0) return ATTN_OK;
+    if (!q || !k_pages || !v_pages || !block_table || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (k_stride_page < 0 || k_stride_token < 0 || k_stride_head < 0 || v_stride_page < 0 || v_stride_token < 0 ||
+        v_stride_head < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
+    // a page is whole TMA boxes of up to 128 rows: 16, 32, 64 or a multiple of 128 tokens
+    if (!(page_size == 16 || page_size == 32 || page_size == 64 || (page_size % 128 == 0 && is_pow2(page_size))))
+        return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G)) return ATTN_ERR_UNSUPPORTED;
+    if (k_stride_token < 128 || v_stride_token < 128) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+    if ((k_stride_page | k_stride_token | k_stride_head | v_stride_page | v_stride_token | v_stride_head) & 7)
+        return ATTN_ERR_MISALIGNED;
+    const int S_max = page_size * pages_per_seq;
+    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(G, S_max));
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+    CacheView cv{};
+    cv.k = k_pages;
+    cv.v = v_pages;
+    cv.ks[0] = k_stride_page, cv.ks[1] = k_stride_token, cv.ks[2] = k_stride_head;
+    cv.vs[0] = v_stride_page, cv.vs[1] = v_stride_token, cv.vs[2] = v_stride_head;
+    cv.page_size = page_size;
+    cv.pt.table = block_table;
+    cv.pt.pages_per_seq = pages_per_seq;
+    int shift = 0;
+    while ((1 << shift) < page_size) ++shift;
+    cv.pt.page_shift = shift;
+    cv.pt.box_rows = page_size < attn::dec::KT ? page_size : attn::dec::KT;
+    cv.pt.num_pages = num_pages;
+    return dispatch_decode_gqa<true>(G, q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, workspace,
+                                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char *attn_status_string(int status) {

@@ -97,6 +97,18 @@ struct Unit {
     int b, kvh, hb, split, key0, nkeys, ntiles;
 };
 
+// Paged cache: logical key t of sequence b sits in row t % page_size of page
+// table[b * pages_per_seq + t / page_size] of a page pool; the K and V tensor
+// maps then address [page][token][kv head][dim] (any strides). A 128-key tile
+// is KT / box_rows TMA boxes, box_rows = min(page_size, KT).
+struct PageTable {
+    const int32_t *table;   // [B][pages_per_seq]; null: contiguous cache
+    int pages_per_seq;
+    int page_shift;         // log2(page_size)
+    int box_rows;
+    int num_pages;
+};
+
 __device__ __forceinline__ int clamp_seqlen(const int32_t *seqlens, int b, int S_max) {
     int L = seqlens[b];
     return L < 0 ? 0 : (L > S_max ? S_max : L);
@@ -131,12 +143,12 @@ __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const in
     return false;
 }
 
-template <int GT>
+template <int GT, bool PAGED>
 __global__ void __launch_bounds__(THREADS, 2)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
                     float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
-                    int S_max, int n_splits, float scale_log2) {
+                    int S_max, int n_splits, float scale_log2, const PageTable pt) {
     using C = Cfg<GT>;
     constexpr int NH = C::NH;
     extern __shared__ uint8_t smem_raw[];
@@ -203,12 +215,32 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         break;
                     }
                     const uint32_t full = smem_u32(&sm.full[s]);
-                    mbar_arrive_expect_tx(full, TILE_BYTES);
                     const CUtensorMap *tm = (j < u.ntiles) ? &tm_k : &tm_v;
                     const int krow = u.key0 + (j < u.ntiles ? j : j - u.ntiles) * KT;
                     const uint32_t dst = smem_u32(sm.ring[s]);
-                    tma_load_4d(dst, tm, full, 0, krow, u.kvh, u.b);
-                    tma_load_4d(dst + BOX_BYTES, tm, full, 64, krow, u.kvh, u.b);
+                    if constexpr (PAGED) {
+                        // boxes holding at least one key below the length; rows of
+                        // the tile past them are never read as valid keys (their
+                        // scores are masked and their value rows cleared)
+                        const int kend = u.key0 + u.nkeys;
+                        const int nbox = min(KT / pt.box_rows, (kend - krow + pt.box_rows - 1) / pt.box_rows);
+                        const uint32_t box_bytes = (uint32_t)pt.box_rows * 128u;
+                        mbar_arrive_expect_tx(full, 2u * box_bytes * (uint32_t)nbox);
+                        const int32_t *row_pages = pt.table + (size_t)u.b * pt.pages_per_seq;
+                        for (int x = 0; x < nbox; ++x) {
+                            const int key = krow + x * pt.box_rows;
+                            const int page = row_pages[key >> pt.page_shift];
+                            // a page id outside the pool reads zeros (TMA bounds) and is reported
+                            if ((unsigned)page >= (unsigned)pt.num_pages) atomicOr(&g_status, kStatusRange);
+                            const int prow = key & ((1 << pt.page_shift) - 1);
+                            tma_load_4d(dst + x * box_bytes, tm, full, 0, prow, u.kvh, page);
+                            tma_load_4d(dst + BOX_BYTES + x * box_bytes, tm, full, 64, prow, u.kvh, page);
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(full, TILE_BYTES);
+                        tma_load_4d(dst, tm, full, 0, krow, u.kvh, u.b);
+                        tma_load_4d(dst + BOX_BYTES, tm, full, 64, krow, u.kvh, u.b);
+                    }
                 }
             }
             // Do not leave while copies into this CTA's shared memory are in

@@ -15,6 +15,7 @@ Functions:
   sdpa_rows(q_rows, rows, k, v, ...)             -> (o, lse)   sampled rows
   row_weights(q_row, b, h, i, k, v, ...)         -> (o, lse, w) one row + softmax weights
   online(q, k, v, causal, scale, block_r, block_c) -> (o, lse) FlashAttention-2 recurrence
+  paged_to_cache(pages, block_table, seqlens)    -> cache      page-table gather (layout only)
 
 Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
 d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
@@ -203,3 +204,27 @@ def online(q, k, v, causal: bool, scale: float, block_r: int, block_c: int,
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return o, lse
+
+
+def paged_to_cache(pages, block_table, seqlens):
+    """The logical cache a page table describes ("Attention deep dive",
+    section 5: fixed-size pages addressed through a page table). pages is
+    indexed [page, token in page, kv head, dim]; block_table [B, P] int;
+    seqlens [B]. Token j of sequence b is token j % page_size of page
+    block_table[b, j // page_size]. Returns float64 [B, n_kv, P*page_size,
+    dim]: rows below the (clamped) length copied, rows at or past it zero, and
+    rows of a page id outside the pool zero (the library reads such pages as
+    zeros). No arithmetic: a gather written out row by row."""
+    pages = _f64(pages)
+    table = np.asarray(block_table.cpu().numpy() if hasattr(block_table, "cpu") else block_table, dtype=np.int64)
+    lens = np.asarray(seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int64)
+    num_pages, page_size, n_kv, dim = pages.shape
+    B, P = table.shape
+    cache = np.zeros((B, n_kv, P * page_size, dim))
+    for b in range(B):
+        n = min(max(int(lens[b]), 0), P * page_size)
+        for j in range(n):
+            pg = int(table[b, j // page_size])
+            if 0 <= pg < num_pages:
+                cache[b, :, j, :] = pages[pg, j % page_size]
+    return cache
