@@ -71,13 +71,42 @@ enum {
  *   scale: multiplies q.k before the softmax (finite, > 0; 1/sqrt(d_qk) is
  *     the usual choice).
  * Supported: d_qk == d_v in {32, 64, 128}; any B >= 0, Sq >= 0, Skv >= 1,
- * any n_kv dividing n_q with n_q / n_kv a power of two <= 128; causal needs
+ * any n_kv dividing n_q with n_q / n_kv a power of two <= 256; causal needs
  * Sq <= Skv. Output rows are bf16 rounded to nearest even.
  * Returns ATTN_OK or an error code (nothing launched on error).
  */
 int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              int B, int Sq, int Skv, int n_q, int n_kv, int d_qk, int d_v,
              int causal, float scale, attn_stream_t stream);
+
+/*
+ * attn_fwd_varlen -- attn_fwd over a packed batch of sequences of different
+ * lengths (no padding). Source: "Attention deep dive" (askaiml.pages.dev),
+ * section 5 (engines batch sequences of different lengths); each sequence is
+ * attended exactly as attn_fwd attends one batch element.
+ *
+ *   q   [total_q, n_q,  d_qk] bf16, contiguous (tokens of all sequences, packed)
+ *   k   [total_k, n_kv, d_qk] bf16, contiguous
+ *   v   [total_k, n_kv, d_v ] bf16, contiguous
+ *   o   [total_q, n_q,  d_v ] bf16 (written)
+ *   lse [n_q, total_q] fp32 (written; may be NULL)
+ *   cu_seqlens_q, cu_seqlens_k: [B + 1] int32 on the device, non-decreasing
+ *     offsets: sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *     and key rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.
+ *   max_seqlen_q: an upper bound of every sequence's query count (sizes the
+ *     grid).
+ *   causal: per sequence, query i sees key j iff j <= i + (Skv_b - Sq_b); a
+ *     row that sees no key (Sq_b > Skv_b, or Skv_b = 0) gets O = 0, LSE = -inf.
+ * A sequence whose offsets are negative, decreasing, past total_q / total_k or
+ * longer than max_seqlen_q is skipped (its outputs are left as they were) and
+ * reported as ATTN_ERR_DEVICE_RANGE by attn_device_status.
+ * Supported: d_qk == d_v in {32, 64, 128}; n_q / n_kv a power of two <= 256;
+ * B <= 65535. Returns ATTN_OK or an error code (nothing launched on error).
+ */
+int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                    int B, int max_seqlen_q, int total_q, int total_k,
+                    int n_q, int n_kv, int d_qk, int d_v, int causal, float scale, attn_stream_t stream);
 
 /*
  * attn_decode_workspace_bytes -- scratch size attn_decode needs for these

@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         L.attn_fwd.argtypes = [_vp] * 5 + [_i] * 8 + [ctypes.c_float, _vp]
         L.attn_fwd.restype = _i
+        L.attn_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 9 + [ctypes.c_float, _vp]
+        L.attn_fwd_varlen.restype = _i
         L.attn_decode_workspace_bytes.argtypes = [_i] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
         L.attn_decode_workspace_bytes.restype = _i
         L.attn_decode.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 +
@@ -109,6 +111,32 @@ def attn_fwd(q, k, v, causal: bool, scale: float, o=None, lse=None, stream=None,
     rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, n_q, n_kv, d_qk, d_v,
                         int(bool(causal)), float(scale), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool, scale: float, o=None,
+                    lse=None, stream=None, want_lse=True):
+    """Prefill over a packed batch. q [total_q,n_q,d], k/v [total_k,n_kv,d]
+    bf16 contiguous CUDA tensors; cu_seqlens_q/k int32 [B+1] on the device.
+    Returns (o [total_q,n_q,d] bf16, lse [n_q,total_q] fp32 or None)."""
+    total_q, n_q, d_qk = q.shape
+    total_k, n_kv, _ = k.shape
+    d_v = v.shape[2]
+    B = cu_seqlens_q.numel() - 1
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.numel() != B + 1:
+            raise ValueError("cu_seqlens must be contiguous int32 CUDA tensors of B + 1 offsets")
+    if o is None:
+        o = torch.empty((total_q, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((n_q, total_q), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                               _ptr(cu_seqlens_k), B, int(max_seqlen_q), total_q, total_k, n_q, n_kv, d_qk, d_v,
+                               int(bool(causal)), float(scale), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_fwd_varlen")
     return o, lse
 
 

@@ -97,12 +97,18 @@ int sm_count() {
 // ---------------------------------------------------------------------------
 // prefill
 // ---------------------------------------------------------------------------
+// Packed variable-length batch of attn_fwd_varlen (null for the dense BHSD layout).
+struct VarlenArgs {
+    const int32_t *cu_q, *cu_k;
+    int max_q, total_q, total_k;
+};
+
 template <int D>
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,
-                   int n_q, int n_kv, int causal, float scale, cudaStream_t stream) {
+                   int n_q, int n_kv, int causal, float scale, cudaStream_t stream, const VarlenArgs *vl = nullptr) {
     using C = attn::pf::Cfg<D>;
     const int G = n_q / n_kv;
-    attn::pf::Params p;
+    attn::pf::Params p{};
     p.B = B;
     p.Sq = Sq;
     p.Skv = Skv;
@@ -112,49 +118,83 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     p.causal = causal;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.lse = lse;
+    const int Sq_plan = vl ? vl->max_q : Sq;   // position blocks cover the longest sequence
     if (G >= 2) {
         p.Ht = G / 2;
         p.Pt = 256 / G;
         p.pair_by_heads = 1;
-        p.n_pb = (Sq + p.Pt - 1) / p.Pt;
+        p.n_pb = (Sq_plan + p.Pt - 1) / p.Pt;
     } else {
         p.Ht = 1;
         p.Pt = 128;
         p.pair_by_heads = 0;
-        p.n_pb = (Sq + 255) / 256;
+        p.n_pb = (Sq_plan + 255) / 256;
     }
     CUtensorMap tq, tk, tv, to;
-    {
-        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * n_q};
-        const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
-        const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)p.Pt, (uint32_t)p.Ht};
-        if (!make_map(&tq, q, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
-        if (!make_map(&to, o, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
-    }
-    {
-        const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Skv, (uint64_t)B * n_kv};
-        const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Skv * D * 2};
-        const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)attn::pf::BN, 1u};
-        if (!make_map(&tk, k, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
-        if (!make_map(&tv, v, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+    if (vl) {
+        p.cu_q = vl->cu_q;
+        p.cu_k = vl->cu_k;
+        p.total_q = vl->total_q;
+        p.total_k = vl->total_k;
+        p.o = reinterpret_cast<__nv_bfloat16 *>(o);
+        // q, o [total_q][n_q][D]: box = BOXD dims x Ht heads x Pt positions
+        const uint64_t qd[3] = {(uint64_t)D, (uint64_t)n_q, (uint64_t)vl->total_q};
+        const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)n_q * D * 2};
+        const uint32_t qb[3] = {(uint32_t)C::BOXD, (uint32_t)p.Ht, (uint32_t)p.Pt};
+        if (!make_map(&tq, q, 3, qd, qs, qb, C::ROWB)) return ATTN_ERR_CUDA;
+        if (!make_map(&to, o, 3, qd, qs, qb, C::ROWB)) return ATTN_ERR_CUDA;
+        // k, v [total_k][n_kv][D]: box = BOXD dims x 1 head x BN keys
+        const uint64_t kd[3] = {(uint64_t)D, (uint64_t)n_kv, (uint64_t)vl->total_k};
+        const uint64_t ks[2] = {(uint64_t)D * 2, (uint64_t)n_kv * D * 2};
+        const uint32_t kb[3] = {(uint32_t)C::BOXD, 1u, (uint32_t)attn::pf::BN};
+        if (!make_map(&tk, k, 3, kd, ks, kb, C::ROWB)) return ATTN_ERR_CUDA;
+        if (!make_map(&tv, v, 3, kd, ks, kb, C::ROWB)) return ATTN_ERR_CUDA;
+    } else {
+        {
+            const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * n_q};
+            const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
+            const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)p.Pt, (uint32_t)p.Ht};
+            if (!make_map(&tq, q, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+            if (!make_map(&to, o, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+        }
+        {
+            const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Skv, (uint64_t)B * n_kv};
+            const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Skv * D * 2};
+            const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)attn::pf::BN, 1u};
+            if (!make_map(&tk, k, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+            if (!make_map(&tv, v, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+        }
     }
     const size_t smem = attn::pf::smem_bytes<D>();
     static uint64_t attr_done = 0;  // per template instance, one bit per device
-    if (!ensure_smem_attr(attn::pf::prefill_kernel<D>, smem, attr_done)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, false>, smem, attr_done)) return ATTN_ERR_CUDA;
+    static uint64_t attr_done_v = 0;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, true>, smem, attr_done_v)) return ATTN_ERR_CUDA;
     // The kernel rebalances registers between warpgroups (setmaxnreg); that is
     // only safe if it was built with exactly the register count the split
     // assumes, otherwise the increase could never be granted.
     static int regs_checked = 0;
     if (regs_checked == 0) {
         cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D>) != cudaSuccess) return ATTN_ERR_CUDA;
-        regs_checked = (fa.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
+        cudaFuncAttributes fv;
+        if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D, false>) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&fv, attn::pf::prefill_kernel<D, true>) != cudaSuccess) return ATTN_ERR_CUDA;
+        regs_checked = (fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
     }
     if (regs_checked < 0) return ATTN_ERR_UNSUPPORTED;
-    const long long grid = (long long)p.n_pb * B * n_kv;
-    if (grid <= 0) return ATTN_OK;
-    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    attn::pf::prefill_kernel<D><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to, p);
+    if (vl) {
+        // x: (position block, kv head), heaviest causal blocks first; y: sequence
+        const long long gx = (long long)p.n_pb * n_kv;
+        if (gx <= 0 || B <= 0) return ATTN_OK;
+        if (gx > 0x7fffffffLL || B > 65535) return ATTN_ERR_UNSUPPORTED;
+        attn::pf::prefill_kernel<D, true><<<dim3((unsigned)gx, (unsigned)B), attn::pf::THREADS, smem, stream>>>(
+            tq, tk, tv, to, p);
+    } else {
+        const long long grid = (long long)p.n_pb * B * n_kv;
+        if (grid <= 0) return ATTN_OK;
+        if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+        attn::pf::prefill_kernel<D, false><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to, p);
+    }
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -347,6 +387,36 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
         case 32: return launch_prefill<32>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
         case 64: return launch_prefill<64>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
         default: return launch_prefill<128>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
+    }
+}
+
+int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int32_t *cu_seqlens_q,
+                    const int32_t *cu_seqlens_k, int B, int max_seqlen_q, int total_q, int total_k, int n_q,
+                    int n_kv, int d_qk, int d_v, int causal, float scale, attn_stream_t stream) {
+    if (B < 0 || max_seqlen_q < 0 || total_q < 0 || total_k < 0 || n_q < 1 || n_kv < 1 || d_qk < 1 || d_v < 1)
+        return ATTN_ERR_INVALID_ARG;
+    if (n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+    if (!q || !o || !cu_seqlens_q || !cu_seqlens_k || (total_k > 0 && (!k || !v))) return ATTN_ERR_INVALID_ARG;
+    if (d_qk != d_v || (d_qk != 32 && d_qk != 64 && d_qk != 128)) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G) || G > 256) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(o) || (total_k > 0 && (!aligned16(k) || !aligned16(v))))
+        return ATTN_ERR_MISALIGNED;
+    // With no key rows at all every query row is empty (O = 0, LSE = -inf) and
+    // no K/V tile is ever loaded; the maps are then built over q's memory
+    // only because a tensor map needs a non-empty extent.
+    VarlenArgs vl{cu_seqlens_q, cu_seqlens_k, max_seqlen_q, total_q, total_k > 0 ? total_k : 1};
+    const void *kk = total_k > 0 ? k : static_cast<const void *>(q);
+    const void *vv = total_k > 0 ? v : static_cast<const void *>(q);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (d_qk) {
+        case 32: return launch_prefill<32>(q, kk, vv, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
+        case 64: return launch_prefill<64>(q, kk, vv, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
+        default: return launch_prefill<128>(q, kk, vv, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
     }
 }
 

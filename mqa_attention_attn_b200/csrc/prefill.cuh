@@ -119,10 +119,18 @@ struct Params {
     int B, Sq, Skv, n_q, n_kv, G;
     int Ht, Pt;            // heads and positions per query tile (Ht * Pt = 128)
     int pair_by_heads;     // 1: tiles = two head halves at one position block
-    int n_pb;              // position blocks per (b, kv head)
+    int n_pb;              // position blocks per (b, kv head) (varlen: of the longest sequence)
     int causal;
     float scale_log2;      // scale * log2(e)
     float *lse;            // may be null
+    // Packed variable-length batch (the VARLEN kernel): q [total_q][n_q][D],
+    // k, v [total_k][n_kv][D], o like q, lse [n_q][total_q]; sequence b owns
+    // rows cu_q[b] .. cu_q[b+1]-1 (queries) and cu_k[b] .. cu_k[b+1]-1 (keys).
+    // A query tile's rows are then position-major (row = position * Ht +
+    // head) instead of head-major.
+    const int32_t *cu_q, *cu_k;
+    int total_q, total_k;
+    __nv_bfloat16 *o;      // varlen: rows of a tile that ends past its sequence are stored directly
 };
 
 template <bool B>
@@ -138,7 +146,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return ok;
 }
 
-template <int D>
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -150,10 +158,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t warp = warp_id(), lane = lane_id();
 
     // ---- work unit: (b, kv head, position block), heaviest causal blocks first
-    const int nbh = p.B * p.n_kv;
-    const int bh = blockIdx.x % nbh;
-    const int pb = p.n_pb - 1 - (int)(blockIdx.x / nbh);
-    const int b = bh / p.n_kv, kvh = bh % p.n_kv;
+    int b, kvh, pb;
+    int Sq = p.Sq, Skv = p.Skv, q0 = 0, k0 = 0;   // this sequence's sizes and first rows (varlen)
+    if (VARLEN) {
+        b = blockIdx.y;
+        kvh = blockIdx.x % p.n_kv;
+        pb = p.n_pb - 1 - (int)(blockIdx.x / p.n_kv);
+        q0 = p.cu_q[b];
+        k0 = p.cu_k[b];
+        Sq = p.cu_q[b + 1] - q0;
+        Skv = p.cu_k[b + 1] - k0;
+        if (q0 < 0 || k0 < 0 || Sq < 0 || Skv < 0 || q0 + Sq > p.total_q || k0 + Skv > p.total_k ||
+            Sq > p.n_pb * (p.pair_by_heads ? p.Pt : 2 * p.Pt)) {
+            if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_status, kStatusRange);
+            Sq = 0;   // malformed offsets: this sequence is skipped
+        }
+    } else {
+        const int nbh = p.B * p.n_kv;
+        const int bh = blockIdx.x % nbh;
+        pb = p.n_pb - 1 - (int)(blockIdx.x / nbh);
+        b = bh / p.n_kv;
+        kvh = bh % p.n_kv;
+    }
     int h0[2], p0[2], nt[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -164,12 +190,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             h0[t] = kvh;  // G == 1: query head == KV head
             p0[t] = pb * 2 * p.Pt + t * p.Pt;
         }
-        if (p0[t] >= p.Sq) {
+        if (p0[t] >= Sq) {
             nt[t] = 0;
         } else {
-            const int last = min(p0[t] + p.Pt, p.Sq) - 1;
-            const int keys = p.causal ? min(p.Skv, last + (p.Skv - p.Sq) + 1) : p.Skv;
-            nt[t] = (keys + BN - 1) / BN;
+            const int last = min(p0[t] + p.Pt, Sq) - 1;
+            const int keys = p.causal ? min(Skv, last + (Skv - Sq) + 1) : Skv;
+            nt[t] = keys > 0 ? (keys + BN - 1) / BN : 0;   // 0: no row of the tile sees a key
         }
     }
     const int nmax = max(nt[0], nt[1]);
@@ -222,8 +248,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int t = 0; t < 2; ++t) {
                 if (nt[t] == 0) continue;
                 for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
-                                b * p.n_q + h0[t]);
+                    if (VARLEN)
+                        tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, h0[t],
+                                    q0 + p0[t]);
+                    else
+                        tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
+                                    b * p.n_q + h0[t]);
             }
             // K tiles (V tiles are loaded by warp 2)
             int issued = 0;
@@ -238,8 +268,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const uint32_t fb = smem_u32(&sm.k_full[s]);
                 mbar_arrive_expect_tx(fb, C::KBYTES);
                 for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, j * BN,
-                                b * p.n_kv + kvh);
+                    if (VARLEN)
+                        tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, kvh, k0 + j * BN);
+                    else
+                        tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, j * BN,
+                                    b * p.n_kv + kvh);
                 ++issued;
             }
             // never leave copies in flight into this CTA's shared memory
@@ -262,8 +295,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const uint32_t fb = smem_u32(&sm.v_full[s]);
                 mbar_arrive_expect_tx(fb, C::KBYTES);
                 for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, j * BN,
-                                b * p.n_kv + kvh);
+                    if (VARLEN)
+                        tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, kvh, k0 + j * BN);
+                    else
+                        tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, j * BN,
+                                    b * p.n_kv + kvh);
                 ++issued;
             }
             for (int j = issued - 1; j >= 0 && j >= issued - VSTAGE; --j)
@@ -348,12 +384,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int t = (int)(warp - 4) / 4;
         const uint32_t quad = warp & 3u;
         const int r = (int)(quad * 32 + lane);          // row of the tile = TMEM lane
-        if (nt[t] > 0) {
-            const int hl = r / p.Pt, pl = r % p.Pt;
+        if (p0[t] < Sq) {
+            const int hl = VARLEN ? r % p.Ht : r / p.Pt;
+            const int pl = VARLEN ? r / p.Ht : r % p.Pt;
             const int pos = p0[t] + pl;
             const int head = h0[t] + hl;
-            int lim = p.causal ? pos + (p.Skv - p.Sq) : p.Skv - 1;   // last visible key
-            lim = min(lim, p.Skv - 1);
+            int lim = p.causal ? pos + (Skv - Sq) : Skv - 1;   // last visible key (< 0: none)
+            lim = min(lim, Skv - 1);
             const uint32_t trow = tmem + ((quad * 32u) << 16);
             const uint32_t colS = C::col_s(t), colO = C::col_o(t);
             const float sl = p.scale_log2;
@@ -423,7 +460,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // on B200 this is slower for head dim 128 (the softmax is bound
                 // by issue and latency, not by the special-function unit), so it
                 // is off by default.
-                const float2 nm2 = make_float2(-m_run, -m_run);
+                // a row with no visible key yet keeps m = -inf: exponentiate
+                // against 0 instead (every p is then 0)
+                const float m_use = (VARLEN && m_run == -INFINITY) ? 0.f : m_run;
+                const float2 nm2 = make_float2(-m_use, -m_use);
                 float2 rs = make_float2(0.f, 0.f);
                 // one chunk of exponentials; which pairs take the FMA-pipe
                 // polynomial is fixed at compile time (never on masked tiles)
@@ -466,17 +506,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 l_run += rs.x + rs.y;
             }
             // ---- epilogue: O / l -> bf16 -> swizzled smem -> TMA store; LSE
-            if (ok) ok = warp_wait(smem_u32(&sm.o_done[t]), 0, abort_flag, 0x33);
+            if (ok && ntt > 0) ok = warp_wait(smem_u32(&sm.o_done[t]), 0, abort_flag, 0x33);
             __syncwarp();
             tc_fence_after();
-            const float inv_l = 1.f / l_run;
+            // a row that saw no key: O = 0, LSE = -inf (the empty sum)
+            const float inv_l = (!VARLEN || l_run > 0.f) ? 1.f / l_run : 0.f;
             const uint32_t stage = smem_u32(sm.q[t]);
+            // varlen: a tile reaching past its sequence's last query is stored
+            // row by row (TMA would write into the next sequence's rows)
+            const bool direct = VARLEN && p0[t] + p.Pt > Sq;
             {
                 uint32_t o[D];
+                if (ntt > 0) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
-                    tmem_ld32(trow + colO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
-                tmem_wait_ld();
+                    for (int c = 0; c < D / 32; ++c)
+                        tmem_ld32(trow + colO + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < D; ++e) o[e] = 0u;
+                }
 #pragma unroll
                 for (int q8 = 0; q8 < D / 8; ++q8) {     // 16-byte chunks of 8 values
                     const int e0 = 8 * q8;
@@ -487,16 +536,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     w.y = f2_to_bf2(__uint_as_float(o[e0 + 2]) * inv_l, __uint_as_float(o[e0 + 3]) * inv_l);
                     w.z = f2_to_bf2(__uint_as_float(o[e0 + 4]) * inv_l, __uint_as_float(o[e0 + 5]) * inv_l);
                     w.w = f2_to_bf2(__uint_as_float(o[e0 + 6]) * inv_l, __uint_as_float(o[e0 + 7]) * inv_l);
-                    sts128(stage + bx * C::QBOX + swz<C::SWB>((uint32_t)(r * C::ROWB + ci * 16)), w);
+                    if (direct) {
+                        if (pos < Sq)
+                            *reinterpret_cast<uint4 *>(p.o + ((size_t)(q0 + pos) * p.n_q + head) * D + e0) = w;
+                    } else {
+                        sts128(stage + bx * C::QBOX + swz<C::SWB>((uint32_t)(r * C::ROWB + ci * 16)), w);
+                    }
                 }
             }
-            if (p.lse != nullptr && pos < p.Sq)
-                p.lse[((size_t)b * p.n_q + head) * p.Sq + pos] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+            if (p.lse != nullptr && pos < Sq) {
+                const float lse_v = (!VARLEN || l_run > 0.f) ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+                if (VARLEN)
+                    p.lse[(size_t)head * p.total_q + q0 + pos] = lse_v;
+                else
+                    p.lse[((size_t)b * p.n_q + head) * p.Sq + pos] = lse_v;
+            }
             fence_proxy_async_smem();
             named_bar_sync(2 + t, 128);
-            if (r == 0 && ok) {
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_store_3d(&tm_o, stage + bx * C::QBOX, bx * C::BOXD, p0[t], b * p.n_q + h0[t]);
+            if (r == 0 && ok && !direct) {
+                for (int bx = 0; bx < C::NBOX; ++bx) {
+                    if (VARLEN)
+                        tma_store_3d(&tm_o, stage + bx * C::QBOX, bx * C::BOXD, h0[t], q0 + p0[t]);
+                    else
+                        tma_store_3d(&tm_o, stage + bx * C::QBOX, bx * C::BOXD, p0[t], b * p.n_q + h0[t]);
+                }
                 tma_store_commit();
                 tma_store_wait_read0();
             }

@@ -16,6 +16,7 @@ Functions:
   row_weights(q_row, b, h, i, k, v, ...)         -> (o, lse, w) one row + softmax weights
   online(q, k, v, causal, scale, block_r, block_c) -> (o, lse) FlashAttention-2 recurrence
   paged_to_cache(pages, block_table, seqlens)    -> cache      page-table gather (layout only)
+  sdpa_varlen(q, k, v, cu_q, cu_k, causal, scale) -> (o, lse)  packed batch, one sdpa per sequence
 
 Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
 d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
@@ -228,3 +229,29 @@ def paged_to_cache(pages, block_table, seqlens):
             if 0 <= pg < num_pages:
                 cache[b, :, j, :] = pages[pg, j % page_size]
     return cache
+
+
+def sdpa_varlen(q, k, v, cu_q, cu_k, causal: bool, scale: float, nthreads=None, lib=None):
+    """The plain definition over a packed batch: q [total_q, n_q, d], k/v
+    [total_k, n_kv, d]; sequence b is rows cu_q[b]..cu_q[b+1]-1 of q and
+    cu_k[b]..cu_k[b+1]-1 of k and v, attended on its own exactly as sdpa
+    attends one batch element (causal alignment bottom-right per sequence).
+    Returns (o [total_q, n_q, d_v], lse [n_q, total_q]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = np.asarray(cu_q.cpu().numpy() if hasattr(cu_q, "cpu") else cu_q, dtype=np.int64)
+    ck = np.asarray(cu_k.cpu().numpy() if hasattr(cu_k, "cpu") else cu_k, dtype=np.int64)
+    total_q, n_q, _ = q.shape
+    d_v = v.shape[2]
+    o = np.zeros((total_q, n_q, d_v))
+    lse = np.full((n_q, total_q), -np.inf)
+    for b in range(len(cq) - 1):
+        qs, qe, ks_, ke = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if qe <= qs:
+            continue
+        qb = q[qs:qe].transpose(1, 0, 2)[None]           # [1, n_q, Sq_b, d]
+        kb = k[ks_:ke].transpose(1, 0, 2)[None]          # [1, n_kv, Skv_b, d]
+        vb = v[ks_:ke].transpose(1, 0, 2)[None]
+        ob, lb = sdpa(qb, kb, vb, causal, scale, nthreads=nthreads, lib=lib)
+        o[qs:qe] = ob[0].transpose(1, 0, 2)
+        lse[:, qs:qe] = lb[0]
+    return o, lse

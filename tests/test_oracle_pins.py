@@ -38,3 +38,32 @@ def test_paged_to_cache_round_trip():
     assert np.array_equal(got[0, :, :6], cache[0, :, :6]) and not got[0, :, 6:].any()
     assert not got[1, :, :ps].any() and np.array_equal(got[1, :, ps:], cache[1, :, ps:])
     assert not got[2].any()
+
+
+def test_sdpa_varlen_equals_batched_sdpa_on_equal_lengths():
+    """A packed batch of equal-length sequences is the BHSD batch reshaped;
+    a packed batch of one sequence is that sequence; with lengths 0 and
+    Sq > Skv (causal) the empty rows give O = 0 and LSE = -inf."""
+    rng = np.random.default_rng(8)
+    B, S, n_q, n_kv, d = 3, 7, 4, 2, 5
+    q = rng.standard_normal((B, n_q, S, d))
+    k = rng.standard_normal((B, n_kv, S, d))
+    v = rng.standard_normal((B, n_kv, S, d))
+    o_ref, l_ref = oracle.sdpa(q, k, v, True, 0.4)
+    pack = lambda x: x.transpose(0, 2, 1, 3).reshape(B * S, x.shape[1], d)
+    cu = np.arange(B + 1) * S
+    o, l = oracle.sdpa_varlen(pack(q), pack(k), pack(v), cu, cu, True, 0.4)
+    assert np.array_equal(o, pack(o_ref))
+    assert np.array_equal(l, l_ref.transpose(1, 0, 2).reshape(n_q, B * S))
+    # lengths (2, 0, 3) queries against (1, 2, 3) keys, causal
+    cq, ck = np.array([0, 2, 2, 5]), np.array([0, 1, 3, 6])
+    qv, kv_, vv = rng.standard_normal((5, n_q, d)), rng.standard_normal((6, n_kv, d)), rng.standard_normal((6, n_kv, d))
+    o, l = oracle.sdpa_varlen(qv, kv_, vv, cq, ck, True, 0.5)
+    # sequence 0: Sq 2 > Skv 1 -> query 0 sees no key, query 1 sees key 0
+    assert not o[0].any() and np.all(np.isneginf(l[:, 0]))
+    G = n_q // n_kv
+    for h in range(n_q):
+        assert np.allclose(o[1, h], vv[0, h // G])
+    ob, lb = oracle.sdpa(qv[2:5].transpose(1, 0, 2)[None], kv_[3:6].transpose(1, 0, 2)[None],
+                         vv[3:6].transpose(1, 0, 2)[None], True, 0.5)
+    assert np.array_equal(o[2:5], ob[0].transpose(1, 0, 2)) and np.array_equal(l[:, 2:5], lb[0])
