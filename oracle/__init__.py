@@ -17,6 +17,7 @@ Functions:
   online(q, k, v, causal, scale, block_r, block_c) -> (o, lse) FlashAttention-2 recurrence
   paged_to_cache(pages, block_table, seqlens)    -> cache      page-table gather (layout only)
   sdpa_varlen(q, k, v, cu_q, cu_k, causal, scale) -> (o, lse)  packed batch, one sdpa per sequence
+  sdpa_window(q, k, v, causal, window, n_sink, scale, seqlens=None) -> (o, lse) sliding window + sinks
 
 Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
 d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
@@ -64,6 +65,9 @@ def _declare(lib):
     lib.oracle_row_weights_fp64.restype = _i64
     lib.oracle_online_fp64.argtypes = [_f64p] * 5 + common + [_int, _int, _int]
     lib.oracle_online_fp64.restype = _int
+    lib.oracle_sdpa_window_fp64.argtypes = ([_f64p] * 5 + [_int] * 7 + [_i64] * 6 +
+                                            [_i32p, _int, _int, _int, ctypes.c_double, _int])
+    lib.oracle_sdpa_window_fp64.restype = _int
     return lib
 
 
@@ -254,4 +258,27 @@ def sdpa_varlen(q, k, v, cu_q, cu_k, causal: bool, scale: float, nthreads=None, 
         ob, lb = sdpa(qb, kb, vb, causal, scale, nthreads=nthreads, lib=lib)
         o[qs:qe] = ob[0].transpose(1, 0, 2)
         lse[:, qs:qe] = lb[0]
+    return o, lse
+
+
+def sdpa_window(q, k, v, causal: bool, window: int, n_sink: int, scale: float, seqlens=None, d_v=None,
+                nthreads=None, lib=None):
+    """Plain definition with a sliding window: of the visible keys of sdpa,
+    key j stays only if p - j < window (p = the query's own position, the
+    last visible key) or j < n_sink. Same layouts as sdpa."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, n_q, Sq, d_qk = q.shape
+    _, n_kv, Skv, _ = k.shape
+    d_v = d_v or v.shape[3]
+    o = np.zeros((B, n_q, Sq, d_v))
+    lse = np.zeros((B, n_q, Sq))
+    s_arr, s_ptr = _seq(seqlens)
+    rc = lib.oracle_sdpa_window_fp64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                     B, n_q, n_kv, Sq, Skv, d_qk, d_v,
+                                     *_kv_strides(k), *_kv_strides(v), s_ptr,
+                                     int(bool(causal)), int(window), int(n_sink), float(scale),
+                                     _nthreads(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
     return o, lse

@@ -44,6 +44,13 @@
  *     which calls SDPA with is_causal=False for the lone query).
  *   - an empty visible set gives o = 0 and lse = -inf (the pages are
  *     silent; this is the limit of an empty sum).
+ *   - sliding window (window W > 0): of the keys above, only those with
+ *     p - j < W stay, p being the query's own position (the last visible
+ *     key: i + Skv - Sq in causal prefill, seqlens[b] - 1 in decode),
+ *     "Attention deep dive" (askaiml.pages.dev) section 6, mask (j <= i)
+ *     AND (i - j < W); plus the first n_sink keys, which stay visible to
+ *     every query ("Attention Engineering" section 5, failure mode 2: keep
+ *     the initial sink tokens in a rolling window). W = 0: no window.
  *
  * The online mode follows the FlashAttention-2 exact tiled rescaling
  * recurrence of "Attention Engineering" section 4 (running m, l, O~ per row,
@@ -77,6 +84,7 @@ typedef struct {
     const int32_t *seqlens;
     int causal;
     double scale;
+    int64_t window, n_sink;   /* window 0: every key up to the end is visible */
 } problem_t;
 
 static int check_problem(const problem_t *p, int B)
@@ -85,6 +93,7 @@ static int check_problem(const problem_t *p, int B)
     if (p->d_qk <= 0 || p->d_v <= 0) return -1;
     if (p->n_q % p->n_kv != 0) return -1;
     if (p->causal != 0 && p->causal != 1) return -1;
+    if (p->window < 0 || p->n_sink < 0) return -1;
     return 0;
 }
 
@@ -106,10 +115,17 @@ static int64_t visible_end(const problem_t *p, int b, int64_t i)
     return p->Skv;
 }
 
+/* Is key j (< end) visible? Only the window and the sinks remove keys. */
+static int visible(const problem_t *p, int64_t end, int64_t j)
+{
+    if (p->window == 0) return 1;
+    return (end - 1 - j < p->window) || (j < p->n_sink);
+}
+
 /*
  * One query row, the plain definition: score, scale, mask, two-pass softmax,
  * mix. `s` is scratch of at least Skv doubles. `weights` (optional) receives
- * the softmax weights of the visible keys.
+ * the softmax weights of the visible keys (0 for the others).
  */
 static void attend_row(const problem_t *p, int b, int h, int64_t i,
                        const double *q_row, double *o_row, double *lse_out,
@@ -125,21 +141,23 @@ static void attend_row(const problem_t *p, int b, int h, int64_t i,
         *lse_out = -INFINITY;
         return;
     }
-    /* score and scale */
+    /* score and scale (a window keeps the last key, so some key is visible) */
     for (int64_t j = 0; j < end; ++j) {
+        if (!visible(p, end, j)) continue;
         const double *kj = kb + j * p->k_ss;
         double acc = 0.0;
         for (int c = 0; c < p->d_qk; ++c) acc += q_row[c] * kj[c];
         s[j] = p->scale * acc;
     }
     /* softmax, pass 1: the row maximum */
-    double m = s[0];
-    for (int64_t j = 1; j < end; ++j)
-        if (s[j] > m) m = s[j];
+    double m = -INFINITY;
+    for (int64_t j = 0; j < end; ++j)
+        if (visible(p, end, j) && s[j] > m) m = s[j];
     /* softmax, pass 2: exponentials relative to the maximum, their sum, and
        the weighted sum of value rows */
     double l = 0.0;
     for (int64_t j = 0; j < end; ++j) {
+        if (!visible(p, end, j)) continue;
         const double e = exp(s[j] - m);
         const double *vj = vb + j * p->v_ss;
         l += e;
@@ -148,7 +166,7 @@ static void attend_row(const problem_t *p, int b, int h, int64_t i,
     for (int c = 0; c < p->d_v; ++c) o_row[c] /= l;
     *lse_out = m + log(l);
     if (weights) {
-        for (int64_t j = 0; j < end; ++j) weights[j] = exp(s[j] - m) / l;
+        for (int64_t j = 0; j < end; ++j) weights[j] = visible(p, end, j) ? exp(s[j] - m) / l : 0.0;
     }
 }
 
@@ -172,8 +190,44 @@ int oracle_sdpa_fp64(const double *q, const double *k, const double *v,
                      const int32_t *seqlens, int causal, double scale, int nthreads)
 {
     problem_t p = {k, v, k_sb, k_sh, k_ss, v_sb, v_sh, v_ss,
-                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale};
+                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale, 0, 0};
     if (check_problem(&p, B)) return -1;
+    const int64_t rows = (int64_t)B * n_q * Sq;
+    int nt = set_threads(nthreads);
+    int err = 0;
+#pragma omp parallel num_threads(nt)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t r = 0; r < rows; ++r) {
+                const int64_t i = r % Sq;
+                const int h = (int)((r / Sq) % n_q);
+                const int b = (int)(r / ((int64_t)Sq * n_q));
+                attend_row(&p, b, h, i, q + r * d_qk, o + r * d_v, lse + r, s, NULL);
+            }
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* Full forward with a sliding window of `window` keys (> 0) and `n_sink`
+ * always-visible initial keys (see the visible set above). */
+int oracle_sdpa_window_fp64(const double *q, const double *k, const double *v,
+                            double *o, double *lse,
+                            int B, int n_q, int n_kv, int Sq, int Skv, int d_qk, int d_v,
+                            int64_t k_sb, int64_t k_sh, int64_t k_ss,
+                            int64_t v_sb, int64_t v_sh, int64_t v_ss,
+                            const int32_t *seqlens, int causal, int window, int n_sink,
+                            double scale, int nthreads)
+{
+    problem_t p = {k, v, k_sb, k_sh, k_ss, v_sb, v_sh, v_ss,
+                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale, window, n_sink};
+    if (check_problem(&p, B) || window <= 0) return -1;
     const int64_t rows = (int64_t)B * n_q * Sq;
     int nt = set_threads(nthreads);
     int err = 0;
@@ -212,7 +266,7 @@ int oracle_sdpa_rows_fp64(const double *q_rows, const double *k, const double *v
                           const int32_t *seqlens, int causal, double scale, int nthreads)
 {
     problem_t p = {k, v, k_sb, k_sh, k_ss, v_sb, v_sh, v_ss,
-                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale};
+                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale, 0, 0};
     if (check_problem(&p, B) || n_rows < 0) return -1;
     for (int r = 0; r < n_rows; ++r) {
         if (row_b[r] < 0 || row_b[r] >= B || row_h[r] < 0 || row_h[r] >= n_q ||
@@ -251,7 +305,7 @@ int64_t oracle_row_weights_fp64(const double *q_row, const double *k, const doub
                                 const int32_t *seqlens, int causal, double scale)
 {
     problem_t p = {k, v, k_sb, k_sh, k_ss, v_sb, v_sh, v_ss,
-                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale};
+                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale, 0, 0};
     if (check_problem(&p, B) || b < 0 || b >= B || h < 0 || h >= n_q || i < 0 || i >= Sq)
         return -1;
     double *s = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
@@ -285,7 +339,7 @@ int oracle_online_fp64(const double *q, const double *k, const double *v,
                        int block_r, int block_c, int nthreads)
 {
     problem_t p = {k, v, k_sb, k_sh, k_ss, v_sb, v_sh, v_ss,
-                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale};
+                   n_q, n_kv, Sq, Skv, d_qk, d_v, seqlens, causal, scale, 0, 0};
     if (check_problem(&p, B) || block_r <= 0 || block_c <= 0) return -1;
     const int G = n_q / n_kv;
     const int64_t n_blocks = ((int64_t)Sq + block_r - 1) / block_r;

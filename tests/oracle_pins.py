@@ -336,6 +336,29 @@ def check_rows_mode(lib):
         assert np.array_equal(orr[r], o[b, h, i]) and lr[r] == lse[b, h, i]
 
 
+def check_sliding_window(lib):
+    """Sliding window and sinks against torch SDPA with the explicit boolean
+    mask of "Attention deep dive" section 6, (j <= p) and (p - j < W), widened
+    by the first n_sink keys; bottom-right alignment (Sq < Skv) and the
+    decode form (window ending at seqlens[b] - 1) included."""
+    B, n_q, n_kv, Sq, Skv, d = 2, 4, 2, 13, 29, 8
+    q, k, v = _rand((B, n_q, Sq, d), 60), _rand((B, n_kv, Skv, d), 61), _rand((B, n_kv, Skv, d), 62)
+    pos = torch.arange(Sq)[:, None] + (Skv - Sq)
+    j = torch.arange(Skv)[None, :]
+    for W, ns in [(1, 0), (4, 0), (4, 2), (9, 5), (40, 0)]:
+        mask = (j <= pos) & ((pos - j < W) | (j < ns))
+        ref = F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=0.3, enable_gqa=True)
+        o, _ = oracle.sdpa_window(q, k, v, True, W, ns, 0.3, lib=lib)
+        assert np.max(np.abs(o - ref.numpy())) <= 1e-10, (W, ns)
+    seqlens = np.array([29, 6], dtype=np.int32)
+    o, _ = oracle.sdpa_window(q[:, :, :1], k, v, False, 3, 2, 0.3, seqlens=seqlens, lib=lib)
+    for b, L in enumerate(seqlens):
+        keep = sorted(set(range(min(2, L))) | set(range(max(0, L - 3), L)))
+        ref = F.scaled_dot_product_attention(q[b:b + 1, :, :1], k[b:b + 1, :, keep], v[b:b + 1, :, keep],
+                                             scale=0.3, enable_gqa=True)
+        assert np.max(np.abs(o[b:b + 1] - ref.numpy())) <= 1e-10
+
+
 ALL_CHECKS = [
     check_worked_example, check_worked_example_first_tile, check_worked_example_online,
     check_first_causal_row, check_rows_sum_to_one, check_value_shift, check_key_shift,
@@ -343,4 +366,5 @@ ALL_CHECKS = [
     check_mha_independent_heads, check_permutations, check_torch_sdpa_fp64,
     check_bottom_right_causal, check_decode, check_empty_visible_set, check_mla_alias,
     check_online_equals_two_pass, check_rows_mode,
+    check_sliding_window,
 ]

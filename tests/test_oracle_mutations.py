@@ -31,6 +31,12 @@ MUTATIONS = [
     ("online_rescale_sign", "const double alpha = exp(m[r] - m_new);",
      "const double alpha = exp(m_new - m[r]);"),
     ("online_lse_stale", "lse[row] = m[r] + log(l[r]);", "lse[row] = log(l[r]);"),
+    ("window_off_by_one", "return (end - 1 - j < p->window) || (j < p->n_sink);",
+     "return (end - 1 - j <= p->window) || (j < p->n_sink);"),
+    ("window_sinks_ignored", "return (end - 1 - j < p->window) || (j < p->n_sink);",
+     "return (end - 1 - j < p->window);"),
+    ("window_anchored_at_row_not_position", "return (end - 1 - j < p->window) || (j < p->n_sink);",
+     "return (end - 1 - j - (p->Skv - p->Sq) < p->window) || (j < p->n_sink);"),
 ]
 
 

@@ -67,3 +67,40 @@ def test_sdpa_varlen_equals_batched_sdpa_on_equal_lengths():
     ob, lb = oracle.sdpa(qv[2:5].transpose(1, 0, 2)[None], kv_[3:6].transpose(1, 0, 2)[None],
                          vv[3:6].transpose(1, 0, 2)[None], True, 0.5)
     assert np.array_equal(o[2:5], ob[0].transpose(1, 0, 2)) and np.array_equal(l[:, 2:5], lb[0])
+
+
+def test_sdpa_window_pins():
+    """Sliding window + sinks against what fixes it: a window covering every
+    key is the causal forward; a window of 1 without sinks returns each
+    row's own value row (LSE = scale q.k of that key); and an independent
+    library (torch SDPA in fp64 with the explicit boolean mask of "Attention
+    deep dive" section 6, (j <= i) and (i - j < W), or j < n_sink)."""
+    import torch
+    rng = np.random.default_rng(21)
+    B, n_q, n_kv, S, d = 2, 4, 2, 37, 8
+    q = rng.standard_normal((B, n_q, S, d))
+    k = rng.standard_normal((B, n_kv, S, d))
+    v = rng.standard_normal((B, n_kv, S, d))
+    o_c, l_c = oracle.sdpa(q, k, v, True, 0.3)
+    o_w, l_w = oracle.sdpa_window(q, k, v, True, S, 0, 0.3)
+    assert np.array_equal(o_w, o_c) and np.array_equal(l_w, l_c)
+    o1, l1 = oracle.sdpa_window(q, k, v, True, 1, 0, 0.3)
+    G = n_q // n_kv
+    for h in range(n_q):
+        assert np.array_equal(o1[:, h], v[:, h // G])
+        assert np.allclose(l1[:, h], 0.3 * (q[:, h] * k[:, h // G]).sum(-1), atol=1e-12)
+    for W, ns in [(5, 0), (5, 3), (11, 4), (1, 2)]:
+        o_w, l_w = oracle.sdpa_window(q, k, v, True, W, ns, 0.3)
+        i = np.arange(S)[:, None]
+        j = np.arange(S)[None, :]
+        mask = (j <= i) & ((i - j < W) | (j < ns))
+        kr = torch.tensor(k).repeat_interleave(G, dim=1)
+        vr = torch.tensor(v).repeat_interleave(G, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q), kr, vr, attn_mask=torch.tensor(mask), scale=0.3).numpy()
+        assert np.allclose(o_w, ref, atol=1e-12, rtol=0), (W, ns)
+    # decode form: the window ends at the last visible key seqlens[b] - 1
+    o_d, l_d = oracle.sdpa_window(q[:, :, :1], k, v, False, 4, 1, 0.3, seqlens=[20, 2])
+    keep = [0, 16, 17, 18, 19]
+    o_r, l_r = oracle.sdpa(q[:1, :, :1], k[:1, :, keep], v[:1, :, keep], False, 0.3)
+    assert np.allclose(o_d[:1], o_r, atol=1e-12) and np.allclose(l_d[:1], l_r, atol=1e-12)
