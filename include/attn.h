@@ -80,6 +80,24 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              int causal, float scale, attn_stream_t stream);
 
 /*
+ * attn_fwd_window -- causal attn_fwd with a sliding window and sink keys.
+ * Source: "Attention deep dive" (askaiml.pages.dev), section 6 (sliding-window
+ * attention: token i attends to the last W tokens, mask (j <= i) AND
+ * (i - j < W)); "Attention Engineering: From MHA to GQA, MLA &
+ * FlashAttention", section 5, failure mode 2 (keep the first tokens as
+ * permanent attention sinks in a rolling window).
+ * Layouts, outputs and errors as attn_fwd, with causal fixed: a query at
+ * position p = i + (Skv - Sq) sees key j iff j <= p and (p - j < window or
+ * j < n_sink). Key tiles that hold neither window nor sink keys of a query
+ * tile are never loaded.
+ * Supported: as attn_fwd with causal = 1 (Sq <= Skv); window >= 1,
+ * n_sink >= 0 (0: no sinks).
+ */
+int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse,
+                    int B, int Sq, int Skv, int n_q, int n_kv, int d_qk, int d_v,
+                    int window, int n_sink, float scale, attn_stream_t stream);
+
+/*
  * attn_fwd_varlen -- attn_fwd over a packed batch of sequences of different
  * lengths (no padding). Source: "Attention deep dive" (askaiml.pages.dev),
  * section 5 (engines batch sequences of different lengths); each sequence is
@@ -149,6 +167,24 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
                 int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
                 int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
                 float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_decode_window -- attn_decode with a sliding window and sink keys.
+ * Source: "Attention deep dive" (askaiml.pages.dev), section 6 (each token
+ * attends only to the last W tokens); "Attention Engineering" section 5,
+ * failure mode 2 (the first tokens stay as attention sinks). For a sequence
+ * of length L the visible keys are L-window .. L-1 and 0 .. n_sink-1; key
+ * chunks holding neither are not read. Arguments, layouts, workspace and
+ * errors as attn_decode; window >= 1, n_sink >= 0. Supported: (d_qk, d_v) =
+ * (128, 128).
+ */
+int attn_decode_window(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                       void *o, float *lse,
+                       int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
+                       int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                       int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
+                       int window, int n_sink, float scale,
+                       void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * attn_decode_paged -- attn_decode against a paged KV cache.

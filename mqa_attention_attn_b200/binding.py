@@ -53,12 +53,17 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd.argtypes = [_vp] * 5 + [_i] * 8 + [ctypes.c_float, _vp]
         L.attn_fwd.restype = _i
         L.attn_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 9 + [ctypes.c_float, _vp]
+        L.attn_fwd_window.argtypes = [_vp] * 5 + [_i] * 9 + [ctypes.c_float, _vp]
+        L.attn_fwd_window.restype = _i
         L.attn_fwd_varlen.restype = _i
         L.attn_decode_workspace_bytes.argtypes = [_i] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
         L.attn_decode_workspace_bytes.restype = _i
         L.attn_decode.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 +
                                   [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode.restype = _i
+        L.attn_decode_window.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 + [_i, _i] +
+                                         [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_decode_window.restype = _i
         L.attn_decode_paged.argtypes = ([_vp] * 7 + [_i] * 8 + [_i64] * 6 +
                                         [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode_paged.restype = _i
@@ -111,6 +116,25 @@ def attn_fwd(q, k, v, causal: bool, scale: float, o=None, lse=None, stream=None,
     rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, n_q, n_kv, d_qk, d_v,
                         int(bool(causal)), float(scale), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_window(q, k, v, window: int, n_sink: int, scale: float, o=None, lse=None, stream=None, want_lse=True):
+    """Causal prefill with a sliding window of `window` keys and `n_sink`
+    always-visible initial keys. Layouts as attn_fwd."""
+    B, n_q, Sq, d_qk = q.shape
+    _, n_kv, Skv, _ = k.shape
+    d_v = v.shape[3]
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if o is None:
+        o = torch.empty((B, n_q, Sq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Sq), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, n_q, n_kv, d_qk, d_v,
+                               int(window), int(n_sink), float(scale), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_fwd_window")
     return o, lse
 
 
@@ -179,6 +203,32 @@ def attn_decode(q, kcache, vcache, seqlens, scale: float, d_v=None, o=None, lse=
                            B, n_q, n_kv, d_qk, d_v, S_max, *ks, *vs, float(scale),
                            _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_decode")
+    return o, lse
+
+
+def attn_decode_window(q, kcache, vcache, seqlens, window: int, n_sink: int, scale: float, o=None, lse=None,
+                       workspace=None, stream=None, want_lse=True):
+    """attn_decode keeping only the last `window` keys of each sequence and
+    its first `n_sink` keys. Arguments as attn_decode (head dim 128)."""
+    B, n_q, d_qk = q.shape
+    _, n_kv, S_max, _ = kcache.shape
+    d_v = vcache.shape[3]
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    if seqlens.dtype != torch.int32 or not seqlens.is_cuda:
+        raise ValueError("seqlens must be an int32 CUDA tensor")
+    ks, vs = _elem_strides(kcache), _elem_strides(vcache)
+    if o is None:
+        o = torch.empty((B, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, n_q, n_kv, d_qk, d_v, S_max)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().attn_decode_window(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse),
+                                  B, n_q, n_kv, d_qk, d_v, S_max, *ks, *vs, int(window), int(n_sink), float(scale),
+                                  _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_decode_window")
     return o, lse
 
 

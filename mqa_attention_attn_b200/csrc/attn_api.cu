@@ -105,7 +105,11 @@ struct VarlenArgs {
 
 template <int D>
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,
-                   int n_q, int n_kv, int causal, float scale, cudaStream_t stream, const VarlenArgs *vl = nullptr) {
+                   int n_q, int n_kv, int causal, float scale, cudaStream_t stream, const VarlenArgs *vl = nullptr,
+                   int window = 0, int n_sink = 0) {
+    using attn::pf::kDense;
+    using attn::pf::kVarlen;
+    using attn::pf::kWindow;
     using C = attn::pf::Cfg<D>;
     const int G = n_q / n_kv;
     attn::pf::Params p{};
@@ -118,6 +122,8 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     p.causal = causal;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.lse = lse;
+    p.window = window;
+    p.n_sink = n_sink;
     const int Sq_plan = vl ? vl->max_q : Sq;   // position blocks cover the longest sequence
     if (G >= 2) {
         p.Ht = G / 2;
@@ -167,19 +173,22 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     }
     const size_t smem = attn::pf::smem_bytes<D>();
     static uint64_t attr_done = 0;  // per template instance, one bit per device
-    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, false>, smem, attr_done)) return ATTN_ERR_CUDA;
-    static uint64_t attr_done_v = 0;
-    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, true>, smem, attr_done_v)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kDense>, smem, attr_done)) return ATTN_ERR_CUDA;
+    static uint64_t attr_done_v = 0, attr_done_w = 0;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kVarlen>, smem, attr_done_v)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kWindow>, smem, attr_done_w)) return ATTN_ERR_CUDA;
     // The kernel rebalances registers between warpgroups (setmaxnreg); that is
     // only safe if it was built with exactly the register count the split
     // assumes, otherwise the increase could never be granted.
     static int regs_checked = 0;
     if (regs_checked == 0) {
         cudaFuncAttributes fa;
-        cudaFuncAttributes fv;
-        if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D, false>) != cudaSuccess) return ATTN_ERR_CUDA;
-        if (cudaFuncGetAttributes(&fv, attn::pf::prefill_kernel<D, true>) != cudaSuccess) return ATTN_ERR_CUDA;
-        regs_checked = (fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
+        cudaFuncAttributes fv, fw;
+        if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D, kDense>) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&fv, attn::pf::prefill_kernel<D, kVarlen>) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&fw, attn::pf::prefill_kernel<D, kWindow>) != cudaSuccess) return ATTN_ERR_CUDA;
+        regs_checked = (fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs &&
+                        fw.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
     }
     if (regs_checked < 0) return ATTN_ERR_UNSUPPORTED;
     if (vl) {
@@ -187,13 +196,18 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         const long long gx = (long long)p.n_pb * n_kv;
         if (gx <= 0 || B <= 0) return ATTN_OK;
         if (gx > 0x7fffffffLL || B > 65535) return ATTN_ERR_UNSUPPORTED;
-        attn::pf::prefill_kernel<D, true><<<dim3((unsigned)gx, (unsigned)B), attn::pf::THREADS, smem, stream>>>(
+        attn::pf::prefill_kernel<D, kVarlen><<<dim3((unsigned)gx, (unsigned)B), attn::pf::THREADS, smem, stream>>>(
             tq, tk, tv, to, p);
     } else {
         const long long grid = (long long)p.n_pb * B * n_kv;
         if (grid <= 0) return ATTN_OK;
         if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-        attn::pf::prefill_kernel<D, false><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to, p);
+        if (window > 0)
+            attn::pf::prefill_kernel<D, kWindow><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
+                                                                                                       p);
+        else
+            attn::pf::prefill_kernel<D, kDense><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
+                                                                                                      p);
     }
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -224,6 +238,7 @@ struct CacheView {
     int64_t ks[3], vs[3];              // element strides, outermost first
     attn::dec::PageTable pt;           // pt.table == nullptr: contiguous
     int page_size;
+    attn::dec::Window win;             // sliding window (window 0: none)
 };
 
 template <int GT, bool PAGED>
@@ -273,10 +288,11 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
     const long long max_units = (long long)B * n_kv * n_hb * n_splits;
     const int grid = (int)(max_units < 2LL * n_sm ? max_units : 2LL * n_sm);
     decode_split_kernel<GT, PAGED><<<grid, THREADS, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q, n_kv,
-                                                                    G, n_hb, S_max, n_splits, scale_log2, cv.pt);
+                                                                    G, n_hb, S_max, n_splits, scale_log2, cv.pt,
+                                                                    cv.win);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
-        ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH);
+        ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH, cv.win);
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -390,6 +406,27 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
     }
 }
 
+int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,
+                    int n_q, int n_kv, int d_qk, int d_v, int window, int n_sink, float scale, attn_stream_t stream) {
+    if (B < 0 || Sq < 0 || Skv < 1 || n_q < 1 || n_kv < 1 || d_qk < 1 || d_v < 1) return ATTN_ERR_INVALID_ARG;
+    if (n_q % n_kv != 0 || window < 1 || n_sink < 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || Sq == 0) return ATTN_OK;
+    if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+    if (d_qk != d_v || (d_qk != 32 && d_qk != 64 && d_qk != 128)) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G) || G > 256) return ATTN_ERR_UNSUPPORTED;
+    if (Sq > Skv) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)B * n_q > 0x7fffffffLL || (long long)B * n_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (d_qk) {
+        case 32: return launch_prefill<32>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, 1, scale, s, nullptr, window, n_sink);
+        case 64: return launch_prefill<64>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, 1, scale, s, nullptr, window, n_sink);
+        default: return launch_prefill<128>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, 1, scale, s, nullptr, window, n_sink);
+    }
+}
+
 int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int32_t *cu_seqlens_q,
                     const int32_t *cu_seqlens_k, int B, int max_seqlen_q, int total_q, int total_k, int n_q,
                     int n_kv, int d_qk, int d_v, int causal, float scale, attn_stream_t stream) {
@@ -431,10 +468,13 @@ int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int
     return ATTN_OK;
 }
 
-int attn_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o, float *lse,
-                int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b, int64_t k_stride_h,
-                int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale,
-                void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+int decode_entry(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o, float *lse,
+                 int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b, int64_t k_stride_h,
+                 int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale,
+                 void *workspace, size_t workspace_bytes, attn_stream_t stream, attn::dec::Window win) {
     if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
     if (B == 0) return ATTN_OK;
@@ -458,8 +498,10 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         cv.v = vcache;
         cv.ks[0] = k_stride_b, cv.ks[1] = k_stride_h, cv.ks[2] = k_stride_s;
         cv.vs[0] = v_stride_b, cv.vs[1] = v_stride_h, cv.vs[2] = v_stride_s;
+        cv.win = win;
         return dispatch_decode_gqa<false>(G, q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, workspace, s);
     }
+    if (win.window > 0) return ATTN_ERR_UNSUPPORTED;   // the MLA kernel has no window
     if (d_qk == 576 && d_v == 512 && n_kv == 1) {
         // the value rows must be the first 512 columns of the key rows
         if (vcache != kcache || v_stride_b != k_stride_b || v_stride_s != k_stride_s) return ATTN_ERR_UNSUPPORTED;
@@ -471,6 +513,30 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
         return launch_decode_mla(q, kcache, seqlens, o, lse, B, n_q, S_max, k_stride_b, k_stride_s, scale, s);
     }
     return ATTN_ERR_UNSUPPORTED;
+}
+}  // namespace
+
+extern "C" {
+
+int attn_decode(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o, float *lse,
+                int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b, int64_t k_stride_h,
+                int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale,
+                void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+    return decode_entry(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, d_qk, d_v, S_max, k_stride_b, k_stride_h,
+                        k_stride_s, v_stride_b, v_stride_h, v_stride_s, scale, workspace, workspace_bytes, stream,
+                        attn::dec::Window{0, 0});
+}
+
+int attn_decode_window(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o,
+                       float *lse, int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b,
+                       int64_t k_stride_h, int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h,
+                       int64_t v_stride_s, int window, int n_sink, float scale, void *workspace,
+                       size_t workspace_bytes, attn_stream_t stream) {
+    if (window < 1 || n_sink < 0) return ATTN_ERR_INVALID_ARG;
+    if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
+    return decode_entry(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, d_qk, d_v, S_max, k_stride_b, k_stride_h,
+                        k_stride_s, v_stride_b, v_stride_h, v_stride_s, scale, workspace, workspace_bytes, stream,
+                        attn::dec::Window{window, n_sink});
 }
 
 int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,

@@ -82,6 +82,32 @@ constexpr size_t smem_bytes() {
     return sizeof(Smem<GT>) + 1024;  // + alignment slack
 }
 
+// Sliding window over the cache (window 0: none): of keys 0 .. L-1 a
+// sequence of length L keeps the last `window` and the first `n_sink`.
+struct Window {
+    int window, n_sink;
+};
+
+// The chunks of a sequence of length L that hold a visible key, in order:
+// sink chunks 0 .. n_sc-1, then window chunks wc0 .. ceil(L / CH) - 1.
+struct ChunkPlan {
+    int n, n_sc, wc0;
+    __device__ __forceinline__ int split(int c) const { return c < n_sc ? c : wc0 + (c - n_sc); }
+};
+
+__device__ __forceinline__ ChunkPlan chunk_plan(int L, int CH, Window w) {
+    const int all = (L + CH - 1) / CH;
+    if (w.window <= 0) return ChunkPlan{all, all, all};
+    const int n_sc = (min(w.n_sink, L) + CH - 1) / CH;
+    const int wc0 = max(max(L - w.window, 0) / CH, n_sc);
+    return ChunkPlan{n_sc + max(all - wc0, 0), n_sc, wc0};
+}
+
+// Is key `key` of a sequence of length L visible under the window?
+__device__ __forceinline__ bool window_keeps(int key, int L, Window w) {
+    return w.window <= 0 || key >= L - w.window || key < w.n_sink;
+}
+
 // Work units are the non-empty (b, kv head, head block, chunk) slots, in order
 // b-major, then kv head and head block, then chunk; sequence b contributes
 // n_kv * n_hb * ceil(seqlen_b / CH) units (CH = keys per unit). The CTA walks units c, c + G, ...
@@ -89,13 +115,15 @@ constexpr size_t smem_bytes() {
 struct UnitCursor {
     int b = 0;          // sequence of the current range
     long long base = 0; // first unit index of sequence b
-    int ns = 0;         // chunks of sequence b
+    int ns = 0;         // chunks of sequence b that hold a visible key
     int seqlen = 0;
+    ChunkPlan plan{0, 0, 0};
 };
 
 struct Unit {
-    int b, kvh, hb, split, key0, nkeys, ntiles;
+    int b, kvh, hb, split, key0, nkeys, ntiles, seqlen;
 };
+
 
 // Paged cache: logical key t of sequence b sits in row t % page_size of page
 // table[b * pages_per_seq + t / page_size] of a page pool; the K and V tensor
@@ -117,28 +145,33 @@ __device__ __forceinline__ int clamp_seqlen(const int32_t *seqlens, int b, int S
 // Advance the cursor to the sequence holding unit i (i never decreases) and
 // decode the unit. Returns false when i is past the last unit.
 template <int CH>
+__device__ __forceinline__ void start_sequence(UnitCursor &cur, const int32_t *seqlens, int S_max, Window w) {
+    cur.seqlen = clamp_seqlen(seqlens, cur.b, S_max);
+    cur.plan = chunk_plan(cur.seqlen, CH, w);
+    cur.ns = cur.plan.n;
+}
+
+template <int CH>
 __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const int32_t *seqlens, int B, int S_max,
-                                          int n_hb, int units_per_chunk, Unit &u) {
+                                          int n_hb, int units_per_chunk, Window w, Unit &u) {
     while (cur.b < B) {
         const long long n = (long long)units_per_chunk * cur.ns;
         if (i < cur.base + n) {
             const long long local = i - cur.base;
             const int y = (int)(local / cur.ns);
             u.b = cur.b;
-            u.split = (int)(local % cur.ns);
+            u.split = cur.plan.split((int)(local % cur.ns));
             u.kvh = y / n_hb;
             u.hb = y % n_hb;
             u.key0 = u.split * CH;
             u.nkeys = min(CH, cur.seqlen - u.key0);
             u.ntiles = (u.nkeys + KT - 1) / KT;
+            u.seqlen = cur.seqlen;
             return true;
         }
         cur.base += n;
         ++cur.b;
-        if (cur.b < B) {
-            cur.seqlen = clamp_seqlen(seqlens, cur.b, S_max);
-            cur.ns = (cur.seqlen + CH - 1) / CH;
-        }
+        if (cur.b < B) start_sequence<CH>(cur, seqlens, S_max, w);
     }
     return false;
 }
@@ -148,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
                     float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
-                    int S_max, int n_splits, float scale_log2, const PageTable pt) {
+                    int S_max, int n_splits, float scale_log2, const PageTable pt, const Window win) {
     using C = Cfg<GT>;
     constexpr int NH = C::NH;
     extern __shared__ uint8_t smem_raw[];
@@ -188,8 +221,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     volatile int *abort_flag = &sm.abort_flag;
 
     UnitCursor cur;
-    cur.seqlen = B > 0 ? clamp_seqlen(seqlens, 0, S_max) : 0;
-    cur.ns = (cur.seqlen + C::CH - 1) / C::CH;
+    if (B > 0) start_sequence<C::CH>(cur, seqlens, S_max, win);
     Unit u;
 
     if (warp == PRODUCER_WARP) {
@@ -200,7 +232,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_prefetch_desc(&tm_v);
             int t = 0, n = 0;   // ring tiles issued, units started
             bool ok = true;
-            for (long long i = blockIdx.x; ok && next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+            for (long long i = blockIdx.x; ok && next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
                  i += gridDim.x, ++n) {
                 // the single Q buffer is free once the previous unit's S^T MMAs completed
                 if (n > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n - 1) & 1, abort_flag, 0x101)) break;
@@ -256,7 +288,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         constexpr uint32_t idesc_s = umma_idesc_bf16(KT, NH, 0, 0);   // K tile (K-major) x Q rows (K-major)
         constexpr uint32_t idesc_o = umma_idesc_bf16(D, NH, 1, 1);    // V^T (MN-major) x P^T (MN-major)
         int t = 0, n = 0;
-        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             if (!mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x201)) break;
             bool ok = true;
@@ -336,7 +368,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int tid = threadIdx.x;                       // key row of each tile; dim row of O^T
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         int n = 0;
-        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, u);
+        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             const int h0 = u.kvh * G + u.hb * GT;
             bool ok = mbar_wait(smem_u32(&sm.s_full), n & 1, abort_flag, 0x301);
@@ -354,7 +386,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 m[h] = -INFINITY;
 #pragma unroll
                 for (int j = 0; j < C::TPC; ++j)
-                    if (j < u.ntiles && j * KT + tid < u.nkeys) m[h] = fmaxf(m[h], __uint_as_float(sv[j][h]));
+                    if (j < u.ntiles && j * KT + tid < u.nkeys && window_keeps(u.key0 + j * KT + tid, u.seqlen, win))
+                        m[h] = fmaxf(m[h], __uint_as_float(sv[j][h]));
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], o));
                 if (lane == 0) sm.red_m[n & 1][warp][h] = m[h];
@@ -373,7 +406,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
             for (int j = 0; j < C::TPC; ++j) {
                 if (j >= u.ntiles) break;
-                const bool valid = j * KT + tid < u.nkeys;
+                const bool valid = j * KT + tid < u.nkeys && window_keeps(u.key0 + j * KT + tid, u.seqlen, win);
                 uint32_t pk[NH / 2];
 #pragma unroll
                 for (int h2 = 0; h2 < NH / 2; ++h2) {
@@ -439,14 +472,15 @@ constexpr int COMBINE_THREADS = 128;
 __global__ void __launch_bounds__(COMBINE_THREADS)
 decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__ ws_ml,
                       const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o,
-                      float *__restrict__ lse, int n_q, int n_splits, int S_max, int chunk) {
+                      float *__restrict__ lse, int n_q, int n_splits, int S_max, int chunk, Window win) {
     __shared__ float red[4][D];
     __shared__ float part[4];
     const int h = blockIdx.x, b = blockIdx.y;
     const int tid = threadIdx.x, g = tid >> 5, lane = tid & 31;
     int seqlen = seqlens[b];
     seqlen = seqlen < 0 ? 0 : (seqlen > S_max ? S_max : seqlen);
-    const int ns = (seqlen + chunk - 1) / chunk;
+    const ChunkPlan plan = chunk_plan(seqlen, chunk, win);
+    const int ns = plan.n;   // chunks written for this sequence: splits plan.split(0 .. ns-1)
     const size_t row = (size_t)b * n_q + h;
     const float2 *ml = ws_ml + row * n_splits;
     if (ns == 0) {
@@ -456,7 +490,7 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
     }
     // M = max over chunks
     float M = -INFINITY;
-    for (int s = tid; s < ns; s += COMBINE_THREADS) M = fmaxf(M, ml[s].x);
+    for (int c = tid; c < ns; c += COMBINE_THREADS) M = fmaxf(M, ml[plan.split(c)].x);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     if (lane == 0) part[g] = M;
@@ -467,7 +501,8 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
     float L = 0.f;
     const float *base = ws_o + row * n_splits * (size_t)D + lane * 4;
 #pragma unroll 4
-    for (int s = g; s < ns; s += 4) {
+    for (int c = g; c < ns; c += 4) {
+        const int s = plan.split(c);
         const float2 m_l = ml[s];
         const float w = ex2(m_l.x - M);
         const float4 v = __ldg(reinterpret_cast<const float4 *>(base + (size_t)s * D));

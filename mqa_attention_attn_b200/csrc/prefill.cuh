@@ -130,6 +130,9 @@ struct Params {
     // head) instead of head-major.
     const int32_t *cu_q, *cu_k;
     int total_q, total_k;
+    // Sliding window (the WINDOW kernel, causal): a query at position p sees
+    // key j iff j <= p and (p - j < window or j < n_sink).
+    int window, n_sink;
     __nv_bfloat16 *o;      // varlen: rows of a tile that ends past its sequence are stored directly
 };
 
@@ -146,12 +149,18 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return ok;
 }
 
-template <int D, bool VARLEN>
+// MODE: kDense (BHSD batch), kVarlen (packed batch), kWindow (BHSD, causal
+// sliding window with sink keys).
+enum : int { kDense = 0, kVarlen = 1, kWindow = 2 };
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                const Params p) {
     using C = Cfg<D>;
+    constexpr bool VARLEN = MODE == kVarlen;
+    constexpr bool WINDOW = MODE == kWindow;
     extern __shared__ uint8_t smem_raw[];
     Smem<D> &sm = *reinterpret_cast<Smem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -198,6 +207,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             nt[t] = keys > 0 ? (keys + BN - 1) / BN : 0;   // 0: no row of the tile sees a key
         }
     }
+    // Key tiles visited, as iterations j = 0, 1, ...: normally key tile j. With
+    // a window: the tiles holding sink keys, then the tiles from the first
+    // window of the CTA's earliest row (tile 0's first position) up to each
+    // tile's last causal key; tiles between sinks and window are skipped.
+    int nsk = 0, jw0 = 0;
+    if constexpr (WINDOW) {
+        nsk = (min(p.n_sink, Skv) + BN - 1) / BN;
+        const int lo = max(0, p0[0] + (Skv - Sq) - p.window + 1);   // first key of any row's window
+        jw0 = max(lo / BN, nsk);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+            if (nt[t] > 0) nt[t] = nsk + max(0, nt[t] - jw0);
+    }
+    auto key_tile = [&](int j) { return (WINDOW && j >= nsk) ? jw0 + (j - nsk) : j; };
     const int nmax = max(nt[0], nt[1]);
 
     // ---- setup: barriers (warp 0), TMEM (warp 1)
@@ -271,7 +294,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (VARLEN)
                         tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, kvh, k0 + j * BN);
                     else
-                        tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, j * BN,
+                        tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, key_tile(j) * BN,
                                     b * p.n_kv + kvh);
                 ++issued;
             }
@@ -298,7 +321,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (VARLEN)
                         tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, kvh, k0 + j * BN);
                     else
-                        tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, j * BN,
+                        tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, key_tile(j) * BN,
                                     b * p.n_kv + kvh);
                 ++issued;
             }
@@ -409,14 +432,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int c = 0; c < BN / 32; ++c)
                     tmem_ld32(trow + colS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c]));
                 tmem_wait_ld();
-                const int kbase = j * BN;
+                const int kbase = key_tile(j) * BN;
                 // causal / key-count mask: only on tiles that cross some row's limit
-                const bool masked = __any_sync(0xffffffffu, kbase + BN - 1 > lim);
+                bool cut = kbase + BN - 1 > lim;
+                // window: keys left of the row's window that are not sink keys
+                const int wlo = WINDOW ? lim - p.window + 1 : 0;
+                if constexpr (WINDOW) cut = cut || (kbase < wlo && kbase + BN > p.n_sink);
+                const bool masked = __any_sync(0xffffffffu, cut);
                 if (masked) {
                     const int rem = lim - kbase;
 #pragma unroll
                     for (int e = 0; e < BN; ++e)
                         if (e > rem) x[e] = 0xff800000u;   // -inf
+                    if constexpr (WINDOW) {
+                        const int rem_lo = wlo - kbase, rem_sink = p.n_sink - kbase;
+#pragma unroll
+                        for (int e = 0; e < BN; ++e)
+                            if (e < rem_lo && e >= rem_sink) x[e] = 0xff800000u;
+                    }
                 }
                 // row maximum (four independent 3-input max chains)
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -462,7 +495,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // is off by default.
                 // a row with no visible key yet keeps m = -inf: exponentiate
                 // against 0 instead (every p is then 0)
-                const float m_use = (VARLEN && m_run == -INFINITY) ? 0.f : m_run;
+                const float m_use = ((VARLEN || WINDOW) && m_run == -INFINITY) ? 0.f : m_run;
                 const float2 nm2 = make_float2(-m_use, -m_use);
                 float2 rs = make_float2(0.f, 0.f);
                 // one chunk of exponentials; which pairs take the FMA-pipe
