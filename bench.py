@@ -61,10 +61,11 @@ def prefill_bytes(w) -> float:
                  + 4 * w.B * w.n_q * w.Sq)
 
 
-def decode_bytes(w, seqlens) -> float:
-    """K and V rows below each sequence's length, q, o (bf16) and lse (fp32)."""
+def decode_bytes(w, seqlens, cache_elem_bytes=2) -> float:
+    """K and V rows below each sequence's length (2 bytes per element, or 1
+    for an FP8 cache), q, o (bf16) and lse (fp32)."""
     total_keys = float(sum(int(x) for x in seqlens))
-    kv = total_keys * w.n_kv * (w.d_qk + w.d_v) * 2
+    kv = total_keys * w.n_kv * (w.d_qk + w.d_v) * cache_elem_bytes
     return kv + w.B * w.n_q * (w.d_qk * 2 + w.d_v * 2 + 4)
 
 
@@ -295,6 +296,21 @@ def run_ours(args):
     do_d = args.only in ("all", "decode")
     do_m = args.only in ("all", "mla")
     do_g = args.only in ("all", "paged")
+    do_f = args.only in ("all", "fp8")
+
+    # the GQA decode workload with its cache in e4m3, one scale per KV head
+    if do_f:
+        def to_e4m3(x):
+            amax = x.float().abs().amax(dim=(0, 2, 3)).clamp_min(1e-6)
+            sc = (amax / 448.0).float()
+            return (x.float() / sc[None, :, None, None]).to(torch.float8_e4m3fn), sc.contiguous()
+        k8, ks8 = to_e4m3(kc)
+        v8, vs8 = to_e4m3(vc)
+        of8 = torch.empty_like(od)
+        lf8 = torch.empty_like(ld)
+        work8 = torch.empty(binding.decode_fp8_workspace_bytes(wd.B, wd.n_q, wd.n_kv, wd.Skv), dtype=torch.uint8,
+                            device=dev)
+        by_f = decode_bytes(wd, seqlens, cache_elem_bytes=1)
 
     # the GQA decode workload again, its cache cut into 64-token pages placed
     # in a pool in a seeded random order (the paged-cache serving layout)
@@ -319,7 +335,7 @@ def run_ours(args):
         og = torch.empty_like(od)
         lg = torch.empty_like(ld)
 
-    def step(times_p, times_d, times_m=None, times_g=None):
+    def step(times_p, times_d, times_m=None, times_g=None, times_f=None):
         if do_p:
             cold_l2(1.0)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -353,6 +369,15 @@ def run_ours(args):
             e7.record(stream)
             if times_g is not None:
                 times_g.append((e6, e7))
+        if do_f:
+            cold_l2(5.0)
+            e8, e9 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e8.record(stream)
+            binding.attn_decode_fp8(qd, k8, v8, ks8, vs8, sl_dev, wd.scale, o=of8, lse=lf8, workspace=work8,
+                                    stream=stream)
+            e9.record(stream)
+            if times_f is not None:
+                times_f.append((e8, e9))
 
     def barrier():
         if ws > 1:
@@ -365,12 +390,12 @@ def run_ours(args):
     barrier()
     assert binding.device_status(stream) == 0, "device status not clean after warm-up"
 
-    tp, td, tm, tg = [], [], [], []
+    tp, td, tm, tg, tf = [], [], [], [], []
     with ClockSampler(torch.cuda.current_device()) as clocks:
         barrier()
         t_wall0 = time.perf_counter()
         for _ in range(args.steps):
-            step(tp, td, tm, tg)
+            step(tp, td, tm, tg, tf)
         barrier()
         t_wall = time.perf_counter() - t_wall0
     st = binding.device_status(stream)
@@ -380,6 +405,8 @@ def run_ours(args):
     ms_m = [a.elapsed_time(b) for a, b in tm] or [float("nan")]
     ms_g = [a.elapsed_time(b) for a, b in tg] or [float("nan")]
     mean_g = sum(ms_g) / len(ms_g)
+    ms_f = [a.elapsed_time(b) for a, b in tf] or [float("nan")]
+    mean_f = sum(ms_f) / len(ms_f)
     mean_m = sum(ms_m) / len(ms_m)
     mean_p = sum(ms_p) / len(ms_p)
     mean_d = sum(ms_d) / len(ms_d)
@@ -487,6 +514,12 @@ def run_ours(args):
                          "gbs": by_d / (mean_g / 1e3) / 1e9, "frac_of_peak": by_d / (mean_g / 1e3) / 1e9 / peak_bw,
                          "algorithmic_bytes": by_d,
                          "kernels": "attn::dec::decode_split_kernel<4, paged> + decode_combine_kernel"},
+        "fp8_decode": {"workload": f"{wd.name}, e4m3 cache with one scale per KV head", "ms": mean_f,
+                       "gbs": (by_f / (mean_f / 1e3) / 1e9) if do_f else None,
+                       "frac_of_peak": (by_f / (mean_f / 1e3) / 1e9 / peak_bw) if do_f else None,
+                       "speedup_vs_bf16_cache": (mean_d / mean_f) if (do_f and do_d) else None,
+                       "algorithmic_bytes": by_f if do_f else None,
+                       "kernels": "attn::dec::decode_split_kernel<4, fp8> + decode_combine_kernel"},
     }
 
     cpu_baseline = None
@@ -511,7 +544,7 @@ def run_ours(args):
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
             "clocks": clocks.summary(),
-            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m) + 2 * int(do_g)) * args.steps,
+            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m) + 2 * int(do_g) + 2 * int(do_f)) * args.steps,
             "wall_s_timed_region": t_wall,
         }
         print(json.dumps(line), flush=True)
@@ -540,7 +573,7 @@ def main():
                     help="query rows of the headline workload per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla", "paged"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla", "paged", "fp8"],
                     help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
     if args.impl == "reference":

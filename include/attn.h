@@ -187,6 +187,38 @@ int attn_decode_window(const void *q, const void *kcache, const void *vcache, co
                        void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_decode_fp8 -- attn_decode against an FP8 (e4m3) KV cache with one
+ * scale per KV head. Source: "Flash Attention 3 and Multi-Headed Latent
+ * Attention" (misar.blog), FP8 section (8-bit e4m3 operands with scaling
+ * factors), and "Attention deep dive" (askaiml.pages.dev), section 5
+ * (quantized FP8 / INT8 KV caches halve KV memory).
+ *
+ *   q        [B, n_q, 128] bf16, contiguous (|q| < 65504: the scores are
+ *            computed in f16 x f16 products with fp32 accumulation)
+ *   kcache, vcache: one byte per element (e4m3: 1 sign, 4 exponent, 3
+ *            mantissa bits, bias 7, no infinities); element (b, g, j, c) at
+ *            byte offset b*stride_b + g*stride_h + j*stride_s + c (strides in
+ *            ELEMENTS = bytes, multiples of 16, stride_s >= 128)
+ *   k_scale, v_scale: [n_kv] fp32 on the device; key (b, g, j) is
+ *            e4m3(bytes) * k_scale[g], value likewise with v_scale[g]
+ *   seqlens, o, lse, scale: as attn_decode
+ *   workspace: at least attn_decode_fp8_workspace_bytes(...) bytes, 256-byte
+ *            aligned, caller-owned.
+ * The result is attention over the dequantized cache (the e4m3 values times
+ * their scales), computed exactly as attn_decode computes it for a bf16
+ * cache; half the bytes cross HBM. Supported: head dim 128, n_q / n_kv a
+ * power of two. Returns ATTN_OK or an error code (nothing launched on
+ * error).
+ */
+int attn_decode_fp8_workspace_bytes(int B, int n_q, int n_kv, int S_max, size_t *bytes);
+int attn_decode_fp8(const void *q, const void *kcache, const void *vcache, const float *k_scale,
+                    const float *v_scale, const int32_t *seqlens, void *o, float *lse,
+                    int B, int n_q, int n_kv, int S_max,
+                    int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                    int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
+                    float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_paged -- attn_decode against a paged KV cache.
  * Source: "Attention deep dive" (askaiml.pages.dev), section 5 (production
  * engines keep the KV cache in fixed-size pages addressed through a page

@@ -64,6 +64,11 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_window.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 + [_i, _i] +
                                          [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode_window.restype = _i
+        L.attn_decode_fp8_workspace_bytes.argtypes = [_i] * 4 + [ctypes.POINTER(ctypes.c_size_t)]
+        L.attn_decode_fp8_workspace_bytes.restype = _i
+        L.attn_decode_fp8.argtypes = ([_vp] * 8 + [_i] * 4 + [_i64] * 6 +
+                                      [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_decode_fp8.restype = _i
         L.attn_decode_paged.argtypes = ([_vp] * 7 + [_i] * 8 + [_i64] * 6 +
                                         [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode_paged.restype = _i
@@ -229,6 +234,43 @@ def attn_decode_window(q, kcache, vcache, seqlens, window: int, n_sink: int, sca
                                   B, n_q, n_kv, d_qk, d_v, S_max, *ks, *vs, int(window), int(n_sink), float(scale),
                                   _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_decode_window")
+    return o, lse
+
+
+def decode_fp8_workspace_bytes(B, n_q, n_kv, S_max) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().attn_decode_fp8_workspace_bytes(B, n_q, n_kv, S_max, ctypes.byref(out)),
+           "attn_decode_fp8_workspace_bytes")
+    return int(out.value)
+
+
+def attn_decode_fp8(q, kcache, vcache, k_scale, v_scale, seqlens, scale: float, o=None, lse=None, workspace=None,
+                    stream=None, want_lse=True):
+    """Decode against an e4m3 cache: kcache/vcache [B,n_kv,S_max,128] of
+    torch.float8_e4m3fn (or uint8 bytes), any strides with a unit inner
+    stride; k_scale/v_scale fp32 [n_kv] on the device."""
+    B, n_q, d = q.shape
+    _, n_kv, S_max, _ = kcache.shape
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    for t in (kcache, vcache):
+        if t.element_size() != 1 or not t.is_cuda:
+            raise ValueError("the FP8 cache must be a one-byte-per-element CUDA tensor")
+    for t in (k_scale, v_scale):
+        if t.dtype != torch.float32 or not t.is_cuda or t.numel() != n_kv:
+            raise ValueError("k_scale / v_scale must be fp32 CUDA tensors of n_kv entries")
+    ks, vs = _elem_strides(kcache), _elem_strides(vcache)
+    if o is None:
+        o = torch.empty((B, n_q, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(decode_fp8_workspace_bytes(B, n_q, n_kv, S_max), 1), dtype=torch.uint8,
+                                device=q.device)
+    rc = lib().attn_decode_fp8(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(k_scale), _ptr(v_scale), _ptr(seqlens),
+                               _ptr(o), _ptr(lse), B, n_q, n_kv, S_max, *ks, *vs, float(scale), _ptr(workspace),
+                               workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_decode_fp8")
     return o, lse
 
 

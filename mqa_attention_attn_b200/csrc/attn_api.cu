@@ -45,10 +45,10 @@ CUtensorMapSwizzle swizzle_for(int row_bytes) {
                             : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-// bf16 tensor map of rank `rank`: dims[0] is the contiguous one; strides in
-// bytes for dims 1..rank-1.
+// Tensor map of rank `rank` (bf16 elements, or bytes): dims[0] is the
+// contiguous one; strides in bytes for dims 1..rank-1.
 bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
-              const uint32_t *box, int row_bytes) {
+              const uint32_t *box, int row_bytes, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t gdim[5], gstr[4];
@@ -59,7 +59,7 @@ bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims
         estr[i] = 1;
     }
     for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr,
+    CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr,
                     bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(row_bytes),
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -239,16 +239,17 @@ struct CacheView {
     attn::dec::PageTable pt;           // pt.table == nullptr: contiguous
     int page_size;
     attn::dec::Window win;             // sliding window (window 0: none)
+    attn::dec::Fp8Scales fs;           // FP8 cache: per-KV-head scales
 };
 
-template <int GT, bool PAGED>
+template <int GT, bool PAGED, bool FP8 = false>
 int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens, void *o, float *lse, int B,
                       int n_q, int n_kv, int S_max, float scale, void *ws, cudaStream_t stream) {
     using namespace attn::dec;
-    using C = Cfg<GT>;
+    using C = Cfg<GT, FP8>;
     const int G = n_q / n_kv;
     const int n_hb = G / GT;
-    const int n_splits = decode_n_splits(G, S_max);
+    const int n_splits = (S_max + C::CH - 1) / C::CH;
     CUtensorMap tq, tk, tv;
     {
         // the group's query rows: [B][n_q][128], box = 64 dims x NH heads
@@ -265,6 +266,14 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
         const uint64_t vstr[3] = {(uint64_t)cv.vs[1] * 2, (uint64_t)cv.vs[2] * 2, (uint64_t)cv.vs[0] * 2};
         if (!make_map(&tk, cv.k, 4, dims, kstr, box, 128)) return ATTN_ERR_CUDA;
         if (!make_map(&tv, cv.v, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
+    } else if (FP8) {
+        // one-byte e4m3 elements: [dim][token][kv head][sequence], one 128-byte box per row
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S_max, (uint64_t)n_kv, (uint64_t)B};
+        const uint32_t box[4] = {128u, (uint32_t)KT, 1u, 1u};
+        const uint64_t kstr[3] = {(uint64_t)cv.ks[2], (uint64_t)cv.ks[1], (uint64_t)cv.ks[0]};
+        const uint64_t vstr[3] = {(uint64_t)cv.vs[2], (uint64_t)cv.vs[1], (uint64_t)cv.vs[0]};
+        if (!make_map(&tk, cv.k, 4, dims, kstr, box, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return ATTN_ERR_CUDA;
+        if (!make_map(&tv, cv.v, 4, dims, vstr, box, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return ATTN_ERR_CUDA;
     } else {
         // [dim][token][kv head][sequence]
         const uint64_t dims[4] = {(uint64_t)D, (uint64_t)S_max, (uint64_t)n_kv, (uint64_t)B};
@@ -274,37 +283,51 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
         if (!make_map(&tk, cv.k, 4, dims, kstr, box, 128)) return ATTN_ERR_CUDA;
         if (!make_map(&tv, cv.v, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
     }
-    const size_t smem = smem_bytes<GT>();
+    const size_t smem = smem_bytes<GT, FP8>();
     static uint64_t attr_done = 0;
-    if (!ensure_smem_attr(decode_split_kernel<GT, PAGED>, smem, attr_done)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(decode_split_kernel<GT, PAGED, FP8>, smem, attr_done)) return ATTN_ERR_CUDA;
     float *ws_o = reinterpret_cast<float *>(ws);
     size_t o_bytes = (size_t)B * n_q * n_splits * D * sizeof(float);
     o_bytes = (o_bytes + 255) & ~size_t(255);
     float2 *ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(ws) + o_bytes);
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
-    // persistent: two CTAs per SM, never more than the largest possible unit count
+    // persistent: as many CTAs as fit on the SMs at once (two per SM), never
+    // more than the largest possible unit count
     const int n_sm = sm_count();
     if (n_sm <= 0) return ATTN_ERR_CUDA;
+    constexpr int threads = FP8 ? THREADS_FP8 : THREADS;
+    static int per_sm[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+    if (per_sm[dev] == 0) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, decode_split_kernel<GT, PAGED, FP8>, threads, smem) !=
+                cudaSuccess ||
+            nb < 1)
+            return ATTN_ERR_CUDA;
+        per_sm[dev] = nb;
+    }
     const long long max_units = (long long)B * n_kv * n_hb * n_splits;
-    const int grid = (int)(max_units < 2LL * n_sm ? max_units : 2LL * n_sm);
-    decode_split_kernel<GT, PAGED><<<grid, THREADS, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q, n_kv,
-                                                                    G, n_hb, S_max, n_splits, scale_log2, cv.pt,
-                                                                    cv.win);
+    const long long resident = (long long)per_sm[dev] * n_sm;
+    const int grid = (int)(max_units < resident ? max_units : resident);
+    decode_split_kernel<GT, PAGED, FP8><<<grid, threads, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q,
+                                                                         n_kv, G, n_hb, S_max, n_splits, scale_log2,
+                                                                         cv.pt, cv.win, cv.fs);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
         ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH, cv.win);
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-template <bool PAGED>
+template <bool PAGED, bool FP8 = false>
 int dispatch_decode_gqa(int G, const void *q, const CacheView &cv, const int32_t *seqlens, void *o, float *lse,
                         int B, int n_q, int n_kv, int S_max, float scale, void *ws, cudaStream_t s) {
     switch (decode_head_block(G)) {
-        case 1: return launch_decode_gqa<1, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
-        case 2: return launch_decode_gqa<2, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
-        case 4: return launch_decode_gqa<4, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
-        case 8: return launch_decode_gqa<8, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
-        default: return launch_decode_gqa<16, PAGED>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 1: return launch_decode_gqa<1, PAGED, FP8>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 2: return launch_decode_gqa<2, PAGED, FP8>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 4: return launch_decode_gqa<4, PAGED, FP8>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        case 8: return launch_decode_gqa<8, PAGED, FP8>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
+        default: return launch_decode_gqa<16, PAGED, FP8>(q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, ws, s);
     }
 }
 
@@ -537,6 +560,46 @@ int attn_decode_window(const void *q, const void *kcache, const void *vcache, co
     return decode_entry(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, d_qk, d_v, S_max, k_stride_b, k_stride_h,
                         k_stride_s, v_stride_b, v_stride_h, v_stride_s, scale, workspace, workspace_bytes, stream,
                         attn::dec::Window{window, n_sink});
+}
+
+int attn_decode_fp8_workspace_bytes(int B, int n_q, int n_kv, int S_max, size_t *bytes) {
+    if (!bytes || B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    const int ch = attn::dec::chunk_keys(decode_head_block(n_q / n_kv), true);
+    *bytes = decode_ws_bytes(B, n_q, 128, (S_max + ch - 1) / ch);
+    return ATTN_OK;
+}
+
+int attn_decode_fp8(const void *q, const void *kcache, const void *vcache, const float *k_scale,
+                    const float *v_scale, const int32_t *seqlens, void *o, float *lse, int B, int n_q, int n_kv,
+                    int S_max, int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s, int64_t v_stride_b,
+                    int64_t v_stride_h, int64_t v_stride_s, float scale, void *workspace, size_t workspace_bytes,
+                    attn_stream_t stream) {
+    if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0) return ATTN_OK;
+    if (!q || !kcache || !vcache || !k_scale || !v_scale || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (k_stride_b < 0 || k_stride_h < 0 || k_stride_s < 0 || v_stride_b < 0 || v_stride_h < 0 || v_stride_s < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (k_stride_s < 128 || v_stride_s < 128) return ATTN_ERR_INVALID_ARG;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+    if ((k_stride_b | k_stride_h | k_stride_s | v_stride_b | v_stride_h | v_stride_s) & 15)
+        return ATTN_ERR_MISALIGNED;   // one-byte elements: strides in multiples of 16 bytes
+    size_t need = 0;
+    attn_decode_fp8_workspace_bytes(B, n_q, n_kv, S_max, &need);
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+    CacheView cv{};
+    cv.k = kcache;
+    cv.v = vcache;
+    cv.ks[0] = k_stride_b, cv.ks[1] = k_stride_h, cv.ks[2] = k_stride_s;
+    cv.vs[0] = v_stride_b, cv.vs[1] = v_stride_h, cv.vs[2] = v_stride_s;
+    cv.fs.k_scale = k_scale;
+    cv.fs.v_scale = v_scale;
+    return dispatch_decode_gqa<false, true>(G, q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, workspace,
+                                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,

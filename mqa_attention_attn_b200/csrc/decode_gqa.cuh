@@ -39,8 +39,11 @@ namespace dec {
 constexpr int D = 128;            // head dim (keys and values)
 constexpr int KT = 128;           // keys per tile (the MMA's M for S^T)
 // Keys per chunk (one work unit): 1024 while a head block has at most 8
-// heads, 512 for 16 (the chunk's scores then fill the same registers).
-__host__ __device__ constexpr int chunk_keys(int GT) { return GT <= 8 ? 1024 : 512; }
+// heads, 512 for 16 (the chunk's scores then fill the same registers); 512
+// for the FP8 cache (its CTAs have two more warps and fewer registers each).
+__host__ __device__ constexpr int chunk_keys(int GT, bool fp8 = false) {
+    return (GT <= 8 && !fp8) ? 1024 : 512;
+}
 constexpr int NSTAGE = ATTN_DEC_STAGES;
 constexpr int BOX_BYTES = KT * 128;         // one 64-dim box: 128 rows x 128 B
 constexpr int TILE_BYTES = 2 * BOX_BYTES;   // 32 KB
@@ -48,11 +51,17 @@ constexpr int NSW = 4;            // softmax warps (TMEM lane quarters)
 constexpr int PRODUCER_WARP = 4;
 constexpr int MMA_WARP = 5;
 constexpr int THREADS = 6 * 32;
+// FP8 (e4m3) cache: TMA brings 128 x 128-byte tiles into an 8-bit ring and
+// two more warps (6, 7) widen them to the f16 tiles the MMAs read.
+constexpr int CONV_WARP0 = 6;
+constexpr int THREADS_FP8 = 8 * 32;
+constexpr int NSTAGE8 = 2;
+constexpr int TILE8_BYTES = KT * D;         // 16 KB: 128 rows x 128 one-byte values
 
-template <int GT>
+template <int GT, bool FP8 = false>
 struct Cfg {
     static constexpr int NH = GT < 8 ? 8 : GT;             // MMA N (query-head columns)
-    static constexpr int CH = chunk_keys(GT);               // keys per unit
+    static constexpr int CH = chunk_keys(GT, FP8);          // keys per unit
     static constexpr int TPC = CH / KT;                     // tiles per unit
     static constexpr int QBOX = NH * 128;                   // one 64-dim half of the Q rows
     static constexpr int COL_S = 0;                         // S^T: TPC tiles x NH columns
@@ -62,25 +71,34 @@ struct Cfg {
     static_assert(GT == 1 || GT == 2 || GT == 4 || GT == 8 || GT == 16 || GT == 32, "head block");
 };
 
-template <int GT>
+template <int GT, bool FP8 = false>
 struct Smem {
-    using C = Cfg<GT>;
-    uint8_t ring[NSTAGE][TILE_BYTES];       // 1024-byte aligned (swizzle atoms)
+    using C = Cfg<GT, FP8>;
+    uint8_t ring[NSTAGE][TILE_BYTES];       // 1024-byte aligned (swizzle atoms); f16 when FP8
+    uint8_t ring8[FP8 ? NSTAGE8 : 1][FP8 ? TILE8_BYTES : 1024];   // e4m3 tiles as loaded
     uint8_t q[2][C::QBOX];                  // Q rows, two 64-dim boxes, 128-byte swizzle
     uint8_t p[C::NH / 8][C::CH * 16];       // P^T: [8-head block][key][8 heads] bf16
     float red_m[2][NSW][GT];                // double-buffered by unit parity
     float red_l[2][NSW][GT];
     uint64_t full[NSTAGE];
     uint64_t empty[NSTAGE];
+    uint64_t full8[NSTAGE8], empty8[NSTAGE8];
     uint64_t q_full, q_empty, s_full, p_full, o_full, mma_done;
+    uint64_t q_conv;                        // FP8: Q rows converted to f16
     uint32_t tmem_base;
     int abort_flag;
 };
 
-template <int GT>
+template <int GT, bool FP8 = false>
 constexpr size_t smem_bytes() {
-    return sizeof(Smem<GT>) + 1024;  // + alignment slack
+    return sizeof(Smem<GT, FP8>) + 1024;  // + alignment slack
 }
+
+// FP8 cache scales: element (b, g, j, c) of the cache means
+// e4m3(byte) * k_scale[g] (keys) or * v_scale[g] (values).
+struct Fp8Scales {
+    const float *k_scale, *v_scale;   // [n_kv]; null on the bf16 path
+};
 
 // Sliding window over the cache (window 0: none): of keys 0 .. L-1 a
 // sequence of length L keeps the last `window` and the first `n_sink`.
@@ -176,24 +194,47 @@ __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const in
     return false;
 }
 
-template <int GT, bool PAGED>
-__global__ void __launch_bounds__(THREADS, 2)
+// Widen 8 bytes of e4m3 values (two words) to 8 f16 values (four words).
+// e4m3 -> f16 is exact (every e4m3 value is an f16 value).
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
+    uint4 r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.x) : "h"((unsigned short)(lo & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.y) : "h"((unsigned short)(lo >> 16)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.z) : "h"((unsigned short)(hi & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.w) : "h"((unsigned short)(hi >> 16)));
+    return r;
+}
+__device__ __forceinline__ uint32_t f2_to_h2_sat(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <int GT, bool PAGED, bool FP8 = false>
+__global__ void __launch_bounds__(FP8 ? THREADS_FP8 : THREADS, 2)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
                     float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
-                    int S_max, int n_splits, float scale_log2, const PageTable pt, const Window win) {
-    using C = Cfg<GT>;
+                    int S_max, int n_splits, float scale_log2, const PageTable pt, const Window win,
+                    const Fp8Scales fs) {
+    using C = Cfg<GT, FP8>;
     constexpr int NH = C::NH;
     extern __shared__ uint8_t smem_raw[];
-    Smem<GT> &sm = *reinterpret_cast<Smem<GT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<GT, FP8> &sm =
+        *reinterpret_cast<Smem<GT, FP8> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t warp = warp_id(), lane = lane_id();
     const int units_per_chunk = n_kv * n_hb;   // units of one chunk index of one sequence
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(smem_u32(&sm.full[s]), 1);
+            mbar_init(smem_u32(&sm.full[s]), FP8 ? 2 : 1);   // FP8: one arrive per converter warp
             mbar_init(smem_u32(&sm.empty[s]), 1);
         }
+        for (int s = 0; s < NSTAGE8; ++s) {
+            mbar_init(smem_u32(&sm.full8[s]), 1);
+            mbar_init(smem_u32(&sm.empty8[s]), 2);
+        }
+        mbar_init(smem_u32(&sm.q_conv), 2);
         mbar_init(smem_u32(&sm.q_full), 1);
         mbar_init(smem_u32(&sm.q_empty), 1);
         mbar_init(smem_u32(&sm.s_full), 1);
@@ -241,14 +282,26 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tma_load_3d(smem_u32(sm.q[0]), &tm_q, smem_u32(&sm.q_full), 0, h0, u.b);
                 tma_load_3d(smem_u32(sm.q[1]), &tm_q, smem_u32(&sm.q_full), 64, h0, u.b);
                 for (int j = 0; j < 2 * u.ntiles; ++j, ++t) {
+                    const CUtensorMap *tm = (j < u.ntiles) ? &tm_k : &tm_v;
+                    const int krow = u.key0 + (j < u.ntiles ? j : j - u.ntiles) * KT;
+                    if constexpr (FP8) {
+                        // 8-bit ring, drained by the converter warps
+                        const int s8 = t % NSTAGE8;
+                        if (!mbar_wait(smem_u32(&sm.empty8[s8]), ((t / NSTAGE8) & 1) ^ 1, abort_flag, 0x105)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t full8 = smem_u32(&sm.full8[s8]);
+                        mbar_arrive_expect_tx(full8, TILE8_BYTES);
+                        tma_load_4d(smem_u32(sm.ring8[s8]), tm, full8, 0, krow, u.kvh, u.b);
+                        continue;
+                    }
                     const int s = t % NSTAGE;
                     if (!mbar_wait(smem_u32(&sm.empty[s]), ((t / NSTAGE) & 1) ^ 1, abort_flag, 0x102)) {
                         ok = false;
                         break;
                     }
                     const uint32_t full = smem_u32(&sm.full[s]);
-                    const CUtensorMap *tm = (j < u.ntiles) ? &tm_k : &tm_v;
-                    const int krow = u.key0 + (j < u.ntiles ? j : j - u.ntiles) * KT;
                     const uint32_t dst = smem_u32(sm.ring[s]);
                     if constexpr (PAGED) {
                         // boxes holding at least one key below the length; rows of
@@ -278,19 +331,26 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // Do not leave while copies into this CTA's shared memory are in
             // flight: wait (bounded) for the last issued tile of each stage
             // and the last Q load.
-            for (int j = t - 1; j >= 0 && j >= t - NSTAGE; --j)
-                mbar_wait(smem_u32(&sm.full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x103);
+            if constexpr (FP8) {
+                for (int j = t - 1; j >= 0 && j >= t - NSTAGE8; --j)
+                    mbar_wait(smem_u32(&sm.full8[j % NSTAGE8]), (j / NSTAGE8) & 1, nullptr, 0x106);
+            } else {
+                for (int j = t - 1; j >= 0 && j >= t - NSTAGE; --j)
+                    mbar_wait(smem_u32(&sm.full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x103);
+            }
             if (n > 0) mbar_wait(smem_u32(&sm.q_full), (n - 1) & 1, nullptr, 0x104);
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
         // ---------------- MMA issue (one thread), ring bookkeeping (whole warp) ----------------
-        constexpr uint32_t idesc_s = umma_idesc_bf16(KT, NH, 0, 0);   // K tile (K-major) x Q rows (K-major)
-        constexpr uint32_t idesc_o = umma_idesc_bf16(D, NH, 1, 1);    // V^T (MN-major) x P^T (MN-major)
+        // K tile (K-major) x Q rows (K-major); V^T (MN-major) x P^T (MN-major);
+        // operands bf16, or f16 on the FP8 path (widened tiles)
+        constexpr uint32_t idesc_s = FP8 ? umma_idesc_f16(KT, NH, 0, 0) : umma_idesc_bf16(KT, NH, 0, 0);
+        constexpr uint32_t idesc_o = FP8 ? umma_idesc_f16(D, NH, 1, 1) : umma_idesc_bf16(D, NH, 1, 1);
         int t = 0, n = 0;
         for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
-            if (!mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x201)) break;
+            if (!mbar_wait(smem_u32(FP8 ? &sm.q_conv : &sm.q_full), n & 1, abort_flag, 0x201)) break;
             bool ok = true;
             for (int j = 0; j < u.ntiles; ++j) {
                 const int g = t + j, s = g % NSTAGE;
@@ -328,7 +388,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     break;
                 }
                 const int rows = u.nkeys - j * KT;   // valid value rows of this tile
-                if (rows < KT) {
+                if (!FP8 && rows < KT) {             // (the converter clears them on the FP8 path)
                     // Rows past the sequence end get weight 0, but 0 * (NaN or
                     // Inf) is not 0: clear them so that whatever the cache holds
                     // beyond the length cannot reach the output.
@@ -363,6 +423,62 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (lane == 0) umma_commit(smem_u32(&sm.mma_done));
         __syncwarp();
         mbar_wait(smem_u32(&sm.mma_done), 0, nullptr, 0x205);
+    } else if (FP8 && warp >= CONV_WARP0) {
+        // ---------------- FP8: widen e4m3 tiles to f16 (two warps, 64 rows each) ----------------
+        const int cw = (int)warp - CONV_WARP0;
+        int t = 0, n = 0;
+        bool ok = true;
+        for (long long i = blockIdx.x; ok && next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
+             i += gridDim.x, ++n) {
+            // the unit's Q rows, bf16 -> f16 in place (same byte positions)
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x401));
+            if (!ok) break;
+            for (int c = cw * 32 + (int)lane; c < 2 * C::QBOX / 16; c += 64) {
+                const uint32_t a = smem_u32(sm.q[0]) + (uint32_t)c * 16u;
+                uint4 w = lds128(a);
+                float2 f;
+                f = bf2_to_f2(w.x), w.x = f2_to_h2_sat(f.x, f.y);
+                f = bf2_to_f2(w.y), w.y = f2_to_h2_sat(f.x, f.y);
+                f = bf2_to_f2(w.z), w.z = f2_to_h2_sat(f.x, f.y);
+                f = bf2_to_f2(w.w), w.w = f2_to_h2_sat(f.x, f.y);
+                sts128(a, w);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.q_conv));
+            for (int j = 0; j < 2 * u.ntiles; ++j, ++t) {
+                const int s8 = t % NSTAGE8, s = t % NSTAGE;
+                bool w_ok = mbar_wait(smem_u32(&sm.full8[s8]), (t / NSTAGE8) & 1, abort_flag, 0x402);
+                w_ok = w_ok && mbar_wait(smem_u32(&sm.empty[s]), ((t / NSTAGE) & 1) ^ 1, abort_flag, 0x403);
+                ok = __all_sync(0xffffffffu, w_ok);
+                if (!ok) break;
+                // rows past the length become 0 (their scores are masked; 0 * NaN would not be 0)
+                const int rows = u.nkeys - (j < u.ntiles ? j : j - u.ntiles) * KT;
+                const uint32_t src = smem_u32(sm.ring8[s8]), dst = smem_u32(sm.ring[s]);
+#pragma unroll 4
+                for (int k = 0; k < 16; ++k) {
+                    const int idx = k * 32 + (int)lane;          // 16-byte source chunks of this warp's rows
+                    const int r = cw * 64 + (idx >> 3), c = idx & 7;   // row; chunk = dims 16c .. 16c+15
+                    uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
+                    if (r < rows) {
+                        const uint4 w = lds128(src + (uint32_t)r * 128u + (uint32_t)((c ^ (r & 7)) << 4));
+                        o0 = e4m3x8_to_f16x8(w.x, w.y);
+                        o1 = e4m3x8_to_f16x8(w.z, w.w);
+                    }
+                    // dims 16c .. 16c+15 land in 64-dim box c/4, 16-byte chunks 2(c%4) and 2(c%4)+1
+                    const int c0 = (c & 3) * 2;
+                    const uint32_t row = dst + (uint32_t)(c >> 2) * BOX_BYTES + (uint32_t)r * 128u;
+                    sts128(row + (uint32_t)((c0 ^ (r & 7)) << 4), o0);
+                    sts128(row + (uint32_t)(((c0 + 1) ^ (r & 7)) << 4), o1);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&sm.full[s]));
+                    mbar_arrive(smem_u32(&sm.empty8[s8]));
+                }
+            }
+        }
     } else if (warp < NSW) {
         // ---------------- softmax + partial output (128 threads, thread = TMEM lane) ----------------
         const int tid = threadIdx.x;                       // key row of each tile; dim row of O^T
@@ -371,6 +487,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             const int h0 = u.kvh * G + u.hb * GT;
+            // FP8: the key scale of this KV head scales every score
+            const float su = FP8 ? scale_log2 * fs.k_scale[u.kvh] : scale_log2;
             bool ok = mbar_wait(smem_u32(&sm.s_full), n & 1, abort_flag, 0x301);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
@@ -399,10 +517,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 float mm = sm.red_m[n & 1][0][h];
 #pragma unroll
                 for (int w = 1; w < NSW; ++w) mm = fmaxf(mm, sm.red_m[n & 1][w][h]);
-                mc[h] = mm * scale_log2;     // finite: every unit holds at least one key
+                mc[h] = mm * su;             // finite: every unit holds at least one key
                 l[h] = 0.f;
             }
-            // p = 2^(s * scale * log2 e - m), written as P^T rows of bf16 [key][8 heads]
+            // p = 2^(s * scale * log2 e - m), written as P^T rows [key][8 heads] (bf16; f16 on the FP8 path)
 #pragma unroll
             for (int j = 0; j < C::TPC; ++j) {
                 if (j >= u.ntiles) break;
@@ -411,12 +529,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int h2 = 0; h2 < NH / 2; ++h2) {
                     float p0 = 0.f, p1 = 0.f;
-                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[j][2 * h2]), scale_log2, -mc[2 * h2]));
+                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[j][2 * h2]), su, -mc[2 * h2]));
                     if (2 * h2 + 1 < GT && valid)
-                        p1 = ex2(fmaf(__uint_as_float(sv[j][2 * h2 + 1]), scale_log2, -mc[2 * h2 + 1]));
+                        p1 = ex2(fmaf(__uint_as_float(sv[j][2 * h2 + 1]), su, -mc[2 * h2 + 1]));
                     if (2 * h2 < GT) l[2 * h2] += p0;
                     if (2 * h2 + 1 < GT) l[2 * h2 + 1] += p1;
-                    pk[h2] = f2_to_bf2(p0, p1);
+                    pk[h2] = FP8 ? f2_to_h2_sat(p0, p1) : f2_to_bf2(p0, p1);
                 }
 #pragma unroll
                 for (int hb8 = 0; hb8 < NH / 8; ++hb8)
@@ -441,9 +559,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             if (named_bar_or(1, NSW * 32, !ok)) break;
             const size_t row0 = (size_t)u.b * n_q + h0;
+            const float vsc = FP8 ? fs.v_scale[u.kvh] : 1.f;   // FP8: the value scale of this KV head
 #pragma unroll
             for (int h = 0; h < GT; ++h)
-                ws_o[((row0 + h) * n_splits + u.split) * D + tid] = __uint_as_float(ov[h]);
+                ws_o[((row0 + h) * n_splits + u.split) * D + tid] = __uint_as_float(ov[h]) * vsc;
 #pragma unroll
             for (int h = 0; h < GT; ++h)
                 if (tid == h) {

@@ -292,6 +292,15 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, i
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// Instruction descriptor for kind::f16 with f16 A and B, fp32 accumulate.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4)                      // D format: f32
+           | ((uint32_t)a_mn << 15)       // A major (A and B format 0: f16)
+           | ((uint32_t)b_mn << 16)       // B major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
 // ----------------------------------------------------------------------------
 // small numeric helpers
 // ----------------------------------------------------------------------------

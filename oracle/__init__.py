@@ -18,6 +18,7 @@ Functions:
   paged_to_cache(pages, block_table, seqlens)    -> cache      page-table gather (layout only)
   sdpa_varlen(q, k, v, cu_q, cu_k, causal, scale) -> (o, lse)  packed batch, one sdpa per sequence
   sdpa_window(q, k, v, causal, window, n_sink, scale, seqlens=None) -> (o, lse) sliding window + sinks
+  dequant_e4m3(bytes, scale)                     -> fp64      FP8 (e4m3) cache values
 
 Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
 d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
@@ -282,3 +283,25 @@ def sdpa_window(q, k, v, causal: bool, window: int, n_sink: int, scale: float, s
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return o, lse
+
+
+def dequant_e4m3(raw, scale=None, head_axis=1):
+    """Values of an FP8 e4m3 cache ("Flash Attention 3 and Multi-Headed Latent
+    Attention", FP8 section: 8-bit e4m3 operands with scaling factors): each
+    byte is 1 sign bit, 4 exponent bits (bias 7) and 3 mantissa bits;
+    exponent 0 is subnormal (m * 2^-9), the pattern S.1111.111 is NaN and
+    there are no infinities (largest finite 448). `scale` [n_kv] multiplies
+    the values of each KV head (axis `head_axis`). Returns float64."""
+    b = np.asarray(raw.cpu().numpy() if hasattr(raw, "cpu") else raw).view(np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = sign * val
+    val = np.where((e == 15) & (b & 7 == 7), np.nan, val)
+    if scale is not None:
+        sc = np.asarray(scale.cpu().numpy() if hasattr(scale, "cpu") else scale, dtype=np.float64)
+        shape = [1] * val.ndim
+        shape[head_axis] = -1
+        val = val * sc.reshape(shape)
+    return val

@@ -104,3 +104,20 @@ def test_sdpa_window_pins():
     keep = [0, 16, 17, 18, 19]
     o_r, l_r = oracle.sdpa(q[:1, :, :1], k[:1, :, keep], v[:1, :, keep], False, 0.3)
     assert np.allclose(o_d[:1], o_r, atol=1e-12) and np.allclose(l_d[:1], l_r, atol=1e-12)
+
+
+def test_dequant_e4m3_matches_an_independent_decoder():
+    """All 256 byte patterns against torch's float8_e4m3fn conversion (an
+    independent implementation), plus the format's landmarks: 448 is the
+    largest finite value, 2^-9 the smallest subnormal, 0x7F / 0xFF are NaN."""
+    import torch
+    raw = np.arange(256, dtype=np.uint8)
+    got = oracle.dequant_e4m3(raw)
+    ref = torch.from_numpy(raw.copy()).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and np.isnan(got[0x7F]) and np.isnan(got[0xFF])
+    assert got[0x38] == 1.0 and got[0xB8] == -1.0
+    # per-head scale along axis 1
+    x = np.full((2, 3, 4), 0x38, np.uint8)
+    assert np.array_equal(oracle.dequant_e4m3(x, [1.0, 0.5, 2.0])[0, :, 0], [1.0, 0.5, 2.0])
