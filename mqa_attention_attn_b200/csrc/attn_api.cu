@@ -76,6 +76,11 @@ bool ensure_smem_attr(K kernel, size_t bytes, uint64_t &done_mask) {
     if (done_mask & bit) return true;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
+    // all of the unified L1 / shared storage as shared memory, so that the
+    // occupancy the grid is sized by counts every CTA that fits
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return false;
     done_mask |= bit;
     return true;
 }
@@ -291,24 +296,16 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
     o_bytes = (o_bytes + 255) & ~size_t(255);
     float2 *ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(ws) + o_bytes);
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
-    // persistent: as many CTAs as fit on the SMs at once (two per SM), never
+    // persistent: as many CTAs as fit on the SMs at once (two per SM while
+    // two fit in the SM's 228 KB of shared memory, with 1 KB reserved per
+    // CTA; the register budget of two is fixed by the launch bounds), never
     // more than the largest possible unit count
     const int n_sm = sm_count();
     if (n_sm <= 0) return ATTN_ERR_CUDA;
     constexpr int threads = FP8 ? THREADS_FP8 : THREADS;
-    static int per_sm[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
-    if (per_sm[dev] == 0) {
-        int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, decode_split_kernel<GT, PAGED, FP8>, threads, smem) !=
-                cudaSuccess ||
-            nb < 1)
-            return ATTN_ERR_CUDA;
-        per_sm[dev] = nb;
-    }
+    const int per_sm = (int)(233472 / (smem + 1024)) >= 2 ? 2 : 1;
     const long long max_units = (long long)B * n_kv * n_hb * n_splits;
-    const long long resident = (long long)per_sm[dev] * n_sm;
+    const long long resident = (long long)per_sm * n_sm;
     const int grid = (int)(max_units < resident ? max_units : resident);
     decode_split_kernel<GT, PAGED, FP8><<<grid, threads, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q,
                                                                          n_kv, G, n_hb, S_max, n_splits, scale_log2,

@@ -38,11 +38,11 @@ namespace dec {
 
 constexpr int D = 128;            // head dim (keys and values)
 constexpr int KT = 128;           // keys per tile (the MMA's M for S^T)
-// Keys per chunk (one work unit): 1024 while a head block has at most 8
-// heads, 512 for 16 (the chunk's scores then fill the same registers); 512
-// for the FP8 cache (its CTAs have two more warps and fewer registers each).
+// Keys per chunk (one work unit): 2048 while a head block has at most 8
+// heads, 1024 for 16 (the chunk's S^T, 16 or 8 tiles x NH columns, then
+// stays within 256 TMEM columns so that two CTAs share an SM).
 __host__ __device__ constexpr int chunk_keys(int GT, bool fp8 = false) {
-    return (GT <= 8 && !fp8) ? 1024 : 512;
+    return (void)fp8, GT <= 8 ? 2048 : 1024;
 }
 constexpr int NSTAGE = ATTN_DEC_STAGES;
 constexpr int BOX_BYTES = KT * 128;         // one 64-dim box: 128 rows x 128 B
@@ -52,9 +52,14 @@ constexpr int PRODUCER_WARP = 4;
 constexpr int MMA_WARP = 5;
 constexpr int THREADS = 6 * 32;
 // FP8 (e4m3) cache: TMA brings 128 x 128-byte tiles into an 8-bit ring and
-// two more warps (6, 7) widen them to the f16 tiles the MMAs read.
+// NCONV more warps (6 ..) widen them to the f16 tiles the MMAs read.
+#ifndef ATTN_DEC_NCONV
+#define ATTN_DEC_NCONV 4
+#endif
+constexpr int NCONV = ATTN_DEC_NCONV;
+static_assert(NCONV == 2 || NCONV == 4, "converter warps");
 constexpr int CONV_WARP0 = 6;
-constexpr int THREADS_FP8 = 8 * 32;
+constexpr int THREADS_FP8 = (6 + NCONV) * 32;
 constexpr int NSTAGE8 = 2;
 constexpr int TILE8_BYTES = KT * D;         // 16 KB: 128 rows x 128 one-byte values
 
@@ -77,13 +82,14 @@ struct Smem {
     uint8_t ring[NSTAGE][TILE_BYTES];       // 1024-byte aligned (swizzle atoms); f16 when FP8
     uint8_t ring8[FP8 ? NSTAGE8 : 1][FP8 ? TILE8_BYTES : 1024];   // e4m3 tiles as loaded
     uint8_t q[2][C::QBOX];                  // Q rows, two 64-dim boxes, 128-byte swizzle
-    uint8_t p[C::NH / 8][C::CH * 16];       // P^T: [8-head block][key][8 heads] bf16
+    uint8_t p[2][C::NH / 8][KT * 16];       // P^T of one tile, two slots: [8-head block][key][8 heads]
     float red_m[2][NSW][GT];                // double-buffered by unit parity
     float red_l[2][NSW][GT];
     uint64_t full[NSTAGE];
     uint64_t empty[NSTAGE];
     uint64_t full8[NSTAGE8], empty8[NSTAGE8];
-    uint64_t q_full, q_empty, s_full, p_full, o_full, mma_done;
+    uint64_t q_full, q_empty, s_full, o_full, mma_done;
+    uint64_t p_full[2], p_empty[2];         // per-tile P hand-off, softmax <-> MMA
     uint64_t q_conv;                        // FP8: Q rows converted to f16
     uint32_t tmem_base;
     int abort_flag;
@@ -211,7 +217,7 @@ __device__ __forceinline__ uint32_t f2_to_h2_sat(float lo, float hi) {
 }
 
 template <int GT, bool PAGED, bool FP8 = false>
-__global__ void __launch_bounds__(FP8 ? THREADS_FP8 : THREADS, 2)
+__global__ void __launch_bounds__(FP8 ? THREADS_FP8 : THREADS, (FP8 && GT >= 16) ? 1 : 2)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
                     float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
@@ -227,18 +233,21 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(smem_u32(&sm.full[s]), FP8 ? 2 : 1);   // FP8: one arrive per converter warp
+            mbar_init(smem_u32(&sm.full[s]), FP8 ? NCONV : 1);   // FP8: one arrive per converter warp
             mbar_init(smem_u32(&sm.empty[s]), 1);
         }
         for (int s = 0; s < NSTAGE8; ++s) {
             mbar_init(smem_u32(&sm.full8[s]), 1);
-            mbar_init(smem_u32(&sm.empty8[s]), 2);
+            mbar_init(smem_u32(&sm.empty8[s]), NCONV);
         }
-        mbar_init(smem_u32(&sm.q_conv), 2);
+        mbar_init(smem_u32(&sm.q_conv), NCONV);
         mbar_init(smem_u32(&sm.q_full), 1);
         mbar_init(smem_u32(&sm.q_empty), 1);
         mbar_init(smem_u32(&sm.s_full), 1);
-        mbar_init(smem_u32(&sm.p_full), NSW * 32);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&sm.p_full[x]), NSW * 32);
+            mbar_init(smem_u32(&sm.p_empty[x]), 1);
+        }
         mbar_init(smem_u32(&sm.o_full), 1);
         mbar_init(smem_u32(&sm.mma_done), 1);
         sm.abort_flag = 0;
@@ -347,7 +356,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // operands bf16, or f16 on the FP8 path (widened tiles)
         constexpr uint32_t idesc_s = FP8 ? umma_idesc_f16(KT, NH, 0, 0) : umma_idesc_bf16(KT, NH, 0, 0);
         constexpr uint32_t idesc_o = FP8 ? umma_idesc_f16(D, NH, 1, 1) : umma_idesc_bf16(D, NH, 1, 1);
-        int t = 0, n = 0;
+        int t = 0, n = 0, pc = 0;   // ring tiles, units, P tiles handed over
         for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             if (!mbar_wait(smem_u32(FP8 ? &sm.q_conv : &sm.q_full), n & 1, abort_flag, 0x201)) break;
@@ -379,11 +388,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             __syncwarp();
             t += u.ntiles;
-            if (!mbar_wait(smem_u32(&sm.p_full), n & 1, abort_flag, 0x203)) break;
-            tc_fence_after();
-            for (int j = 0; j < u.ntiles; ++j) {
+            for (int j = 0; j < u.ntiles; ++j, ++pc) {
                 const int g = t + j, s = g % NSTAGE;
-                if (!mbar_wait(smem_u32(&sm.full[s]), (g / NSTAGE) & 1, abort_flag, 0x204)) {
+                if (!mbar_wait(smem_u32(&sm.full[s]), (g / NSTAGE) & 1, abort_flag, 0x204) ||
+                    !mbar_wait(smem_u32(&sm.p_full[pc & 1]), (pc >> 1) & 1, abort_flag, 0x203)) {
                     ok = false;
                     break;
                 }
@@ -407,10 +415,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int ks = 0; ks < KT / 16; ++ks) {
                         // A = V^T: 16 keys x 128 dims of the tile; B = P^T rows of the same 16 keys
                         const uint64_t ad = umma_smem_desc(smem_u32(sm.ring[s]) + ks * 16 * 128, BOX_BYTES, 1024, 2);
-                        const uint64_t bd = umma_smem_desc(smem_u32(sm.p[0]) + (j * KT + ks * 16) * 16, 128, C::CH * 16, 0);
+                        const uint64_t bd = umma_smem_desc(smem_u32(sm.p[pc & 1][0]) + ks * 16 * 16, 128, KT * 16, 0);
                         umma_ss(tmem + C::COL_O, ad, bd, idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(smem_u32(&sm.empty[s]));
+                    umma_commit(smem_u32(&sm.p_empty[pc & 1]));
                 }
                 __syncwarp();
             }
@@ -424,7 +433,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncwarp();
         mbar_wait(smem_u32(&sm.mma_done), 0, nullptr, 0x205);
     } else if (FP8 && warp >= CONV_WARP0) {
-        // ---------------- FP8: widen e4m3 tiles to f16 (two warps, 64 rows each) ----------------
+        // ---------------- FP8: widen e4m3 tiles to f16 (NCONV warps, 128 / NCONV rows each) ----------------
         const int cw = (int)warp - CONV_WARP0;
         int t = 0, n = 0;
         bool ok = true;
@@ -433,7 +442,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // the unit's Q rows, bf16 -> f16 in place (same byte positions)
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x401));
             if (!ok) break;
-            for (int c = cw * 32 + (int)lane; c < 2 * C::QBOX / 16; c += 64) {
+            for (int c = cw * 32 + (int)lane; c < 2 * C::QBOX / 16; c += NCONV * 32) {
                 const uint32_t a = smem_u32(sm.q[0]) + (uint32_t)c * 16u;
                 uint4 w = lds128(a);
                 float2 f;
@@ -455,21 +464,32 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // rows past the length become 0 (their scores are masked; 0 * NaN would not be 0)
                 const int rows = u.nkeys - (j < u.ntiles ? j : j - u.ntiles) * KT;
                 const uint32_t src = smem_u32(sm.ring8[s8]), dst = smem_u32(sm.ring[s]);
-#pragma unroll 4
-                for (int k = 0; k < 16; ++k) {
-                    const int idx = k * 32 + (int)lane;          // 16-byte source chunks of this warp's rows
-                    const int r = cw * 64 + (idx >> 3), c = idx & 7;   // row; chunk = dims 16c .. 16c+15
-                    uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
-                    if (r < rows) {
-                        const uint4 w = lds128(src + (uint32_t)r * 128u + (uint32_t)((c ^ (r & 7)) << 4));
-                        o0 = e4m3x8_to_f16x8(w.x, w.y);
-                        o1 = e4m3x8_to_f16x8(w.z, w.w);
+                // 16-byte source chunks (16 dims each) of this warp's rows, 32 / NCONV
+                // per lane, in batches of 8: all loads of a batch, then its stores
+                constexpr int CPL = 32 / NCONV;
+#pragma unroll
+                for (int kb = 0; kb < CPL; kb += 8) {
+                    uint4 w[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int idx = (kb + k) * 32 + (int)lane;
+                        const int r = cw * (KT / NCONV) + (idx >> 3), c = idx & 7;
+                        w[k] = r < rows ? lds128(src + (uint32_t)r * 128u + (uint32_t)((c ^ (r & 7)) << 4))
+                                        : make_uint4(0u, 0u, 0u, 0u);
                     }
-                    // dims 16c .. 16c+15 land in 64-dim box c/4, 16-byte chunks 2(c%4) and 2(c%4)+1
-                    const int c0 = (c & 3) * 2;
-                    const uint32_t row = dst + (uint32_t)(c >> 2) * BOX_BYTES + (uint32_t)r * 128u;
-                    sts128(row + (uint32_t)((c0 ^ (r & 7)) << 4), o0);
-                    sts128(row + (uint32_t)(((c0 + 1) ^ (r & 7)) << 4), o1);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int idx = (kb + k) * 32 + (int)lane;
+                        const int r = cw * (KT / NCONV) + (idx >> 3), c = idx & 7;
+                        // rows past the length stay 0 (0x00 bytes widen to +0)
+                        const uint4 o0 = e4m3x8_to_f16x8(w[k].x, w[k].y);
+                        const uint4 o1 = e4m3x8_to_f16x8(w[k].z, w[k].w);
+                        // dims 16c .. 16c+15 land in 64-dim box c/4, 16-byte chunks 2(c%4), 2(c%4)+1
+                        const int c0 = (c & 3) * 2;
+                        const uint32_t row = dst + (uint32_t)(c >> 2) * BOX_BYTES + (uint32_t)r * 128u;
+                        sts128(row + (uint32_t)((c0 ^ (r & 7)) << 4), o0);
+                        sts128(row + (uint32_t)(((c0 + 1) ^ (r & 7)) << 4), o1);
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -483,7 +503,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ---------------- softmax + partial output (128 threads, thread = TMEM lane) ----------------
         const int tid = threadIdx.x;                       // key row of each tile; dim row of O^T
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        int n = 0;
+        int n = 0, pc = 0;   // units, P tiles handed over
         for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             const int h0 = u.kvh * G + u.hb * GT;
@@ -492,20 +512,27 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = mbar_wait(smem_u32(&sm.s_full), n & 1, abort_flag, 0x301);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            uint32_t sv[C::TPC][NH];
-#pragma unroll
-            for (int j = 0; j < C::TPC; ++j)
-                if (j < u.ntiles) tmem_ld<NH>(lane_base + C::COL_S + j * NH, sv[j]);
-            tmem_wait_ld();
-            // chunk maximum per head
+            // pass 1: chunk maximum per head, the chunk's S^T read from TMEM four tiles at a time
             float m[GT];
 #pragma unroll
-            for (int h = 0; h < GT; ++h) {
-                m[h] = -INFINITY;
+            for (int h = 0; h < GT; ++h) m[h] = -INFINITY;
+            for (int jg = 0; jg < u.ntiles; jg += 4) {
+                uint32_t sv[4][NH];
 #pragma unroll
-                for (int j = 0; j < C::TPC; ++j)
-                    if (j < u.ntiles && j * KT + tid < u.nkeys && window_keeps(u.key0 + j * KT + tid, u.seqlen, win))
-                        m[h] = fmaxf(m[h], __uint_as_float(sv[j][h]));
+                for (int jj = 0; jj < 4; ++jj)
+                    if (jg + jj < u.ntiles) tmem_ld<NH>(lane_base + C::COL_S + (jg + jj) * NH, sv[jj]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int key = (jg + jj) * KT + tid;
+                    if (jg + jj < u.ntiles && key < u.nkeys && window_keeps(u.key0 + key, u.seqlen, win)) {
+#pragma unroll
+                        for (int h = 0; h < GT; ++h) m[h] = fmaxf(m[h], __uint_as_float(sv[jj][h]));
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < GT; ++h) {
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], o));
                 if (lane == 0) sm.red_m[n & 1][warp][h] = m[h];
@@ -520,30 +547,36 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mc[h] = mm * su;             // finite: every unit holds at least one key
                 l[h] = 0.f;
             }
-            // p = 2^(s * scale * log2 e - m), written as P^T rows [key][8 heads] (bf16; f16 on the FP8 path)
-#pragma unroll
-            for (int j = 0; j < C::TPC; ++j) {
-                if (j >= u.ntiles) break;
-                const bool valid = j * KT + tid < u.nkeys && window_keeps(u.key0 + j * KT + tid, u.seqlen, win);
+            // pass 2: p = 2^(s * scale * log2 e - m) tile by tile, each tile's
+            // P^T rows [key][8 heads] (bf16; f16 on the FP8 path) handed to the
+            // MMA thread through one of two slots
+            for (int j = 0; j < u.ntiles; ++j, ++pc) {
+                uint32_t sv[NH];
+                tmem_ld<NH>(lane_base + C::COL_S + j * NH, sv);
+                tmem_wait_ld();
+                const int key = j * KT + tid;
+                const bool valid = key < u.nkeys && window_keeps(u.key0 + key, u.seqlen, win);
                 uint32_t pk[NH / 2];
 #pragma unroll
                 for (int h2 = 0; h2 < NH / 2; ++h2) {
                     float p0 = 0.f, p1 = 0.f;
-                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[j][2 * h2]), su, -mc[2 * h2]));
-                    if (2 * h2 + 1 < GT && valid)
-                        p1 = ex2(fmaf(__uint_as_float(sv[j][2 * h2 + 1]), su, -mc[2 * h2 + 1]));
+                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[2 * h2]), su, -mc[2 * h2]));
+                    if (2 * h2 + 1 < GT && valid) p1 = ex2(fmaf(__uint_as_float(sv[2 * h2 + 1]), su, -mc[2 * h2 + 1]));
                     if (2 * h2 < GT) l[2 * h2] += p0;
                     if (2 * h2 + 1 < GT) l[2 * h2 + 1] += p1;
                     pk[h2] = FP8 ? f2_to_h2_sat(p0, p1) : f2_to_bf2(p0, p1);
                 }
+                // the slot is free once the P.V of the tile two before has completed
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.p_empty[pc & 1]), ((pc >> 1) & 1) ^ 1,
+                                                       abort_flag, 0x303));
 #pragma unroll
                 for (int hb8 = 0; hb8 < NH / 8; ++hb8)
-                    sts128(smem_u32(sm.p[hb8]) + (uint32_t)(j * KT + tid) * 16u,
+                    sts128(smem_u32(sm.p[pc & 1][hb8]) + (uint32_t)tid * 16u,
                            make_uint4(pk[hb8 * 4 + 0], pk[hb8 * 4 + 1], pk[hb8 * 4 + 2], pk[hb8 * 4 + 3]));
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sm.p_full[pc & 1]));
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.p_full));
 #pragma unroll
             for (int h = 0; h < GT; ++h) {
 #pragma unroll

@@ -63,11 +63,11 @@ def test_decode_validation(lib):
     out = ctypes.c_size_t(0)
     assert lib.attn_decode_workspace_bytes(32, 32, 8, 128, 128, 32768, ctypes.byref(out)) == 0
     # partial outputs (fp32, 128 wide) + (m, l) per (b, h, chunk); G = 4 heads
-    # per unit: chunks of 1024 keys
-    assert out.value == 32 * 32 * 32 * 128 * 4 + 32 * 32 * 32 * 8
-    # G = 16: chunks of 512 keys
+    # per unit: chunks of 2048 keys
+    assert out.value == 32 * 32 * 16 * 128 * 4 + 32 * 32 * 16 * 8
+    # G = 16: chunks of 1024 keys
     assert lib.attn_decode_workspace_bytes(2, 32, 2, 128, 128, 4096, ctypes.byref(out)) == 0
-    assert out.value == 2 * 32 * 8 * 128 * 4 + 2 * 32 * 8 * 8
+    assert out.value == 2 * 32 * 4 * 128 * 4 + 2 * 32 * 4 * 8
     assert lib.attn_decode_workspace_bytes(32, 32, 8, 96, 96, 4096, ctypes.byref(out)) == -2
     args = dict(B=2, n_q=8, n_kv=2, d_qk=128, d_v=128, S_max=1024)
     need = ctypes.c_size_t(0)

@@ -74,9 +74,11 @@ def test_window_decode_skips_unread_chunks():
     kc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
     vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
     for b, L in enumerate(seq.tolist()):
-        lo = (L - W) // 1024 * 1024              # first key of the first window chunk
-        kc[b, :, 1024:lo] = float("nan")         # whole chunks between the sinks and the window
-        vc[b, :, 1024:lo] = float("nan")
+        # whole 2048-key spans between the sinks' chunk and the window's first
+        # chunk (chunks hold 2048 keys at this group size): never read
+        lo = (L - W) // 2048 * 2048
+        kc[b, :, 2048:lo] = float("nan")
+        vc[b, :, 2048:lo] = float("nan")
     o, lse = binding.attn_decode_window(q, kc, vc, seq.cuda(), W, ns, 0.1)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
     o_ref, lse_ref = oracle.sdpa_window(q[:, :, None, :], kc, vc, False, W, ns, 0.1, seqlens=seq.numpy())
