@@ -484,11 +484,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         // rows past the length stay 0 (0x00 bytes widen to +0)
                         const uint4 o0 = e4m3x8_to_f16x8(w[k].x, w[k].y);
                         const uint4 o1 = e4m3x8_to_f16x8(w[k].z, w[k].w);
-                        // dims 16c .. 16c+15 land in 64-dim box c/4, 16-byte chunks 2(c%4), 2(c%4)+1
-                        const int c0 = (c & 3) * 2;
-                        const uint32_t row = dst + (uint32_t)(c >> 2) * BOX_BYTES + (uint32_t)r * 128u;
-                        sts128(row + (uint32_t)((c0 ^ (r & 7)) << 4), o0);
-                        sts128(row + (uint32_t)(((c0 + 1) ^ (r & 7)) << 4), o1);
+                        // dims 16c .. 16c+15 land in 64-dim box c/4, 16-byte chunks 2(c%4), 2(c%4)+1.
+                        // The two boxes share banks, so lanes of box 1 store their odd chunk
+                        // first: each 8-lane phase of a store then hits 8 distinct bank groups.
+                        const int c0 = (c & 3) * 2, sw = c >> 2;
+                        const uint32_t row = dst + (uint32_t)sw * BOX_BYTES + (uint32_t)r * 128u;
+                        sts128(row + (uint32_t)(((c0 + sw) ^ (r & 7)) << 4), sw ? o1 : o0);
+                        sts128(row + (uint32_t)(((c0 + 1 - sw) ^ (r & 7)) << 4), sw ? o0 : o1);
                     }
                 }
                 fence_proxy_async_smem();
