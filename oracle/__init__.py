@@ -19,6 +19,9 @@ Functions:
   sdpa_varlen(q, k, v, cu_q, cu_k, causal, scale) -> (o, lse)  packed batch, one sdpa per sequence
   sdpa_window(q, k, v, causal, window, n_sink, scale, seqlens=None) -> (o, lse) sliding window + sinks
   dequant_e4m3(bytes, scale)                     -> fp64      FP8 (e4m3) cache values
+  rope_tables(n_pos, d, base)                    -> (cos, sin) rotary tables [n_pos, d/2]
+  rope(x, cos, sin, positions)                   -> fp64      rotary position embedding
+  sdpa_rope(q, k, v, causal, scale, cos, sin)    -> (o, lse)  sdpa on rotated queries and keys
 
 Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
 d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
@@ -69,6 +72,10 @@ def _declare(lib):
     lib.oracle_sdpa_window_fp64.argtypes = ([_f64p] * 5 + [_int] * 7 + [_i64] * 6 +
                                             [_i32p, _int, _int, _int, ctypes.c_double, _int])
     lib.oracle_sdpa_window_fp64.restype = _int
+    lib.oracle_rope_tables_fp64.argtypes = [_f64p, _f64p, _int, _int, ctypes.c_double]
+    lib.oracle_rope_tables_fp64.restype = _int
+    lib.oracle_rope_fp64.argtypes = [_f64p, _f64p, _i64, _int, _i32p, _f64p, _f64p, _int]
+    lib.oracle_rope_fp64.restype = _int
     return lib
 
 
@@ -305,3 +312,46 @@ def dequant_e4m3(raw, scale=None, head_axis=1):
         shape[head_axis] = -1
         val = val * sc.reshape(shape)
     return val
+
+
+def rope_tables(n_pos: int, d: int, base: float, lib=None):
+    """cos(m theta_j), sin(m theta_j) for m < n_pos, j < d/2, theta_j =
+    base^(-2j/d) ("Attention Engineering: From MHA to GQA, MLA &
+    FlashAttention", section 1: the geometric base frequencies and the
+    [positions, d/2] cache tables). fp64, shape [n_pos, d/2] each."""
+    lib = lib or load()
+    c = np.zeros((n_pos, d // 2))
+    s = np.zeros((n_pos, d // 2))
+    if lib.oracle_rope_tables_fp64(_ptr(c), _ptr(s), int(n_pos), int(d), float(base)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return c, s
+
+
+def rope(x, cos, sin, positions, lib=None):
+    """Rotate every plane (x_{2j}, x_{2j+1}) of the last axis by its
+    position's angle (section 1, real 2x2 block form). x [..., S, d];
+    positions [S] (or broadcastable to x.shape[:-1]) index the tables
+    cos/sin [n_pos, d/2] (fp32 values are widened exactly). Returns fp64."""
+    lib = lib or load()
+    x = _f64(x)
+    d = x.shape[-1]
+    pos = np.ascontiguousarray(np.broadcast_to(np.asarray(positions, dtype=np.int32), x.shape[:-1]))
+    c = _f64(cos)
+    s = _f64(sin)
+    out = np.zeros_like(x)
+    rc = lib.oracle_rope_fp64(_ptr(x), _ptr(out), int(np.prod(x.shape[:-1])), int(d), _ptr(pos, _i32p),
+                              _ptr(c), _ptr(s), int(c.shape[0]))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (position outside the tables?)")
+    return out
+
+
+def sdpa_rope(q, k, v, causal: bool, scale: float, cos, sin, nthreads=None, lib=None):
+    """sdpa on rotated queries and keys (section 2, GQA formulation with
+    RoPE(Q) RoPE(K)^T): key j at position j, query i at position
+    Skv - Sq + i (the bottom-right alignment of the causal mask); values are
+    not rotated."""
+    Sq, Skv = q.shape[2], k.shape[2]
+    qr = rope(q, cos, sin, np.arange(Skv - Sq, Skv), lib=lib)
+    kr = rope(k, cos, sin, np.arange(Skv), lib=lib)
+    return sdpa(qr, kr, v, causal, scale, nthreads=nthreads, lib=lib)

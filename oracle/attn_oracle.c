@@ -434,3 +434,52 @@ int oracle_online_fp64(const double *q, const double *k, const double *v,
     }
     return err ? -1 : 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Rotary position embedding ("Attention Engineering: From MHA to GQA, MLA &
+ * FlashAttention", section 1, Rotary Position Embeddings: the complex-plane
+ * derivation and its real 2x2 block form; section 2, the GQA formulation
+ * applies it to the queries and the keys before the scores).
+ *
+ * The head dimension d is split into d/2 planes (x_{2j}, x_{2j+1}). At
+ * position m, plane j turns by the angle m * theta_j with the geometric base
+ * frequencies theta_j = base^(-2j/d), j = 0 .. d/2-1.
+ * ------------------------------------------------------------------------ */
+
+/* cos_t / sin_t [n_pos][d/2]: cos(m theta_j), sin(m theta_j). */
+int oracle_rope_tables_fp64(double *cos_t, double *sin_t, int n_pos, int d, double base) {
+    if (n_pos < 0 || d <= 0 || d % 2 != 0 || !(base > 0.0)) return -1;
+    const int half = d / 2;
+    for (int j = 0; j < half; ++j) {
+        const double theta = pow(base, -2.0 * (double)j / (double)d);
+        for (int m = 0; m < n_pos; ++m) {
+            const double a = (double)m * theta;
+            cos_t[(int64_t)m * half + j] = cos(a);
+            sin_t[(int64_t)m * half + j] = sin(a);
+        }
+    }
+    return 0;
+}
+
+/* x, out [n_vec][d]; vector i sits at position pos[i] (a row of the tables).
+ * Each plane is multiplied by the rotation matrix [[c, -s], [s, c]]:
+ *   out_{2j}   = x_{2j} c - x_{2j+1} s
+ *   out_{2j+1} = x_{2j} s + x_{2j+1} c,   c = cos_t[pos][j], s = sin_t[pos][j]. */
+int oracle_rope_fp64(const double *x, double *out, int64_t n_vec, int d, const int32_t *pos,
+                     const double *cos_t, const double *sin_t, int n_pos) {
+    if (n_vec < 0 || d <= 0 || d % 2 != 0) return -1;
+    const int half = d / 2;
+    for (int64_t i = 0; i < n_vec; ++i) {
+        const int m = pos[i];
+        if (m < 0 || m >= n_pos) return -1;
+        const double *xi = x + i * d;
+        double *oi = out + i * d;
+        for (int j = 0; j < half; ++j) {
+            const double c = cos_t[(int64_t)m * half + j], s = sin_t[(int64_t)m * half + j];
+            const double xe = xi[2 * j], xo = xi[2 * j + 1];
+            oi[2 * j] = xe * c - xo * s;
+            oi[2 * j + 1] = xe * s + xo * c;
+        }
+    }
+    return 0;
+}

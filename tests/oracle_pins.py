@@ -359,6 +359,84 @@ def check_sliding_window(lib):
         assert np.max(np.abs(o[b:b + 1] - ref.numpy())) <= 1e-10
 
 
+
+# --------------------------------------------------------------------------
+# rotary position embedding
+# --------------------------------------------------------------------------
+def check_rope_tables(lib):
+    """Closed forms of the tables of "Attention Engineering: From MHA to GQA,
+    MLA & FlashAttention", section 1 (theta_j = base^(-2j/d)): plane 0 turns
+    by exactly m radians, plane d/4 of d = 128 at base 10^4 by m / 100, plane
+    d/2 - 1 by m * base^(-(d-2)/d); position 0 is the identity."""
+    n_pos, d, base = 300, 128, 10000.0
+    c, s = oracle.rope_tables(n_pos, d, base, lib=lib)
+    m = np.arange(n_pos, dtype=np.float64)
+    assert np.max(np.abs(c[:, 0] - np.cos(m))) <= 1e-14 and np.max(np.abs(s[:, 0] - np.sin(m))) <= 1e-14
+    assert np.max(np.abs(c[:, 32] - np.cos(m / 100.0))) <= 1e-14
+    assert np.max(np.abs(s[:, 32] - np.sin(m / 100.0))) <= 1e-14
+    last = m * 10000.0 ** (-126.0 / 128.0)
+    assert np.max(np.abs(s[:, 63] - np.sin(last))) <= 1e-14
+    assert np.all(c[0] == 1.0) and np.all(s[0] == 0.0)
+    c8, s8 = oracle.rope_tables(5, 8, 500000.0, lib=lib)        # Llama-3 base, tiny d
+    assert abs(s8[3, 1] - math.sin(3 * 500000.0 ** -0.25)) <= 1e-15
+
+
+def check_rope_complex_form(lib):
+    """The rotation equals multiplying z_j = x_{2j} + i x_{2j+1} by
+    exp(i m theta_j) (section 1, complex-plane derivation), here with numpy's
+    complex exponential and tables built outside the oracle."""
+    d, S = 16, 11
+    x = _rand((3, S, d), 70).numpy()
+    theta = 10000.0 ** (-np.arange(d // 2) * 2.0 / d)
+    pos = np.array([0, 1, 2, 5, 7, 8, 20, 33, 34, 40, 63], dtype=np.int32)
+    ang = np.arange(64)[:, None] * theta[None, :]
+    got = oracle.rope(x, np.cos(ang), np.sin(ang), pos, lib=lib)
+    z = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * pos[:, None] * theta[None, :])
+    ref = np.empty_like(x)
+    ref[..., 0::2], ref[..., 1::2] = z.real, z.imag
+    assert np.max(np.abs(got - ref)) <= 1e-13
+
+
+def check_rope_relative_position(lib):
+    """<RoPE(q, m), RoPE(k, n)> depends on m - n only (section 1, the
+    relative-distance invariance identity), and the rotation keeps each
+    plane's length."""
+    d = 32
+    c, s = oracle.rope_tables(400, d, 10000.0, lib=lib)
+    q, k = _rand((1, d), 71).numpy(), _rand((1, d), 72).numpy()
+    dots = []
+    for m, n in [(5, 2), (105, 102), (303, 300), (3, 0)]:
+        rq = oracle.rope(q, c, s, [m], lib=lib)
+        rk = oracle.rope(k, c, s, [n], lib=lib)
+        dots.append(float(rq @ rk.T))
+    assert max(dots) - min(dots) <= 1e-12 * max(1.0, abs(dots[0]))
+    assert abs(dots[0] - float(q @ k.T)) > 1e-3          # the rotation does act
+    rq = oracle.rope(q, c, s, [123], lib=lib)
+    assert np.max(np.abs(np.hypot(rq[:, 0::2], rq[:, 1::2]) - np.hypot(q[:, 0::2], q[:, 1::2]))) <= 1e-13
+
+
+def check_rope_attention(lib):
+    """sdpa_rope: a lone query (decode) sits at the last key's position, so it
+    equals the last row of the causal prefill; and the rotated scores of the
+    first causal row are those of q_0 and k_0 unrotated (position 0)."""
+    B, n_q, n_kv, S, d = 1, 4, 2, 9, 16
+    q, k, v = _rand((B, n_q, S, d), 73), _rand((B, n_kv, S, d), 74), _rand((B, n_kv, S, d), 75)
+    c, s = oracle.rope_tables(S, d, 10000.0, lib=lib)
+    o, lse = oracle.sdpa_rope(q, k, v, True, 0.25, c, s, lib=lib)
+    o1, lse1 = oracle.sdpa_rope(q[:, :, -1:], k, v, False, 0.25, c, s, lib=lib)
+    assert np.max(np.abs(o1[:, :, 0] - o[:, :, -1])) <= 1e-12
+    assert np.max(np.abs(lse1[:, :, 0] - lse[:, :, -1])) <= 1e-12
+    kv0 = k[0, :, 0].numpy()
+    ref = 0.25 * np.einsum("hd,hd->h", q[0, :, 0].numpy(), np.repeat(kv0, n_q // n_kv, axis=0))
+    assert np.max(np.abs(lse[0, :, 0] - ref)) <= 1e-12
+    # shifting every position by t leaves attention unchanged
+    c2, s2 = oracle.rope_tables(S + 7, d, 10000.0, lib=lib)
+    qs = oracle.rope(q, c2, s2, np.arange(7, 7 + S), lib=lib)
+    ks = oracle.rope(k, c2, s2, np.arange(7, 7 + S), lib=lib)
+    o2, _ = oracle.sdpa(qs, ks, v, True, 0.25, lib=lib)
+    assert np.max(np.abs(o2 - o)) <= 1e-12
+
+
 ALL_CHECKS = [
     check_worked_example, check_worked_example_first_tile, check_worked_example_online,
     check_first_causal_row, check_rows_sum_to_one, check_value_shift, check_key_shift,
@@ -367,4 +445,5 @@ ALL_CHECKS = [
     check_bottom_right_causal, check_decode, check_empty_visible_set, check_mla_alias,
     check_online_equals_two_pass, check_rows_mode,
     check_sliding_window,
+    check_rope_tables, check_rope_complex_form, check_rope_relative_position, check_rope_attention,
 ]

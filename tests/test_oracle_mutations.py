@@ -37,6 +37,12 @@ MUTATIONS = [
      "return (end - 1 - j < p->window);"),
     ("window_anchored_at_row_not_position", "return (end - 1 - j < p->window) || (j < p->n_sink);",
      "return (end - 1 - j - (p->Skv - p->Sq) < p->window) || (j < p->n_sink);"),
+    ("rope_sin_sign", "oi[2 * j] = xe * c - xo * s;", "oi[2 * j] = xe * c + xo * s;"),
+    ("rope_rotate_half", "const double xe = xi[2 * j], xo = xi[2 * j + 1];",
+     "const double xe = xi[j], xo = xi[j + half];"),
+    ("rope_theta_exponent", "pow(base, -2.0 * (double)j / (double)d)", "pow(base, -(double)j / (double)d)"),
+    ("rope_position_shift", "const int m = pos[i];", "const int m = pos[i] > 0 ? pos[i] - 1 : 0;"),
+    ("rope_cos_sin_swapped", "cos_t[(int64_t)m * half + j] = cos(a);", "cos_t[(int64_t)m * half + j] = sin(a);"),
 ]
 
 
