@@ -298,6 +298,71 @@ int attn_decode_noalloc(const void *q, const void *kcache, const void *vcache, c
                         int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
                         float scale, attn_stream_t stream);
 
+/*
+ * Rotary position embedding (RoPE).
+ * Source: "Attention Engineering: From MHA to GQA, MLA & FlashAttention",
+ * section 1 (Rotary Position Embeddings: the head dimension is split into
+ * d/2 planes (x_{2j}, x_{2j+1}); at position m plane j is turned by the
+ * angle m * theta_j, theta_j = base^(-2j/d), i.e. multiplied by the 2x2
+ * rotation [[cos, -sin], [sin, cos]]; the angles are kept in cos/sin tables
+ * of shape [positions, d/2]) and section 2 (the GQA formulation applies it
+ * to the queries and the keys before the scores; values are not rotated).
+ *
+ * Tables: cos, sin [n_pos, d/2] fp32 on the device, 16-byte aligned, row m
+ * holding cos(m theta_j) and sin(m theta_j).
+ */
+
+/*
+ * attn_rope_tables -- fill cos/sin [n_pos, d/2] for the given base (10000 in
+ * the original RoPE, 500000 in Llama-3). Angles in fp64, rounded once to
+ * fp32. d even, n_pos >= 0, base finite and > 0. Asynchronous on `stream`.
+ */
+int attn_rope_tables(float *cos, float *sin, int n_pos, int d, double base, attn_stream_t stream);
+
+/*
+ * attn_rope_apply -- y = RoPE(x): x, y [B, H, S, d] bf16 contiguous (y may be
+ * x: rotated in place); row (b, h, s) sits at position pos0 + s, and
+ * pos0 + S <= n_pos. Computed in fp32, rounded once to bf16 (nearest even).
+ * This is how keys enter a KV cache in rotated form. d a multiple of 8.
+ */
+int attn_rope_apply(const void *x, void *y, int B, int H, int S, int d, int pos0,
+                    const float *cos, const float *sin, int n_pos, attn_stream_t stream);
+
+/*
+ * attn_fwd_rope -- attn_fwd on rotated queries and keys:
+ *   O = softmax(scale * RoPE(Q) RoPE(K)^T + mask) V
+ * with key j at position j and query row i at position i + (Skv - Sq) (the
+ * alignment of the causal mask). q, k, v, o, lse, causal, scale as attn_fwd
+ * (q and k are given unrotated). The keys are rotated once into k_rot
+ * ([B, n_kv, Skv, d_qk] bf16, caller-owned, written; it may be k itself,
+ * which is then overwritten): each key tile is read by every query tile of
+ * its group, so it is rotated by one bandwidth-bound pass rather than in
+ * each of them. The queries are rotated inside the attention kernel, in
+ * shared memory, before their first score MMA. Rotated values are rounded
+ * to bf16 before the MMAs (the precision of the tensor-core operands).
+ * Supported: as attn_fwd, plus Sq <= Skv <= n_pos. Two launches on `stream`.
+ */
+int attn_fwd_rope(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int Sq, int Skv, int n_q, int n_kv, int d_qk, int d_v,
+                  int causal, float scale, const float *cos, const float *sin, int n_pos,
+                  void *k_rot, attn_stream_t stream);
+
+/*
+ * attn_decode_rope -- attn_decode (head dim 128) with the query rotated at
+ * position seqlens[b] - 1 (the new token is the last one in the cache),
+ * inside the kernel before its score MMAs. The cache holds keys that were
+ * rotated when they were written (attn_rope_apply), as the KV cache of a
+ * RoPE model does. Arguments as attn_decode plus the tables; a length above
+ * n_pos uses the last table row and raises ATTN_ERR_DEVICE_RANGE in
+ * attn_device_status. The MLA shape is not supported here.
+ */
+int attn_decode_rope(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens,
+                     void *o, float *lse, int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
+                     int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                     int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
+                     const float *cos, const float *sin, int n_pos, float scale,
+                     void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
 /* Human-readable text of a status code (static storage). */
 const char *attn_status_string(int status);
 

@@ -72,6 +72,15 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_paged.argtypes = ([_vp] * 7 + [_i] * 8 + [_i64] * 6 +
                                         [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode_paged.restype = _i
+        L.attn_rope_tables.argtypes = [_vp, _vp, _i, _i, ctypes.c_double, _vp]
+        L.attn_rope_tables.restype = _i
+        L.attn_rope_apply.argtypes = [_vp, _vp] + [_i] * 5 + [_vp, _vp, _i, _vp]
+        L.attn_rope_apply.restype = _i
+        L.attn_fwd_rope.argtypes = [_vp] * 5 + [_i] * 8 + [ctypes.c_float, _vp, _vp, _i, _vp, _vp]
+        L.attn_fwd_rope.restype = _i
+        L.attn_decode_rope.argtypes = ([_vp] * 6 + [_i] * 6 + [_i64] * 6 + [_vp, _vp, _i] +
+                                       [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_decode_rope.restype = _i
         L.attn_status_string.argtypes = [_i]
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_device_status.argtypes = [_vp]
@@ -321,3 +330,87 @@ def selftest_ex2(x, stream=None):
     _check(lib().attn_selftest_ex2(_ptr(x), _ptr(yp), _ptr(ys), x.numel(), ctypes.c_void_p(_stream(stream))),
            "attn_selftest_ex2")
     return yp, ys
+
+
+def _tables(cos, sin):
+    for t in (cos, sin):
+        if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and t.dim() == 2):
+            raise ValueError("rotary tables must be contiguous fp32 CUDA tensors [n_pos, d/2]")
+    if cos.shape != sin.shape:
+        raise ValueError("cos and sin tables differ in shape")
+    return cos.shape[0], cos.shape[1]
+
+
+def rope_tables(n_pos: int, d: int, base: float, device="cuda", stream=None):
+    """cos, sin [n_pos, d/2] fp32 on the device (attn_rope_tables)."""
+    cos = torch.empty((n_pos, d // 2), dtype=torch.float32, device=device)
+    sin = torch.empty_like(cos)
+    _check(lib().attn_rope_tables(_ptr(cos), _ptr(sin), int(n_pos), int(d), float(base),
+                                  ctypes.c_void_p(_stream(stream))), "attn_rope_tables")
+    return cos, sin
+
+
+def rope_apply(x, cos, sin, pos0: int = 0, out=None, stream=None):
+    """RoPE of x [B, H, S, d] bf16 (row s at position pos0 + s); returns out
+    (a new tensor unless given; it may be x)."""
+    if not (x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 4):
+        raise ValueError("x must be a contiguous bf16 CUDA tensor [B, H, S, d]")
+    n_pos, _ = _tables(cos, sin)
+    if out is None:
+        out = torch.empty_like(x)
+    B, H, S, d = x.shape
+    _check(lib().attn_rope_apply(_ptr(x), _ptr(out), B, H, S, d, int(pos0), _ptr(cos), _ptr(sin), n_pos,
+                                 ctypes.c_void_p(_stream(stream))), "attn_rope_apply")
+    return out
+
+
+def attn_fwd_rope(q, k, v, causal: bool, scale: float, cos, sin, k_rot=None, o=None, lse=None, stream=None,
+                  want_lse=True):
+    """attn_fwd on RoPE-rotated q and k (given unrotated); the rotated keys
+    are written to k_rot (allocated unless given; it may be k). Returns
+    (o, lse, k_rot)."""
+    B, n_q, Sq, d_qk = q.shape
+    _, n_kv, Skv, _ = k.shape
+    d_v = v.shape[3]
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    n_pos, _ = _tables(cos, sin)
+    if k_rot is None:
+        k_rot = torch.empty_like(k)
+    if o is None:
+        o = torch.empty((B, n_q, Sq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Sq), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, n_q, n_kv, d_qk, d_v,
+                             int(bool(causal)), float(scale), _ptr(cos), _ptr(sin), n_pos, _ptr(k_rot),
+                             ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_fwd_rope")
+    return o, lse, k_rot
+
+
+def attn_decode_rope(q, kcache, vcache, seqlens, scale: float, cos, sin, o=None, lse=None, workspace=None,
+                     stream=None, want_lse=True):
+    """attn_decode with q rotated at position seqlens[b] - 1 (the cache holds
+    rotated keys). Arguments as attn_decode plus the tables (head dim 128)."""
+    B, n_q, d_qk = q.shape
+    _, n_kv, S_max, _ = kcache.shape
+    d_v = vcache.shape[3]
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    if seqlens.dtype != torch.int32 or not seqlens.is_cuda:
+        raise ValueError("seqlens must be an int32 CUDA tensor")
+    n_pos, _ = _tables(cos, sin)
+    ks, vs = _elem_strides(kcache), _elem_strides(vcache)
+    if o is None:
+        o = torch.empty((B, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, n_q, n_kv, d_qk, d_v, S_max)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().attn_decode_rope(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse),
+                                B, n_q, n_kv, d_qk, d_v, S_max, *ks, *vs, _ptr(cos), _ptr(sin), n_pos,
+                                float(scale), _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_decode_rope")
+    return o, lse

@@ -111,8 +111,9 @@ struct VarlenArgs {
 template <int D>
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,
                    int n_q, int n_kv, int causal, float scale, cudaStream_t stream, const VarlenArgs *vl = nullptr,
-                   int window = 0, int n_sink = 0) {
+                   int window = 0, int n_sink = 0, const attn::rope::Tables *rope = nullptr) {
     using attn::pf::kDense;
+    using attn::pf::kRope;
     using attn::pf::kVarlen;
     using attn::pf::kWindow;
     using C = attn::pf::Cfg<D>;
@@ -129,6 +130,7 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     p.lse = lse;
     p.window = window;
     p.n_sink = n_sink;
+    if (rope) p.rope = *rope;
     const int Sq_plan = vl ? vl->max_q : Sq;   // position blocks cover the longest sequence
     if (G >= 2) {
         p.Ht = G / 2;
@@ -179,21 +181,23 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     const size_t smem = attn::pf::smem_bytes<D>();
     static uint64_t attr_done = 0;  // per template instance, one bit per device
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kDense>, smem, attr_done)) return ATTN_ERR_CUDA;
-    static uint64_t attr_done_v = 0, attr_done_w = 0;
+    static uint64_t attr_done_v = 0, attr_done_w = 0, attr_done_r = 0;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kVarlen>, smem, attr_done_v)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kWindow>, smem, attr_done_w)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kRope>, smem, attr_done_r)) return ATTN_ERR_CUDA;
     // The kernel rebalances registers between warpgroups (setmaxnreg); that is
     // only safe if it was built with exactly the register count the split
     // assumes, otherwise the increase could never be granted.
     static int regs_checked = 0;
     if (regs_checked == 0) {
         cudaFuncAttributes fa;
-        cudaFuncAttributes fv, fw;
+        cudaFuncAttributes fv, fw, fr;
         if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D, kDense>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fv, attn::pf::prefill_kernel<D, kVarlen>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fw, attn::pf::prefill_kernel<D, kWindow>) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&fr, attn::pf::prefill_kernel<D, kRope>) != cudaSuccess) return ATTN_ERR_CUDA;
         regs_checked = (fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs &&
-                        fw.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
+                        fw.numRegs == attn::pf::kLaunchRegs && fr.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
     }
     if (regs_checked < 0) return ATTN_ERR_UNSUPPORTED;
     if (vl) {
@@ -207,7 +211,10 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         const long long grid = (long long)p.n_pb * B * n_kv;
         if (grid <= 0) return ATTN_OK;
         if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-        if (window > 0)
+        if (rope)
+            attn::pf::prefill_kernel<D, kRope><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
+                                                                                                     p);
+        else if (window > 0)
             attn::pf::prefill_kernel<D, kWindow><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
                                                                                                        p);
         else
@@ -245,6 +252,7 @@ struct CacheView {
     int page_size;
     attn::dec::Window win;             // sliding window (window 0: none)
     attn::dec::Fp8Scales fs;           // FP8 cache: per-KV-head scales
+    attn::rope::Tables rt{nullptr, nullptr, 0};   // rotary tables for the query (cos null: none)
 };
 
 template <int GT, bool PAGED, bool FP8 = false>
@@ -309,7 +317,7 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
     const int grid = (int)(max_units < resident ? max_units : resident);
     decode_split_kernel<GT, PAGED, FP8><<<grid, threads, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q,
                                                                          n_kv, G, n_hb, S_max, n_splits, scale_log2,
-                                                                         cv.pt, cv.win, cv.fs);
+                                                                         cv.pt, cv.win, cv.fs, cv.rt);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
         ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH, cv.win);
@@ -494,7 +502,8 @@ namespace {
 int decode_entry(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o, float *lse,
                  int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b, int64_t k_stride_h,
                  int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale,
-                 void *workspace, size_t workspace_bytes, attn_stream_t stream, attn::dec::Window win) {
+                 void *workspace, size_t workspace_bytes, attn_stream_t stream, attn::dec::Window win,
+                 const attn::rope::Tables *rt = nullptr) {
     if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
     if (B == 0) return ATTN_OK;
@@ -519,9 +528,10 @@ int decode_entry(const void *q, const void *kcache, const void *vcache, const in
         cv.ks[0] = k_stride_b, cv.ks[1] = k_stride_h, cv.ks[2] = k_stride_s;
         cv.vs[0] = v_stride_b, cv.vs[1] = v_stride_h, cv.vs[2] = v_stride_s;
         cv.win = win;
+        if (rt) cv.rt = *rt;
         return dispatch_decode_gqa<false>(G, q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, workspace, s);
     }
-    if (win.window > 0) return ATTN_ERR_UNSUPPORTED;   // the MLA kernel has no window
+    if (win.window > 0 || rt) return ATTN_ERR_UNSUPPORTED;   // the MLA kernel has no window, no rotation
     if (d_qk == 576 && d_v == 512 && n_kv == 1) {
         // the value rows must be the first 512 columns of the key rows
         if (vcache != kcache || v_stride_b != k_stride_b || v_stride_s != k_stride_s) return ATTN_ERR_UNSUPPORTED;
@@ -557,6 +567,97 @@ int attn_decode_window(const void *q, const void *kcache, const void *vcache, co
     return decode_entry(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, d_qk, d_v, S_max, k_stride_b, k_stride_h,
                         k_stride_s, v_stride_b, v_stride_h, v_stride_s, scale, workspace, workspace_bytes, stream,
                         attn::dec::Window{window, n_sink});
+}
+
+// ---- rotary position embedding ----
+int attn_rope_tables(float *cos_t, float *sin_t, int n_pos, int d, double base, attn_stream_t stream) {
+    if (n_pos < 0 || d < 2 || d % 2 != 0 || !std::isfinite(base) || !(base > 0.0)) return ATTN_ERR_INVALID_ARG;
+    if (n_pos == 0) return ATTN_OK;
+    if (!cos_t || !sin_t) return ATTN_ERR_INVALID_ARG;
+    const long long n = (long long)n_pos * (d / 2);
+    const int blocks = (int)std::min<long long>((n + 255) / 256, 4LL * 148);
+    attn::rope::rope_tables_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cos_t, sin_t, n_pos,
+                                                                                             d / 2, base);
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+bool rope_tables_ok(const float *cos_t, const float *sin_t, int n_pos) {
+    return cos_t && sin_t && n_pos >= 1;
+}
+// x, y [BH][S][d]: grid x over the 16-byte words of S rows, y over BH.
+int launch_rope_apply(const void *x, void *y, long long BH, int S, int d, int pos0, const attn::rope::Tables &t,
+                      cudaStream_t stream) {
+    const long long words = (long long)S * (d / 8);
+    if (BH == 0 || words == 0) return ATTN_OK;
+    if (words > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const unsigned gx = (unsigned)((words + 255) / 256);
+    const unsigned gy = (unsigned)std::min<long long>((BH + attn::rope::ROPE_BH - 1) / attn::rope::ROPE_BH, 65535);
+    attn::rope::rope_apply_kernel<<<dim3(gx, gy), 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16 *>(x),
+                                                                    reinterpret_cast<__nv_bfloat16 *>(y), BH, S, d,
+                                                                    pos0, t);
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+int attn_rope_apply(const void *x, void *y, int B, int H, int S, int d, int pos0, const float *cos_t,
+                    const float *sin_t, int n_pos, attn_stream_t stream) {
+    if (B < 0 || H < 0 || S < 0 || d < 8 || d % 8 != 0 || pos0 < 0) return ATTN_ERR_INVALID_ARG;
+    if ((long long)B * H * S == 0) return ATTN_OK;
+    if (!x || !y || !rope_tables_ok(cos_t, sin_t, n_pos)) return ATTN_ERR_INVALID_ARG;
+    if ((long long)pos0 + S > n_pos) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(cos_t) || !aligned16(sin_t)) return ATTN_ERR_MISALIGNED;
+    return launch_rope_apply(x, y, (long long)B * H, S, d, pos0, attn::rope::Tables{cos_t, sin_t, n_pos},
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_rope(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv, int n_q,
+                  int n_kv, int d_qk, int d_v, int causal, float scale, const float *cos_t, const float *sin_t,
+                  int n_pos, void *k_rot, attn_stream_t stream) {
+    if (B < 0 || Sq < 0 || Skv < 1 || n_q < 1 || n_kv < 1 || d_qk < 1 || d_v < 1) return ATTN_ERR_INVALID_ARG;
+    if (n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || Sq == 0) return ATTN_OK;
+    if (!q || !k || !v || !o || !k_rot || !rope_tables_ok(cos_t, sin_t, n_pos)) return ATTN_ERR_INVALID_ARG;
+    if (n_pos < Skv) return ATTN_ERR_INVALID_ARG;
+    if (d_qk != d_v || (d_qk != 32 && d_qk != 64 && d_qk != 128)) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G) || G > 256) return ATTN_ERR_UNSUPPORTED;
+    if (Sq > Skv) return ATTN_ERR_UNSUPPORTED;   // queries sit at the last Sq key positions
+    if ((long long)B * n_q > 0x7fffffffLL || (long long)B * n_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_rot) ||
+        !aligned16(cos_t) || !aligned16(sin_t))
+        return ATTN_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const attn::rope::Tables t{cos_t, sin_t, n_pos};
+    // keys: rotated once, into k_rot (many query tiles read each key tile)
+    int rc = launch_rope_apply(k, k_rot, (long long)B * n_kv, Skv, d_qk, 0, t, s);
+    if (rc != ATTN_OK) return rc;
+    // queries: rotated in shared memory by the attention kernel
+    switch (d_qk) {
+        case 32: return launch_prefill<32>(q, k_rot, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s, nullptr, 0, 0, &t);
+        case 64: return launch_prefill<64>(q, k_rot, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s, nullptr, 0, 0, &t);
+        default: return launch_prefill<128>(q, k_rot, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s, nullptr, 0, 0, &t);
+    }
+}
+
+int attn_decode_rope(const void *q, const void *kcache, const void *vcache, const int32_t *seqlens, void *o,
+                     float *lse, int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, int64_t k_stride_b,
+                     int64_t k_stride_h, int64_t k_stride_s, int64_t v_stride_b, int64_t v_stride_h,
+                     int64_t v_stride_s, const float *cos_t, const float *sin_t, int n_pos, float scale,
+                     void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+    if (!rope_tables_ok(cos_t, sin_t, n_pos)) return ATTN_ERR_INVALID_ARG;
+    if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(cos_t) || !aligned16(sin_t)) return ATTN_ERR_MISALIGNED;
+    const attn::rope::Tables t{cos_t, sin_t, n_pos};
+    return decode_entry(q, kcache, vcache, seqlens, o, lse, B, n_q, n_kv, d_qk, d_v, S_max, k_stride_b, k_stride_h,
+                        k_stride_s, v_stride_b, v_stride_h, v_stride_s, scale, workspace, workspace_bytes, stream,
+                        attn::dec::Window{0, 0}, &t);
 }
 
 int attn_decode_fp8_workspace_bytes(int B, int n_q, int n_kv, int S_max, size_t *bytes) {

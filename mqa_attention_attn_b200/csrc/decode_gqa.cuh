@@ -27,6 +27,7 @@
 // the softmax.
 #pragma once
 
+#include "rope.cuh"
 #include "sm100.cuh"
 
 #ifndef ATTN_DEC_STAGES
@@ -222,7 +223,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
                     float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
                     int S_max, int n_splits, float scale_log2, const PageTable pt, const Window win,
-                    const Fp8Scales fs) {
+                    const Fp8Scales fs, const rope::Tables rt) {
     using C = Cfg<GT, FP8>;
     constexpr int NH = C::NH;
     extern __shared__ uint8_t smem_raw[];
@@ -360,6 +361,27 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             if (!mbar_wait(smem_u32(FP8 ? &sm.q_conv : &sm.q_full), n & 1, abort_flag, 0x201)) break;
+            if (!FP8 && rt.cos != nullptr) {
+                // rotary embedding of the unit's query rows (the new token sits at
+                // position seqlen - 1; the cached keys are stored rotated): NH rows
+                // x 16 chunks of 8 dims, spread over the warp
+                int pos = u.seqlen - 1;
+                if (pos >= rt.n_pos) {
+                    if (lane == 0) atomicOr(&g_status, kStatusRange);
+                    pos = rt.n_pos - 1;
+                }
+                const float *cr = rt.cos + (size_t)pos * (D / 2), *sr = rt.sin + (size_t)pos * (D / 2);
+                for (int i = (int)lane; i < NH * 16; i += 32) {
+                    const int row = i >> 4, bx = (i >> 3) & 1, c = i & 7;
+                    const uint32_t a = smem_u32(sm.q[bx]) + swz<3>((uint32_t)(row * 128 + c * 16));
+                    const int j0 = bx * 32 + c * 4;
+                    const float4 cc = __ldg(reinterpret_cast<const float4 *>(cr + j0));
+                    const float4 ss = __ldg(reinterpret_cast<const float4 *>(sr + j0));
+                    sts128(a, rope::rope_chunk(lds128(a), cc, ss));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
             bool ok = true;
             for (int j = 0; j < u.ntiles; ++j) {
                 const int g = t + j, s = g % NSTAGE;

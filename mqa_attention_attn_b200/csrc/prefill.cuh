@@ -32,12 +32,18 @@
 // the tensor core runs the other tile's MMAs. Epilogue: O / l -> bf16 ->
 // swizzled shared memory -> TMA store; LSE = (m + log2 l) * ln 2.
 //
+// With rotary position embedding (the ROPE kernel), each softmax warpgroup
+// first rotates its Q tile in shared memory, one row per thread (position
+// Skv - Sq + i of query i), before the first S MMA of that tile; the keys
+// arrive already rotated.
+//
 // Roles (384 threads): warps 0 and 2 TMA producers (Q and K; V), warp 1 MMA
 // issuer and TMEM owner, warps 4-7 and 8-11 the softmax / epilogue
 // warpgroups of tiles 0 and 1 (warp w reads TMEM lanes 32*(w%4) .. +31, so
 // each warpgroup covers 128 rows).
 #pragma once
 
+#include "rope.cuh"
 #include "sm100.cuh"
 
 namespace attn {
@@ -103,6 +109,7 @@ struct Smem {
     uint64_t p_full[2][kPChunks];  // one per hand-off chunk of P
     uint64_t o_done[2];
     uint64_t mma_done;
+    uint64_t q_rot[2];             // ROPE: Q tile t rotated in place
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -133,6 +140,8 @@ struct Params {
     // Sliding window (the WINDOW kernel, causal): a query at position p sees
     // key j iff j <= p and (p - j < window or j < n_sink).
     int window, n_sink;
+    // Rotary tables (the ROPE kernel): cos/sin [n_pos][D/2], n_pos >= Skv.
+    rope::Tables rope;
     __nv_bfloat16 *o;      // varlen: rows of a tile that ends past its sequence are stored directly
 };
 
@@ -150,8 +159,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // MODE: kDense (BHSD batch), kVarlen (packed batch), kWindow (BHSD, causal
-// sliding window with sink keys).
-enum : int { kDense = 0, kVarlen = 1, kWindow = 2 };
+// sliding window with sink keys), kRope (BHSD batch, queries rotated here).
+enum : int { kDense = 0, kVarlen = 1, kWindow = 2, kRope = 3 };
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -161,6 +170,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     using C = Cfg<D>;
     constexpr bool VARLEN = MODE == kVarlen;
     constexpr bool WINDOW = MODE == kWindow;
+    constexpr bool ROPE = MODE == kRope;
     extern __shared__ uint8_t smem_raw[];
     Smem<D> &sm = *reinterpret_cast<Smem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -237,6 +247,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(smem_u32(&sm.o_done[t]), 1);
         }
         mbar_init(smem_u32(&sm.mma_done), 1);
+        for (int t = 0; t < 2; ++t) mbar_init(smem_u32(&sm.q_rot[t]), 128);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -374,8 +385,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ok = mbar_wait(smem_u32(&sm.k_full[0]), 0, abort_flag, 0x22);
                 if (ok) {
                     tc_fence_after();
-                    for (int t = 0; t < 2; ++t)
-                        if (nt[t] > 0) issue_s(t, 0);
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (nt[t] == 0) continue;
+                        // ROPE: this tile's rows have been rotated in place
+                        if (ROPE) ok = mbar_wait(smem_u32(&sm.q_rot[t]), 0, abort_flag, 0x27);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(t, 0);
+                    }
                 }
             }
             for (int j = 0; ok && j < nmax; ++j) {
@@ -412,6 +429,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int pl = VARLEN ? r / p.Ht : r % p.Pt;
             const int pos = p0[t] + pl;
             const int head = h0[t] + hl;
+            if constexpr (ROPE) {
+                // rotate the Q tile in place, each row at its absolute position
+                // (row's position in the tile: row % Pt, the tile being head-major);
+                // the angles are fetched while the tile is still in flight
+                rope::RopeTile<D, C::ROWB> rt;
+                const int Pt = p.Pt, pbase = p0[t] + (Skv - Sq), last = Skv - 1;
+                rt.fetch(p.rope, r, [&](int row) { return min(pbase + row % Pt, last); });
+                if (warp_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x36)) {
+                    const int pend = Sq - p0[t];   // rows at positions >= Sq hold no query
+                    rt.apply(smem_u32(sm.q[t]), C::QBOX, r, [&](int row) { return row % Pt < pend; });
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(smem_u32(&sm.q_rot[t]));
+            }
             int lim = p.causal ? pos + (Skv - Sq) : Skv - 1;   // last visible key (< 0: none)
             lim = min(lim, Skv - 1);
             const uint32_t trow = tmem + ((quad * 32u) << 16);

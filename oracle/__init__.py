@@ -21,7 +21,8 @@ Functions:
   dequant_e4m3(bytes, scale)                     -> fp64      FP8 (e4m3) cache values
   rope_tables(n_pos, d, base)                    -> (cos, sin) rotary tables [n_pos, d/2]
   rope(x, cos, sin, positions)                   -> fp64      rotary position embedding
-  sdpa_rope(q, k, v, causal, scale, cos, sin)    -> (o, lse)  sdpa on rotated queries and keys
+  sdpa_rope(q, k, v, causal, scale, cos, sin)    -> (o, lse)  sdpa on rotated (bf16) queries and keys
+  round_bf16(x)                                  -> fp64      nearest bf16 value, ties to even
 
 Layouts: q [B, n_q, Sq, d_qk]; k [B, n_kv, Skv, d_k_row]; v [B, n_kv, Skv,
 d_v_row] (any strides; the last dimension is read up to d_qk / d_v, so a
@@ -346,12 +347,25 @@ def rope(x, cos, sin, positions, lib=None):
     return out
 
 
-def sdpa_rope(q, k, v, causal: bool, scale: float, cos, sin, nthreads=None, lib=None):
+def round_bf16(x):
+    """Round fp64 values to the nearest bf16 value (8 significant bits, ties
+    to even), returned as fp64. Normal range only (|x| >= 2^-126 or 0)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                  # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def sdpa_rope(q, k, v, causal: bool, scale: float, cos, sin, operand_bf16: bool = True, nthreads=None,
+              lib=None):
     """sdpa on rotated queries and keys (section 2, GQA formulation with
     RoPE(Q) RoPE(K)^T): key j at position j, query i at position
     Skv - Sq + i (the bottom-right alignment of the causal mask); values are
-    not rotated."""
+    not rotated. With operand_bf16 the rotated queries and keys are rounded
+    to bf16 first: they are activations of a bf16 model, the operand type of
+    the score contraction."""
     Sq, Skv = q.shape[2], k.shape[2]
     qr = rope(q, cos, sin, np.arange(Skv - Sq, Skv), lib=lib)
     kr = rope(k, cos, sin, np.arange(Skv), lib=lib)
+    if operand_bf16:
+        qr, kr = round_bf16(qr), round_bf16(kr)
     return sdpa(qr, kr, v, causal, scale, nthreads=nthreads, lib=lib)

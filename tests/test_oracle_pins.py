@@ -1,5 +1,6 @@
 """The fp64 oracle against its pins (CPU only)."""
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -121,3 +122,15 @@ def test_dequant_e4m3_matches_an_independent_decoder():
     # per-head scale along axis 1
     x = np.full((2, 3, 4), 0x38, np.uint8)
     assert np.array_equal(oracle.dequant_e4m3(x, [1.0, 0.5, 2.0])[0, :, 0], [1.0, 0.5, 2.0])
+
+
+def test_round_bf16_matches_torch():
+    """The oracle's bf16 rounding against torch's fp32 -> bf16 conversion
+    (round to nearest even) on fp32 values, ties and near-ties included."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(200000, generator=g, dtype=torch.float32) * torch.exp2(torch.randint(-20, 20, (200000,)).float())
+    ties = torch.tensor([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 3 * 2 ** -9 + 2 ** -30, 255.5, 256.5],
+                        dtype=torch.float32)
+    x = torch.cat([x, ties])
+    ref = x.to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.round_bf16(x.double().numpy()), ref)
