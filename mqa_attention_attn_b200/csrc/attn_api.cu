@@ -211,10 +211,23 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         const long long grid = (long long)p.n_pb * B * n_kv;
         if (grid <= 0) return ATTN_OK;
         if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-        if (rope)
-            attn::pf::prefill_kernel<D, kRope><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
-                                                                                                     p);
-        else if (window > 0)
+        if (rope) {
+            // launched as a programmatic dependent of the key rotation: the
+            // prologue (barriers, TMEM, Q load and rotation) overlaps it and
+            // only the K producer waits for it
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)grid);
+            cfg.blockDim = dim3(attn::pf::THREADS);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, attn::pf::prefill_kernel<D, kRope>, tq, tk, tv, to, p) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+        } else if (window > 0)
             attn::pf::prefill_kernel<D, kWindow><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
                                                                                                        p);
         else

@@ -289,7 +289,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
                                     b * p.n_q + h0[t]);
             }
-            // K tiles (V tiles are loaded by warp 2)
+            // K tiles (V tiles are loaded by warp 2). ROPE: the rotated keys come
+            // from the grid launched just before this one
+            if (ROPE) griddep_wait();
             int issued = 0;
             for (int j = 0; j < nmax; ++j) {
                 const int s = j % KSTAGE;
@@ -434,11 +436,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // (row's position in the tile: row % Pt, the tile being head-major);
                 // the angles are fetched while the tile is still in flight
                 rope::RopeTile<D, C::ROWB> rt;
-                const int Pt = p.Pt, pbase = p0[t] + (Skv - Sq), last = Skv - 1;
-                rt.fetch(p.rope, r, [&](int row) { return min(pbase + row % Pt, last); });
+                const int pmask = p.Pt - 1;                 // Pt is a power of two
+                const int pbase = p0[t] + (Skv - Sq), last = Skv - 1;
+                rt.fetch(p.rope, r, [&](int row) { return min(pbase + (row & pmask), last); });
                 if (warp_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x36)) {
                     const int pend = Sq - p0[t];   // rows at positions >= Sq hold no query
-                    rt.apply(smem_u32(sm.q[t]), C::QBOX, r, [&](int row) { return row % Pt < pend; });
+                    rt.apply(smem_u32(sm.q[t]), C::QBOX, r, [&](int row) { return (row & pmask) < pend; });
                     fence_proxy_async_smem();
                 }
                 mbar_arrive(smem_u32(&sm.q_rot[t]));

@@ -102,6 +102,7 @@ __global__ void rope_tables_kernel(float *cos_t, float *sin_t, int n_pos, int ha
 constexpr int ROPE_BH = 4;
 __global__ void rope_apply_kernel(const __nv_bfloat16 *x, __nv_bfloat16 *y, long long BH, int S, int d, int pos0,
                                   Tables t) {
+    griddep_launch_dependents();                 // the attention kernel may start its prologue
     const int cpr = d / 8;                       // words per row
     const int w = blockIdx.x * blockDim.x + threadIdx.x;
     if (w >= S * cpr) return;

@@ -99,6 +99,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     return mbar_wait_slow(bar, parity, abort_flag, site, kWaitLimitNs);
 }
 
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialization may start before the previous grid in the stream ends;
+// griddep_wait() blocks until that grid has completed and its writes are
+// visible (a no-op for a normally launched grid). griddep_launch_dependents()
+// lets the next such grid start once every CTA of this one has issued it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // Named barrier over `count` threads (a multiple of 32) of this CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
