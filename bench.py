@@ -297,6 +297,18 @@ def run_ours(args):
     do_m = args.only in ("all", "mla")
     do_g = args.only in ("all", "paged")
     do_f = args.only in ("all", "fp8")
+    do_r = args.only in ("all", "rope")
+
+    # rotary position embedding on the prefill and decode workloads (tables
+    # for the Llama-3 base 500000): prefill takes q, k unrotated, decode a
+    # cache that holds rotated keys
+    ROPE_BASE = 500000.0
+    if do_r:
+        cos_p, sin_p = binding.rope_tables(w.Skv, w.d_qk, ROPE_BASE, device=dev)
+        cos_d, sin_d = binding.rope_tables(wd.Skv, wd.d_qk, ROPE_BASE, device=dev)
+        k_rot = torch.empty_like(k)
+        o_r, lse_r = torch.empty_like(o), torch.empty_like(lse)
+        od_r, ld_r = torch.empty_like(od), torch.empty_like(ld)
 
     # the GQA decode workload with its cache in e4m3, one scale per KV head
     if do_f:
@@ -335,7 +347,7 @@ def run_ours(args):
         og = torch.empty_like(od)
         lg = torch.empty_like(ld)
 
-    def step(times_p, times_d, times_m=None, times_g=None, times_f=None):
+    def step(times_p, times_d, times_m=None, times_g=None, times_f=None, times_rp=None, times_rd=None):
         if do_p:
             cold_l2(1.0)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -378,6 +390,23 @@ def run_ours(args):
             e9.record(stream)
             if times_f is not None:
                 times_f.append((e8, e9))
+        if do_r:
+            cold_l2(6.0)
+            e10, e11 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e10.record(stream)
+            binding.attn_fwd_rope(q, k, v, w.causal, w.scale, cos_p, sin_p, k_rot=k_rot, o=o_r, lse=lse_r,
+                                  stream=stream)
+            e11.record(stream)
+            if times_rp is not None:
+                times_rp.append((e10, e11))
+            cold_l2(7.0)
+            e12, e13 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e12.record(stream)
+            binding.attn_decode_rope(qd, kc, vc, sl_dev, wd.scale, cos_d, sin_d, o=od_r, lse=ld_r, workspace=work,
+                                     stream=stream)
+            e13.record(stream)
+            if times_rd is not None:
+                times_rd.append((e12, e13))
 
     def barrier():
         if ws > 1:
@@ -390,12 +419,12 @@ def run_ours(args):
     barrier()
     assert binding.device_status(stream) == 0, "device status not clean after warm-up"
 
-    tp, td, tm, tg, tf = [], [], [], [], []
+    tp, td, tm, tg, tf, trp, trd = [], [], [], [], [], [], []
     with ClockSampler(torch.cuda.current_device()) as clocks:
         barrier()
         t_wall0 = time.perf_counter()
         for _ in range(args.steps):
-            step(tp, td, tm, tg, tf)
+            step(tp, td, tm, tg, tf, trp, trd)
         barrier()
         t_wall = time.perf_counter() - t_wall0
     st = binding.device_status(stream)
@@ -410,6 +439,10 @@ def run_ours(args):
     mean_m = sum(ms_m) / len(ms_m)
     mean_p = sum(ms_p) / len(ms_p)
     mean_d = sum(ms_d) / len(ms_d)
+    ms_rp = [a.elapsed_time(b) for a, b in trp] or [float("nan")]
+    ms_rd = [a.elapsed_time(b) for a, b in trd] or [float("nan")]
+    mean_rp = sum(ms_rp) / len(ms_rp)
+    mean_rd = sum(ms_rd) / len(ms_rd)
 
     agg_p = aggregate({"time_s": sum(ms_p) / 1e3, "work": fl_p * args.steps}, ws)
     agg_d = aggregate({"time_s": sum(ms_d) / 1e3, "work": by_d * args.steps}, ws)
@@ -520,6 +553,17 @@ def run_ours(args):
                        "speedup_vs_bf16_cache": (mean_d / mean_f) if (do_f and do_d) else None,
                        "algorithmic_bytes": by_f if do_f else None,
                        "kernels": "attn::dec::decode_split_kernel<4, fp8> + decode_combine_kernel"},
+        "rope_prefill": {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": mean_rp,
+                         "tflops": (fl_p / (mean_rp / 1e3) / 1e12) if do_r else None,
+                         "frac_of_peak": (fl_p / (mean_rp / 1e3) / 1e12 / peak_tf) if do_r else None,
+                         "overhead_vs_attn_fwd": (mean_rp / mean_p - 1.0) if (do_r and do_p) else None,
+                         "kernels": "attn::rope::rope_apply_kernel (keys, once) + attn::pf::prefill_kernel<128, rope> "
+                                    "(queries rotated in shared memory)"},
+        "rope_decode": {"workload": f"{wd.name}, query rotated at seqlen - 1, cache of rotated keys",
+                        "ms": mean_rd, "gbs": (by_d / (mean_rd / 1e3) / 1e9) if do_r else None,
+                        "frac_of_peak": (by_d / (mean_rd / 1e3) / 1e9 / peak_bw) if do_r else None,
+                        "kernels": "attn::dec::decode_split_kernel<4> (query rotated in the MMA warp) + "
+                                   "decode_combine_kernel"},
     }
 
     cpu_baseline = None
@@ -544,7 +588,8 @@ def run_ours(args):
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
             "clocks": clocks.summary(),
-            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m) + 2 * int(do_g) + 2 * int(do_f)) * args.steps,
+            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m) + 2 * int(do_g) + 2 * int(do_f) + 4 * int(do_r)) *
+                            args.steps,
             "wall_s_timed_region": t_wall,
         }
         print(json.dumps(line), flush=True)
@@ -573,7 +618,7 @@ def main():
                     help="query rows of the headline workload per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla", "paged", "fp8"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla", "paged", "fp8", "rope"],
                     help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
     if args.impl == "reference":
