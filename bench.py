@@ -552,13 +552,23 @@ def run_ours(args):
                        "frac_of_peak": (by_f / (mean_f / 1e3) / 1e9 / peak_bw) if do_f else None,
                        "speedup_vs_bf16_cache": (mean_d / mean_f) if (do_f and do_d) else None,
                        "algorithmic_bytes": by_f if do_f else None,
-                       "kernels": "attn::dec::decode_split_kernel<4, fp8> + decode_combine_kernel"},
+                       "kernels": "attn::dec::decode_split_kernel<4, fp8> + decode_combine_kernel",
+                       "roofline": ({"bound": "hbm", "achieved": by_f / (mean_f / 1e3) / 1e9, "peak": peak_bw,
+                                     "unit": "GB/s", "frac": by_f / (mean_f / 1e3) / 1e9 / peak_bw,
+                                     "traffic": traffic.get("decode_split_kernel_4_fp8"),
+                                     "note": "achieved over split + merge launches; traffic of the split kernel"}
+                                    if do_f else None)},
         "rope_prefill": {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": mean_rp,
                          "tflops": (fl_p / (mean_rp / 1e3) / 1e12) if do_r else None,
                          "frac_of_peak": (fl_p / (mean_rp / 1e3) / 1e12 / peak_tf) if do_r else None,
                          "overhead_vs_attn_fwd": (mean_rp / mean_p - 1.0) if (do_r and do_p) else None,
                          "kernels": "attn::rope::rope_apply_kernel (keys, once) + attn::pf::prefill_kernel<128, rope> "
-                                    "(queries rotated in shared memory)"},
+                                    "(queries rotated in shared memory)",
+                         "roofline": ({"bound": "tensor", "achieved": fl_p / (mean_rp / 1e3) / 1e12, "peak": peak_tf,
+                                       "unit": "TFLOP/s", "frac": fl_p / (mean_rp / 1e3) / 1e12 / peak_tf,
+                                       "traffic": traffic.get("prefill_kernel_128_rope"),
+                                       "note": "achieved over both launches; traffic of the attention kernel"}
+                                      if do_r else None)},
         "rope_decode": {"workload": f"{wd.name}, query rotated at seqlen - 1, cache of rotated keys",
                         "ms": mean_rd, "gbs": (by_d / (mean_rd / 1e3) / 1e9) if do_r else None,
                         "frac_of_peak": (by_d / (mean_rd / 1e3) / 1e9 / peak_bw) if do_r else None,
