@@ -1,8 +1,10 @@
 // decode_gqa.cuh -- single-token GQA decode against a KV cache, split-KV.
 //
 // A work unit is (sequence b, KV head g, a block of GT query heads of that
-// group, one chunk of CH consecutive cached keys, CH = 1024 or 512). The grid is
-// persistent (two CTAs per SM); each CTA walks its share of the units.
+// group, one chunk of CH consecutive cached keys, CH = 2048 or 1024). The grid
+// is persistent (as many CTAs per SM as shared memory allows: two for the
+// bf16 and e4m3 caches at up to 8 heads per block); each CTA walks its share
+// of the units.
 //
 // Per unit, with the group's GT query rows as the narrow operand of the
 // 5th-generation tensor core (padded to NH = max(8, GT) columns):
@@ -12,9 +14,11 @@
 // K and V tiles (128 keys x 128 dims, two 64-dim boxes with the 128-byte
 // swizzle) stream HBM -> shared memory by TMA through a ring that a producer
 // warp keeps full across units; one thread issues the MMAs; four warps
-// (one TMEM lane quarter each) do the softmax and write the partial
+// (one TMEM lane quarter each) do the softmax, hand each tile's P^T to the
+// MMA thread through one of two shared slots, and write the partial
 // (o, m, l) of the chunk to the workspace. A second kernel merges the chunks
-// of each (b, h) by their log-sum-exp weights.
+// of each (b, h) by their log-sum-exp weights. With rotary tables given, the
+// MMA warp first rotates the unit's query rows at position seqlen - 1.
 //
 // Each K/V element is read from HBM once and used by all GT heads of its
 // group (the grouped sharing of "Attention Engineering: From MHA to GQA, MLA
