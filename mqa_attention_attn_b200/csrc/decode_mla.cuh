@@ -188,22 +188,25 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int s = j % NSTAGE;
                 tc_fence_after();
                 const uint32_t dcol = tmem + ((j & 1) ? COL_S1 : COL_S0);
-#pragma unroll 1
+                // the 36 MMAs fully unrolled, each descriptor the tile's (or Q's)
+                // base descriptor plus a constant offset in its 16-byte address
+                // field: the issuing thread spends no time between MMAs, which at
+                // N = 64 finish in fewer cycles than a loop iteration takes
+                const uint64_t kd0 = umma_smem_desc(smem_u32(sm.k[s][0]), 16, 1024, 2);
+                const uint64_t qd0 = umma_smem_desc(smem_u32(sm.q[0]), 16, 1024, 2);
+#pragma unroll
                 for (int bx = 0; bx < NBT; ++bx) {
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t bd = umma_smem_desc(smem_u32(sm.k[s][bx]) + 32 * k4, 16, 1024, 2);
-                        umma_ts(dcol, tmem + COL_QT + 32 * bx + 8 * k4, bd, idesc_s, (bx > 0 || k4 > 0) ? 1u : 0u);
-                    }
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        umma_ts(dcol, tmem + COL_QT + 32 * bx + 8 * k4, kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4),
+                                idesc_s, (bx > 0 || k4 > 0) ? 1u : 0u);
                 }
-#pragma unroll 1
+#pragma unroll
                 for (int bx = NBT; bx < NB; ++bx) {
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t ad = umma_smem_desc(smem_u32(sm.q[bx - NBT]) + 32 * k4, 16, 1024, 2);
-                        const uint64_t bd = umma_smem_desc(smem_u32(sm.k[s][bx]) + 32 * k4, 16, 1024, 2);
-                        umma_ss(dcol, ad, bd, idesc_s, 1u);
-                    }
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        umma_ss(dcol, qd0 + (uint64_t)(((bx - NBT) * QBOX + 32 * k4) >> 4),
+                                kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4), idesc_s, 1u);
                 }
                 umma_commit(smem_u32(&sm.s_full[j & 1]));
             };
