@@ -42,7 +42,7 @@ constexpr int NBS = NB - NBT;     // Q boxes 4-8 (columns 256-575) in shared mem
 constexpr int QBOX = M * 128;     // one 64-column box of Q: 128 rows x 128 B
 constexpr int KBOX = KT * 128;    // one 64-column box of a key tile: 64 rows x 128 B
 constexpr int NSTAGE = 2;
-constexpr int THREADS = 256;      // warp 0 TMA, warp 1 MMA, warps 4-7 softmax
+constexpr int THREADS = 256;      // warp 0 TMA, warp 1 score MMAs, warp 2 P.V MMAs, warps 4-7 softmax
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_S1 = 64;   // S double buffer (P over its first half)
@@ -55,6 +55,8 @@ struct Smem {
     uint64_t q_full;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint64_t s_full[2], p_full[2];
+    uint64_t s_free[2];                    // the P.V that read S buffer b has completed
+    uint64_t s_done;                       // every score MMA has completed
     uint64_t qt_ready;                     // Q columns 0-255 copied into TMEM
     uint64_t pv_done;                      // one phase per P.V MMA group
     uint64_t o_done;
@@ -106,10 +108,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.s_full[i]), 1);
             mbar_init(smem_u32(&sm.p_full[i]), 128);
+            mbar_init(smem_u32(&sm.s_free[i]), 1);
         }
         mbar_init(smem_u32(&sm.qt_ready), 128);
         mbar_init(smem_u32(&sm.pv_done), 1);
         mbar_init(smem_u32(&sm.o_done), 1);
+        mbar_init(smem_u32(&sm.s_done), 1);
         mbar_init(smem_u32(&sm.tail_ready), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -176,24 +180,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (lane == 0) mbar_arrive(smem_u32(&sm.tail_ready));
         }
     } else if (warp == 1) {
-        // ======================= MMA issuer =======================
+        // ======================= score MMAs =======================
+        // One thread issues S(j) = Q K_j^T for every tile, as soon as the tile
+        // has landed and its S buffer is free (the P.V of tile j-2 that read
+        // P from it has completed). The P.V MMAs come from warp 2, so that
+        // they do not queue behind the next tile's 36 score MMAs.
         if (lane == 0 && nt > 0) {
             const uint32_t idesc_s = umma_idesc_bf16(M, KT, 0, 0);
-            const uint32_t idesc_o = umma_idesc_bf16(M, 256, 0, 1);
             bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x421) &&
                       mbar_wait(smem_u32(&sm.qt_ready), 0, abort_flag, 0x425);
-            tc_fence_after();
-            // S(j) = Q K_j^T: columns 0-255 with A from TMEM, 256-575 from smem
-            auto issue_s = [&](int j) {
+            const uint64_t qd0 = umma_smem_desc(smem_u32(sm.q[0]), 16, 1024, 2);
+            for (int j = 0; ok && j < nt; ++j) {
                 const int s = j % NSTAGE;
+                ok = mbar_wait(smem_u32(&sm.kv_full[s]), (j / NSTAGE) & 1, abort_flag, 0x422);
+                if (ok && j == nt - 1 && tail < KT) ok = mbar_wait(smem_u32(&sm.tail_ready), 0, abort_flag, 0x426);
+                if (ok && j >= 2)
+                    ok = mbar_wait(smem_u32(&sm.s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, 0x427);
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t dcol = tmem + ((j & 1) ? COL_S1 : COL_S0);
                 // the 36 MMAs fully unrolled, each descriptor the tile's (or Q's)
                 // base descriptor plus a constant offset in its 16-byte address
-                // field: the issuing thread spends no time between MMAs, which at
-                // N = 64 finish in fewer cycles than a loop iteration takes
+                // field: at N = 64 an MMA finishes in fewer cycles than a loop
+                // iteration of the issuing thread would take
+                const uint32_t dcol = tmem + ((j & 1) ? COL_S1 : COL_S0);
                 const uint64_t kd0 = umma_smem_desc(smem_u32(sm.k[s][0]), 16, 1024, 2);
-                const uint64_t qd0 = umma_smem_desc(smem_u32(sm.q[0]), 16, 1024, 2);
 #pragma unroll
                 for (int bx = 0; bx < NBT; ++bx) {
 #pragma unroll
@@ -209,51 +219,37 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4), idesc_s, 1u);
                 }
                 umma_commit(smem_u32(&sm.s_full[j & 1]));
-            };
-            // O_r += P(i) V_i, V = this CTA's 256 columns of the tile
-            auto issue_pv = [&](int i) {
+            }
+            // no score MMA may still run when TMEM is released
+            umma_commit(smem_u32(&sm.s_done));
+            mbar_wait(smem_u32(&sm.s_done), 0, nullptr, 0x428);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ======================= P.V MMAs =======================
+        // O_r += P(i) V_i as soon as P(i) is written (S(i), which read the same
+        // tile, completed before the softmax saw it); V = this CTA's 256
+        // columns of the tile. Commits release the tile's stage, the S buffer
+        // and the O state the softmax may rescale.
+        if (lane == 0 && nt > 0) {
+            const uint32_t idesc_o = umma_idesc_bf16(M, 256, 0, 1);
+            bool ok = true;
+            for (int i = 0; ok && i < nt; ++i) {
                 const int s = i % NSTAGE;
+                ok = mbar_wait(smem_u32(&sm.p_full[i & 1]), (i >> 1) & 1, abort_flag, 0x423);
+                if (!ok) break;
                 tc_fence_after();
                 const uint32_t pcol = tmem + ((i & 1) ? COL_S1 : COL_S0);
-                const uint32_t vbox = smem_u32(sm.k[s][4 * rank]);
+                const uint64_t vd0 = umma_smem_desc(smem_u32(sm.k[s][4 * rank]), KBOX, 1024, 2);
 #pragma unroll
-                for (int ks = 0; ks < KT / 16; ++ks) {
-                    const uint64_t bd = umma_smem_desc(vbox + ks * 16 * 128, KBOX, 1024, 2);
-                    umma_ts(tmem + COL_O, pcol + ks * 8, bd, idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
-                }
+                for (int ks = 0; ks < KT / 16; ++ks)
+                    umma_ts(tmem + COL_O, pcol + ks * 8, vd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
+                            (i > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(smem_u32(&sm.kv_empty[s]));
                 umma_commit(smem_u32(&sm.pv_done));
-            };
-            // Issue in dependency order, whichever is ready first: S(next_s)
-            // needs its cache tile and a free S buffer (the P.V of tile
-            // next_s - 2 issued); P.V(next_pv) needs its P.
-            int next_s = 0, next_pv = 0;
-            unsigned long long t_last = globaltimer_ns();
-            while (ok && next_pv < nt) {
-                bool progressed = false;
-                if (next_s < nt && next_s <= next_pv + 1 &&
-                    mbar_try_wait(smem_u32(&sm.kv_full[next_s % NSTAGE]), (next_s / NSTAGE) & 1) &&
-                    (next_s != nt - 1 || tail == KT || mbar_try_wait(smem_u32(&sm.tail_ready), 0))) {
-                    issue_s(next_s);
-                    ++next_s;
-                    progressed = true;
-                }
-                if (next_pv < next_s && mbar_try_wait(smem_u32(&sm.p_full[next_pv & 1]), (next_pv >> 1) & 1)) {
-                    issue_pv(next_pv);
-                    ++next_pv;
-                    progressed = true;
-                }
-                if (progressed) {
-                    t_last = globaltimer_ns();
-                } else if (*abort_flag) {
-                    ok = false;
-                } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
-                    atomicOr(&g_status, kStatusTimeout);
-                    atomicCAS(&g_timeout_site, 0u, 0x426u);
-                    *abort_flag = 1;
-                    ok = false;
-                }
+                umma_commit(smem_u32(&sm.s_free[i & 1]));
             }
+            // every P.V MMA has completed (the score MMAs before them)
             umma_commit(smem_u32(&sm.o_done));
             mbar_wait(smem_u32(&sm.o_done), 0, nullptr, 0x424);
         }
