@@ -82,3 +82,59 @@ def test_decode_validation(lib):
     assert call(n_q=7) == -1                            # n_q % n_kv != 0
     assert call(d_qk=64, d_v=64) == -2                  # not a compiled decode shape
     assert call(k_s=(8 * 1024 * 128, 1024 * 128, 130)) == -3   # row stride not a multiple of 8
+
+
+def test_rope_validation(lib):
+    vp, al = ctypes.c_void_p(16), ctypes.c_void_p(4096)
+    # tables: d must be even, base finite and positive; no positions is a no-op
+    assert lib.attn_rope_tables(vp, vp, 8, 7, 10000.0, None) == -1
+    assert lib.attn_rope_tables(vp, vp, 8, 8, 0.0, None) == -1
+    assert lib.attn_rope_tables(vp, vp, 8, 8, float("inf"), None) == -1
+    assert lib.attn_rope_tables(None, vp, 8, 8, 10000.0, None) == -1
+    assert lib.attn_rope_tables(None, None, 0, 8, 10000.0, None) == 0
+    # rotation pass: d a multiple of 8, every position inside the tables, 16-byte alignment
+    assert lib.attn_rope_apply(vp, vp, 1, 2, 16, 12, 0, al, al, 64, None) == -1
+    assert lib.attn_rope_apply(vp, vp, 1, 2, 16, 64, 49, al, al, 64, None) == -1
+    assert lib.attn_rope_apply(vp, vp, 1, 2, 16, 64, -1, al, al, 64, None) == -1
+    assert lib.attn_rope_apply(ctypes.c_void_p(24), vp, 1, 2, 16, 64, 0, al, al, 64, None) == -3
+    assert lib.attn_rope_apply(vp, vp, 0, 2, 16, 64, 0, al, al, 64, None) == 0
+    # prefill: tables covering every key, a key buffer, the prefill shape rules
+    args = lambda n_pos=64, k_rot=vp, d=64, Sq=8, Skv=64, tab=al: (
+        vp, vp, vp, vp, None, 1, Sq, Skv, 4, 2, d, d, 1, 0.125, tab, tab, n_pos, k_rot, None)
+    assert lib.attn_fwd_rope(*args(n_pos=63)) == -1
+    assert lib.attn_fwd_rope(*args(k_rot=None)) == -1
+    assert lib.attn_fwd_rope(*args(tab=None)) == -1
+    assert lib.attn_fwd_rope(*args(d=96)) == -2
+    assert lib.attn_fwd_rope(*args(Sq=65, n_pos=65)) == -2
+    assert lib.attn_fwd_rope(*args(tab=ctypes.c_void_p(4100))) == -3
+    # decode: tables required, head dim 128 only (no MLA form)
+    k_s = (2 * 1024 * 128, 1024 * 128, 128)
+    assert lib.attn_decode_rope(vp, vp, vp, vp, vp, vp, 2, 8, 2, 128, 128, 1024, *k_s, *k_s, None, None, 64,
+                                0.1, al, 1 << 20, None) == -1
+    assert lib.attn_decode_rope(vp, vp, vp, vp, vp, vp, 1, 128, 1, 576, 512, 1024, *k_s, *k_s, al, al, 64,
+                                0.1, al, 1 << 20, None) == -2
+
+
+def test_window_fp8_paged_validation(lib):
+    vp = ctypes.c_void_p(256)
+    # sliding window: window >= 1, n_sink >= 0, queries no longer than keys
+    assert lib.attn_fwd_window(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 0, 0, 0.1, None) == -1
+    assert lib.attn_fwd_window(vp, vp, vp, vp, None, 1, 8, 8, 4, 2, 64, 64, 4, -1, 0.1, None) == -1
+    assert lib.attn_fwd_window(vp, vp, vp, vp, None, 1, 9, 8, 4, 2, 64, 64, 4, 0, 0.1, None) == -2
+    # e4m3 cache: scales required, strides in multiples of 16 bytes, workspace size
+    need = ctypes.c_size_t(0)
+    assert lib.attn_decode_fp8_workspace_bytes(2, 8, 2, 1024, ctypes.byref(need)) == 0
+    s8 = (2 * 1024 * 128, 1024 * 128, 128)
+    fp8 = lambda ks=vp, strides=s8, ws=need.value: lib.attn_decode_fp8(
+        vp, vp, vp, ks, vp, vp, vp, None, 2, 8, 2, 1024, *strides, *strides, 0.1, vp, ws, None)
+    assert fp8(ks=None) == -1
+    assert fp8(strides=(2 * 1024 * 136, 1024 * 136, 136)) == -3
+    assert fp8(ws=need.value - 1) == -4
+    # paged cache: page sizes of whole TMA boxes, a positive pool, workspace size
+    ps = (64 * 2 * 128, 2 * 128, 128)
+    paged = lambda page=64, pool=100, ws=1 << 24: lib.attn_decode_paged(
+        vp, vp, vp, vp, vp, vp, None, 2, 8, 2, 128, 128, page, 16, pool, *ps, *ps, 0.1, vp, ws, None)
+    assert paged(page=0) == -1
+    assert paged(pool=0) == -1
+    assert paged(page=48) == -2
+    assert paged(ws=16) == -4
