@@ -42,7 +42,8 @@ constexpr int NBS = NB - NBT;     // Q boxes 4-8 (columns 256-575) in shared mem
 constexpr int QBOX = M * 128;     // one 64-column box of Q: 128 rows x 128 B
 constexpr int KBOX = KT * 128;    // one 64-column box of a key tile: 64 rows x 128 B
 constexpr int NSTAGE = 2;
-constexpr int THREADS = 256;      // warp 0 TMA, warp 1 score MMAs, warp 2 P.V MMAs, warps 4-7 softmax
+constexpr int NG = 3;             // arrival groups of a ring stage: boxes 0-2, 3-5, 6-8
+constexpr int THREADS = 256;      // warp 0 TMA, warps 1-2 MMAs (even / odd tiles), warps 4-7 softmax
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_S1 = 64;   // S double buffer (P over its first half)
@@ -53,12 +54,11 @@ struct Smem {
     uint8_t q[NBS][QBOX];                  // 80 KB
     uint8_t k[NSTAGE][NB][KBOX];           // 144 KB; stage 1 first stages Q boxes 0-3
     uint64_t q_full;
-    uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
+    uint64_t kv_full[NSTAGE][NG], kv_empty[NSTAGE];
     uint64_t s_full[2], p_full[2];
-    uint64_t s_free[2];                    // the P.V that read S buffer b has completed
-    uint64_t s_done;                       // every score MMA has completed
+    uint64_t s_done[2];                    // every MMA of issuing thread t has completed
     uint64_t qt_ready;                     // Q columns 0-255 copied into TMEM
-    uint64_t pv_done;                      // one phase per P.V MMA group
+    uint64_t pv_done[2];                   // P.V of tile k done: barrier k & 1, phase k >> 1
     uint64_t o_done;
     uint64_t tail_ready;                   // value rows past the length cleared (last tile)
     uint32_t tmem_base;
@@ -102,18 +102,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) {
         mbar_init(smem_u32(&sm.q_full), 1);
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(smem_u32(&sm.kv_full[s]), 1);
+            for (int g = 0; g < NG; ++g) mbar_init(smem_u32(&sm.kv_full[s][g]), 1);
             mbar_init(smem_u32(&sm.kv_empty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.s_full[i]), 1);
             mbar_init(smem_u32(&sm.p_full[i]), 128);
-            mbar_init(smem_u32(&sm.s_free[i]), 1);
         }
         mbar_init(smem_u32(&sm.qt_ready), 128);
-        mbar_init(smem_u32(&sm.pv_done), 1);
+        mbar_init(smem_u32(&sm.pv_done[0]), 1);
+        mbar_init(smem_u32(&sm.pv_done[1]), 1);
         mbar_init(smem_u32(&sm.o_done), 1);
-        mbar_init(smem_u32(&sm.s_done), 1);
+        mbar_init(smem_u32(&sm.s_done[0]), 1);
+        mbar_init(smem_u32(&sm.s_done[1]), 1);
         mbar_init(smem_u32(&sm.tail_ready), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -148,15 +149,20 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (ok && j >= NSTAGE)
                     ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / NSTAGE) + 1) & 1, abort_flag, 0x411);
                 if (!ok) break;
-                const uint32_t fb = smem_u32(&sm.kv_full[s]);
-                mbar_arrive_expect_tx(fb, (uint32_t)(NB * KBOX));
-                for (int bx = 0; bx < NB; ++bx)
-                    tma_load_3d(smem_u32(sm.k[s][bx]), &tm_c, fb, 64 * bx, j * KT, b);
+                // one barrier per group of three boxes, so that the score MMAs
+                // of a group start while the later groups are still in flight
+                for (int g = 0; g < NG; ++g) {
+                    const uint32_t fb = smem_u32(&sm.kv_full[s][g]);
+                    mbar_arrive_expect_tx(fb, (uint32_t)(NB / NG * KBOX));
+                    for (int bx = g * (NB / NG); bx < (g + 1) * (NB / NG); ++bx)
+                        tma_load_3d(smem_u32(sm.k[s][bx]), &tm_c, fb, 64 * bx, j * KT, b);
+                }
                 ++issued;
             }
             mbar_wait(qbar, 0, nullptr, 0x412);
             for (int j = issued - 1; j >= 0 && j >= issued - NSTAGE; --j)
-                mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE]), (j / NSTAGE) & 1, nullptr, 0x413);
+                for (int g = 0; g < NG; ++g)
+                    mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE][g]), (j / NSTAGE) & 1, nullptr, 0x413);
         }
         __syncwarp();
         if (tail < KT) {
@@ -165,7 +171,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // the cache holds there cannot reach the output. Done before the
             // last tile's MMAs are issued (they wait for tail_ready).
             const int s = (nt - 1) % NSTAGE;
-            bool ok = mbar_wait(smem_u32(&sm.kv_full[s]), ((nt - 1) / NSTAGE) & 1, abort_flag, 0x414);
+            bool ok = true;
+            for (int g = 0; ok && g < NG; ++g)
+                ok = mbar_wait(smem_u32(&sm.kv_full[s][g]), ((nt - 1) / NSTAGE) & 1, abort_flag, 0x414);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 for (int e = tail * 8 + (int)lane; e < KT * 8; e += 32) {
@@ -179,79 +187,76 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.tail_ready));
         }
-    } else if (warp == 1) {
-        // ======================= score MMAs =======================
-        // One thread issues S(j) = Q K_j^T for every tile, as soon as the tile
-        // has landed and its S buffer is free (the P.V of tile j-2 that read
-        // P from it has completed). The P.V MMAs come from warp 2, so that
-        // they do not queue behind the next tile's 36 score MMAs.
-        if (lane == 0 && nt > 0) {
+    } else if (warp == 1 || warp == 2) {
+        // ======================= MMA issue =======================
+        // Two threads, one per S buffer: warp 1 takes the even tiles (S buffer
+        // 0, ring stage 0), warp 2 the odd ones. Each issues its tile's 36
+        // score MMAs, then, once the softmax has written P, the tile's P.V;
+        // in one thread's program order the next score MMAs into the same S
+        // buffer follow that P.V. The P.V MMAs of both threads accumulate
+        // into the same O, so each waits for the previous tile's P.V to
+        // complete: pv_done[k & 1], committed only by the thread of tile k,
+        // phase k >> 1. A thread at tile j has itself waited for the phase of
+        // tile j - 3 on the other barrier, so the phase it waits for next
+        // cannot be confused with an older one of the same parity.
+        const int par = (int)warp - 1;
+        if (lane == 0 && nt > par) {
             const uint32_t idesc_s = umma_idesc_bf16(M, KT, 0, 0);
+            const uint32_t idesc_o = umma_idesc_bf16(M, 256, 0, 1);
             bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x421) &&
                       mbar_wait(smem_u32(&sm.qt_ready), 0, abort_flag, 0x425);
             const uint64_t qd0 = umma_smem_desc(smem_u32(sm.q[0]), 16, 1024, 2);
-            for (int j = 0; ok && j < nt; ++j) {
-                const int s = j % NSTAGE;
-                ok = mbar_wait(smem_u32(&sm.kv_full[s]), (j / NSTAGE) & 1, abort_flag, 0x422);
+            const uint32_t dcol = tmem + (par ? COL_S1 : COL_S0);
+            for (int j = par; ok && j < nt; j += 2) {
+                const int s = j % NSTAGE;   // == par
+                const uint32_t ph = (uint32_t)(j / NSTAGE) & 1u;
+                ok = mbar_wait(smem_u32(&sm.kv_full[s][0]), ph, abort_flag, 0x422);
                 if (ok && j == nt - 1 && tail < KT) ok = mbar_wait(smem_u32(&sm.tail_ready), 0, abort_flag, 0x426);
-                if (ok && j >= 2)
-                    ok = mbar_wait(smem_u32(&sm.s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, 0x427);
                 if (!ok) break;
                 tc_fence_after();
-                // the 36 MMAs fully unrolled, each descriptor the tile's (or Q's)
-                // base descriptor plus a constant offset in its 16-byte address
-                // field: at N = 64 an MMA finishes in fewer cycles than a loop
-                // iteration of the issuing thread would take
-                const uint32_t dcol = tmem + ((j & 1) ? COL_S1 : COL_S0);
+                // the 36 score MMAs fully unrolled, each descriptor the tile's (or
+                // Q's) base descriptor plus a constant offset in its 16-byte
+                // address field (at N = 64 an MMA finishes in fewer cycles than
+                // a loop iteration of the issuing thread would take); boxes
+                // 3-5 and 6-8 are waited for just before their MMAs
                 const uint64_t kd0 = umma_smem_desc(smem_u32(sm.k[s][0]), 16, 1024, 2);
 #pragma unroll
-                for (int bx = 0; bx < NBT; ++bx) {
+                for (int bx = 0; bx < NB; ++bx) {
+                    if (bx > 0 && bx % (NB / NG) == 0) {
+                        ok = mbar_wait(smem_u32(&sm.kv_full[s][bx / (NB / NG)]), ph, abort_flag, 0x429);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4)
-                        umma_ts(dcol, tmem + COL_QT + 32 * bx + 8 * k4, kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4),
-                                idesc_s, (bx > 0 || k4 > 0) ? 1u : 0u);
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        if (bx < NBT)
+                            umma_ts(dcol, tmem + COL_QT + 32 * bx + 8 * k4, kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4),
+                                    idesc_s, (bx > 0 || k4 > 0) ? 1u : 0u);
+                        else
+                            umma_ss(dcol, qd0 + (uint64_t)(((bx - NBT) * QBOX + 32 * k4) >> 4),
+                                    kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4), idesc_s, 1u);
+                    }
                 }
-#pragma unroll
-                for (int bx = NBT; bx < NB; ++bx) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4)
-                        umma_ss(dcol, qd0 + (uint64_t)(((bx - NBT) * QBOX + 32 * k4) >> 4),
-                                kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4), idesc_s, 1u);
-                }
+                if (!ok) break;
                 umma_commit(smem_u32(&sm.s_full[j & 1]));
-            }
-            // no score MMA may still run when TMEM is released
-            umma_commit(smem_u32(&sm.s_done));
-            mbar_wait(smem_u32(&sm.s_done), 0, nullptr, 0x428);
-        }
-        __syncwarp();
-    } else if (warp == 2) {
-        // ======================= P.V MMAs =======================
-        // O_r += P(i) V_i as soon as P(i) is written (S(i), which read the same
-        // tile, completed before the softmax saw it); V = this CTA's 256
-        // columns of the tile. Commits release the tile's stage, the S buffer
-        // and the O state the softmax may rescale.
-        if (lane == 0 && nt > 0) {
-            const uint32_t idesc_o = umma_idesc_bf16(M, 256, 0, 1);
-            bool ok = true;
-            for (int i = 0; ok && i < nt; ++i) {
-                const int s = i % NSTAGE;
-                ok = mbar_wait(smem_u32(&sm.p_full[i & 1]), (i >> 1) & 1, abort_flag, 0x423);
+                // O_r += P(j) V_j, V = this CTA's 256 columns of the tile, after
+                // the P.V of tile j - 1 (the other thread's) has completed
+                ok = mbar_wait(smem_u32(&sm.p_full[j & 1]), (j >> 1) & 1, abort_flag, 0x423);
+                if (ok && j > 0) ok = mbar_wait(smem_u32(&sm.pv_done[par ^ 1]), ((j - 1) >> 1) & 1, abort_flag, 0x427);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t pcol = tmem + ((i & 1) ? COL_S1 : COL_S0);
                 const uint64_t vd0 = umma_smem_desc(smem_u32(sm.k[s][4 * rank]), KBOX, 1024, 2);
 #pragma unroll
                 for (int ks = 0; ks < KT / 16; ++ks)
-                    umma_ts(tmem + COL_O, pcol + ks * 8, vd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
-                            (i > 0 || ks > 0) ? 1u : 0u);
+                    umma_ts(tmem + COL_O, dcol + ks * 8, vd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
+                            (j > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(smem_u32(&sm.kv_empty[s]));
-                umma_commit(smem_u32(&sm.pv_done));
-                umma_commit(smem_u32(&sm.s_free[i & 1]));
+                umma_commit(smem_u32(&sm.pv_done[par]));
+                if (j == nt - 1) umma_commit(smem_u32(&sm.o_done));   // O final (tile nt-2's P.V already done)
             }
-            // every P.V MMA has completed (the score MMAs before them)
-            umma_commit(smem_u32(&sm.o_done));
-            mbar_wait(smem_u32(&sm.o_done), 0, nullptr, 0x424);
+            // no MMA of this thread may still run when TMEM is released
+            umma_commit(smem_u32(&sm.s_done[par]));
+            mbar_wait(smem_u32(&sm.s_done[par]), 0, nullptr, 0x428);
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -314,10 +319,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (j == 0) {
                 m_run = m_new;
             } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold)) {
-                // O must be stable: wait for the P.V of tile j-1 (phase j-1 of
-                // pv_done; the one of tile j-2 is already covered by s_full of
-                // tile j). The P.V of tile j starts only after p_full below.
-                ok = mbar_wait(smem_u32(&sm.pv_done), (j - 1) & 1, abort_flag, 0x435);
+                // O must be stable: wait for the P.V of tile j-1 (barrier
+                // (j-1) & 1, phase (j-1) >> 1; the P.V of tile j-2 came before
+                // the score MMAs of tile j in the same thread, and that of
+                // tile j-3 was waited for by the P.V of tile j-2). The P.V of
+                // tile j starts only after p_full below.
+                ok = mbar_wait(smem_u32(&sm.pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort_flag, 0x435);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 __syncwarp();
