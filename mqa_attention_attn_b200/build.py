@@ -13,7 +13,6 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn_b200.so")
 SOURCES = ["attn_api.cu"]
-DEPS = ["attn_api.cu", "sm100.cuh", "prefill.cuh", "decode_gqa.cuh", "decode_mla.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -30,11 +29,16 @@ def _nvcc() -> str:
     return "nvcc"
 
 
+def _deps() -> list:
+    """Every CUDA source and header of the library (all of csrc/)."""
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
+
+
 def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, d) for d in DEPS if os.path.exists(os.path.join(CSRC, d))]
+    deps = _deps()
     deps.append(os.path.join(ROOT, "include", "attn.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
