@@ -1,0 +1,348 @@
+"""Executable models of the barrier protocols of the tensor-core kernels
+(race detection on the CPU).
+
+Each model replays one CTA's roles -- TMA producers, MMA-issuing threads,
+softmax warpgroups -- as coroutines under random interleavings, with:
+
+* mbarriers of exact phase / parity semantics: an arrival count and a
+  transaction-byte count per phase; ``try_wait.parity(P)`` succeeds once the
+  most recently completed phase has parity P;
+* TMA copies that land at random later times (``complete_tx``);
+* one in-order queue of MMAs and commits per issuing thread; the queues of
+  different threads drain in arbitrary interleaving (a superset of what one
+  tensor pipe can do), and a commit arrives when its queue reaches it, i.e.
+  after every earlier MMA of that thread.
+
+The data each step reads or overwrites (ring stages, score / P buffers in
+TMEM, the output accumulator) is tracked, and every hazard -- a stage
+refilled before its last reader ran, P overwritten before P V read it, O
+touched while a P V may still run, a wait that can never complete -- raises
+``Hazard``. The kernels modelled: ``attn::pf::prefill_kernel`` (dense mode:
+two ping-pong query tiles, K ring of 2, V ring of 3, three release
+barriers) and ``attn::mla::mla_decode_kernel`` (two issuing threads taking
+even and odd tiles, per-group arrival barriers, the Q staging in ring
+stage 1, the tail clearing). ``bug`` plants one protocol mistake, so that
+tests can show a model catches it.
+"""
+from __future__ import annotations
+
+import random
+
+
+class Hazard(AssertionError):
+    pass
+
+
+def check(cond, *what):
+    if not cond:
+        raise Hazard(what)
+
+
+class Bar:
+    """An mbarrier: expected arrivals per phase, pending transaction bytes."""
+
+    def __init__(self, name: str, count: int):
+        self.name, self.count, self.pending, self.tx, self.phase = name, count, count, 0, 0
+
+    def arrive(self):
+        self.pending -= 1
+        check(self.pending >= 0, "extra arrival", self.name)
+        self._advance()
+
+    def expect_tx(self, n: int):
+        self.tx += n
+
+    def complete_tx(self, n: int):
+        self.tx -= n
+        self._advance()
+
+    def _advance(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def test(self, parity: int) -> bool:
+        return (self.phase & 1) != parity
+
+
+class Sim:
+    def __init__(self, seed: int):
+        self.rng = random.Random(seed)
+        self.bars: dict[str, Bar] = {}
+        self.loads: list = []
+        self.queues: dict[str, list] = {}
+
+    def bar(self, name: str, count: int):
+        self.bars[name] = Bar(name, count)
+
+    def wait(self, name: str, parity: int):
+        while not self.bars[name].test(parity):
+            yield
+
+    def load(self, bar: str, on_land):
+        """A TMA copy completing `bar` (expect_tx + arrive by the issuer)."""
+        b = self.bars[bar]
+        b.expect_tx(1)
+        b.arrive()
+        self.loads.append((bar, on_land))
+
+    def mma(self, thread: str, fn):
+        self.queues.setdefault(thread, []).append(("mma", fn))
+
+    def commit(self, thread: str, bar: str):
+        self.queues.setdefault(thread, []).append(("commit", bar))
+
+    def run(self, roles, limit: int = 400000):
+        alive = list(roles)
+        steps = 0
+        while alive or self.loads or any(self.queues.values()):
+            steps += 1
+            check(steps < limit, "no progress: a wait can never complete")
+            c = self.rng.random()
+            if c < 0.15 and self.loads:
+                bar, on_land = self.loads.pop(self.rng.randrange(len(self.loads)))
+                on_land()
+                self.bars[bar].complete_tx(1)
+                continue
+            if c < 0.40:
+                busy = [k for k, q in self.queues.items() if q]
+                if busy:
+                    kind, x = self.queues[self.rng.choice(busy)].pop(0)
+                    if kind == "mma":
+                        x()
+                    else:
+                        self.bars[x].arrive()
+                    continue
+            if not alive:
+                continue
+            r = self.rng.choice(alive)
+            try:
+                next(r)
+            except StopIteration:
+                alive.remove(r)
+
+
+# ---------------------------------------------------------------------------
+# attn::pf::prefill_kernel (dense mode)
+# ---------------------------------------------------------------------------
+KSTAGE, VSTAGE, NREL = 2, 3, 3
+PREFILL_BUGS = ("k_release_early", "v_release_early", "s_before_pv", "no_v_wait")
+
+
+def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = None):
+    """Tile t visits key tiles 0 .. nt[t]-1 (the second tile may have one
+    more, as consecutive position blocks do, or none)."""
+    sim = Sim(seed)
+    nmax = max(nt)
+    sim.bar("q_full", 1)
+    for s in range(KSTAGE):
+        sim.bar(f"k_full{s}", 1)
+    for s in range(VSTAGE):
+        sim.bar(f"v_full{s}", 1)
+    for i in range(NREL):
+        sim.bar(f"rel{i}", 1)
+    for t in range(2):
+        sim.bar(f"s_full{t}", 1)
+        sim.bar(f"p_full{t}", 1)
+        sim.bar(f"o_done{t}", 1)
+    sim.bar("mma_done", 1)
+    kst, vst = {}, {}
+    s_done, pv_done, sbuf, pbuf = set(), set(), {}, {}
+
+    def producer_k():
+        if nt[0] or nt[1]:
+            sim.load("q_full", lambda: None)
+        for j in range(nmax):
+            s = j % KSTAGE
+            if j >= KSTAGE:
+                it = max(0, j - KSTAGE - (2 if bug == "k_release_early" else 1))
+                yield from sim.wait(f"rel{it % NREL}", (it // NREL) & 1)
+                # K tile j - KSTAGE was last read by the S MMAs issued in iteration j - KSTAGE - 1
+                for t in range(2):
+                    check(j - KSTAGE >= nt[t] or (t, j - KSTAGE) in s_done, "K stage refilled early", j)
+            sim.load(f"k_full{s}", lambda s=s, j=j: kst.__setitem__(s, j))
+            yield
+
+    def producer_v():
+        for j in range(nmax):
+            s = j % VSTAGE
+            if j >= VSTAGE:
+                it = j - VSTAGE - (1 if bug == "v_release_early" else 0)
+                if it >= 0:
+                    yield from sim.wait(f"rel{it % NREL}", (it // NREL) & 1)
+                for t in range(2):
+                    check(j - VSTAGE >= nt[t] or (t, j - VSTAGE) in pv_done, "V stage refilled early", j)
+            sim.load(f"v_full{s}", lambda s=s, j=j: vst.__setitem__(s, j))
+            yield
+
+    def issue_s(t, j):
+        def ex():
+            check(kst.get(j % KSTAGE) == j, "S reads the wrong K tile", t, j)
+            check(pbuf.get(t) is None or (t, pbuf[t]) in pv_done, "S overwrote an unread P", t, j)
+            sbuf[t] = j
+            s_done.add((t, j))
+        sim.mma("mma", ex)
+        sim.commit("mma", f"s_full{t}")
+
+    def issue_pv(t, j):
+        yield from sim.wait(f"p_full{t}", j & 1)
+        def ex():
+            check(pbuf.get(t) == j, "P V reads the wrong P", t, j)
+            check(vst.get(j % VSTAGE) == j, "P V reads the wrong V tile", t, j)
+            pv_done.add((t, j))
+        sim.mma("mma", ex)
+        if j == nt[t] - 1:
+            sim.commit("mma", f"o_done{t}")
+
+    def mma():
+        yield from sim.wait("q_full", 0)
+        if nmax > 0:
+            yield from sim.wait("k_full0", 0)
+            for t in range(2):
+                if nt[t] > 0:
+                    issue_s(t, 0)
+        for j in range(nmax):
+            if bug != "no_v_wait":
+                yield from sim.wait(f"v_full{j % VSTAGE}", (j // VSTAGE) & 1)
+            if j + 1 < nmax:
+                yield from sim.wait(f"k_full{(j + 1) % KSTAGE}", ((j + 1) // KSTAGE) & 1)
+            for t in range(2):
+                if j >= nt[t]:
+                    continue
+                if bug == "s_before_pv" and j + 1 < nt[t]:
+                    issue_s(t, j + 1)
+                    yield from issue_pv(t, j)
+                    continue
+                yield from issue_pv(t, j)
+                if j + 1 < nt[t]:
+                    issue_s(t, j + 1)
+            sim.commit("mma", f"rel{j % NREL}")
+            yield
+        sim.commit("mma", "mma_done")
+        yield from sim.wait("mma_done", 0)
+
+    def softmax(t):
+        for j in range(nt[t]):
+            yield from sim.wait(f"s_full{t}", j & 1)
+            check(sbuf.get(t) == j, "softmax reads the wrong S", t, j)
+            if j > 0 and sim.rng.random() < rescale_p:
+                # O stable: S of tile j was committed after P V of tile j-1
+                check((t, j - 1) in pv_done, "O rescaled while a P V may run", t, j)
+            pbuf[t] = j
+            sim.bars[f"p_full{t}"].arrive()
+            yield
+        if nt[t] > 0:
+            yield from sim.wait(f"o_done{t}", 0)
+            check(all((t, j) in pv_done for j in range(nt[t])), "epilogue before the last P V", t)
+
+    sim.run([producer_k(), producer_v(), mma(), softmax(0), softmax(1)])
+    check(len(pv_done) == nt[0] + nt[1], "P V missing")
+
+
+# ---------------------------------------------------------------------------
+# attn::mla::mla_decode_kernel
+# ---------------------------------------------------------------------------
+NG = 3
+MLA_BUGS = ("kv_empty_parity", "no_qt_ready", "no_tail_ready", "no_group_wait", "pv_unordered")
+
+
+def mla(nt: int, tail_partial: bool, seed: int, rescale_p: float, bug: str | None = None):
+    sim = Sim(seed)
+    for n in ("q_full", "qt_ready", "tail_ready", "o_done"):
+        sim.bar(n, 1)
+    for s in range(2):
+        sim.bar(f"kv_empty{s}", 1)
+        for g in range(NG):
+            sim.bar(f"kv_full{s}_{g}", 1)
+    for i in range(2):
+        for n in ("s_full", "p_full", "pv_done", "s_done"):
+            sim.bar(f"{n}{i}", 1)
+    stage = {(s, g): None for s in range(2) for g in range(NG)}
+    stage[(1, 0)] = stage[(1, 1)] = "Q"      # Q columns 0-255 staged in ring stage 1
+    st = dict(q_copied=False, tail_cleared=False)
+    s_done, pv_done, sbuf, pbuf = set(), set(), {}, {}
+
+    def producer():
+        sim.load("q_full", lambda: None)
+        for j in range(nt):
+            s = j % 2
+            if j == 1 and bug != "no_qt_ready":
+                yield from sim.wait("qt_ready", 0)
+            if j >= 2:
+                par = ((j // 2) + (0 if bug == "kv_empty_parity" else 1)) & 1
+                yield from sim.wait(f"kv_empty{s}", par)
+                check((j - 2) in s_done and (j - 2) in pv_done, "ring stage refilled early", j)
+            for g in range(NG):
+                sim.load(f"kv_full{s}_{g}", lambda s=s, g=g, j=j: stage.__setitem__((s, g), j))
+            yield
+        if nt > 0 and tail_partial:            # rows past the length cleared in the last tile
+            s = (nt - 1) % 2
+            for g in range(NG):
+                yield from sim.wait(f"kv_full{s}_{g}", ((nt - 1) // 2) & 1)
+            check(all(stage[(s, g)] == nt - 1 for g in range(NG)), "tail cleared before its tile landed")
+            st["tail_cleared"] = True
+            sim.bars["tail_ready"].arrive()
+
+    def qcopy():
+        if nt > 0:
+            yield from sim.wait("q_full", 0)
+            check(stage[(1, 0)] == "Q" and stage[(1, 1)] == "Q", "Q staging overwritten before the copy")
+            st["q_copied"] = True
+            sim.bars["qt_ready"].arrive()
+
+    def issuer(par):
+        if nt <= par:
+            return
+        th = f"mma{par}"
+        yield from sim.wait("q_full", 0)
+        yield from sim.wait("qt_ready", 0)
+        for j in range(par, nt, 2):
+            s, ph = j % 2, (j // 2) & 1
+            yield from sim.wait(f"kv_full{s}_0", ph)
+            if j == nt - 1 and tail_partial and bug != "no_tail_ready":
+                yield from sim.wait("tail_ready", 0)
+            for g in range(NG):
+                if g > 0 and bug != "no_group_wait":
+                    yield from sim.wait(f"kv_full{s}_{g}", ph)
+                def ex(j=j, s=s, g=g):
+                    check(stage[(s, g)] == j, "score MMA reads the wrong tile", j, g)
+                    check(not (j == nt - 1 and tail_partial) or st["tail_cleared"], "tail read before cleared", j)
+                    check(g > 0 or pbuf.get(j & 1) is None or pbuf[j & 1] in pv_done, "S overwrote an unread P", j)
+                    if g == NG - 1:
+                        sbuf[j & 1] = j
+                        s_done.add(j)
+                sim.mma(th, ex)
+            sim.commit(th, f"s_full{j & 1}")
+            yield from sim.wait(f"p_full{j & 1}", (j >> 1) & 1)
+            if j > 0 and bug != "pv_unordered":
+                yield from sim.wait(f"pv_done{par ^ 1}", ((j - 1) >> 1) & 1)
+            def pv(j=j, s=s):
+                check(pbuf.get(j & 1) == j, "P V reads the wrong P", j)
+                check(all(stage[(s, g)] == j for g in range(NG)), "P V reads the wrong tile", j)
+                check(j == 0 or (j - 1) in pv_done, "O accumulated out of order", j)
+                pv_done.add(j)
+            sim.mma(th, pv)
+            sim.commit(th, f"kv_empty{s}")
+            sim.commit(th, f"pv_done{par}")
+            if j == nt - 1:
+                sim.commit(th, "o_done")
+            yield
+        sim.commit(th, f"s_done{par}")
+        yield from sim.wait(f"s_done{par}", 0)
+
+    def softmax():
+        for j in range(nt):
+            yield from sim.wait(f"s_full{j & 1}", (j >> 1) & 1)
+            check(sbuf.get(j & 1) == j, "softmax reads the wrong S", j)
+            if j > 0 and sim.rng.random() < rescale_p:
+                yield from sim.wait(f"pv_done{(j - 1) & 1}", ((j - 1) >> 1) & 1)
+                check((j - 1) in pv_done, "O rescaled while a P V may run", j)
+            pbuf[j & 1] = j
+            sim.bars[f"p_full{j & 1}"].arrive()
+            yield
+        if nt > 0:
+            yield from sim.wait("o_done", 0)
+            check(pv_done == set(range(nt)), "epilogue before the last P V")
+
+    sim.run([producer(), qcopy(), issuer(0), issuer(1), softmax()])
+    check(pv_done == set(range(nt)), "P V missing")
