@@ -19,10 +19,12 @@ refilled before its last reader ran, P overwritten before P V read it, O
 touched while a P V may still run, a wait that can never complete -- raises
 ``Hazard``. The kernels modelled: ``attn::pf::prefill_kernel`` (dense mode:
 two ping-pong query tiles, K ring of 2, V ring of 3, three release
-barriers) and ``attn::mla::mla_decode_kernel`` (two issuing threads taking
+barriers), ``attn::mla::mla_decode_kernel`` (two issuing threads taking
 even and odd tiles, per-group arrival barriers, the Q staging in ring
-stage 1, the tail clearing). ``bug`` plants one protocol mistake, so that
-tests can show a model catches it.
+stage 1, the tail clearing) and ``attn::dec::decode_split_kernel``
+(persistent over units, one ring for K then V tiles, two P slots, the
+8-bit path's converter warps between an 8-bit ring and the ring). ``bug``
+plants one protocol mistake, so that tests can show a model catches it.
 """
 from __future__ import annotations
 
@@ -346,3 +348,145 @@ def mla(nt: int, tail_partial: bool, seed: int, rescale_p: float, bug: str | Non
 
     sim.run([producer(), qcopy(), issuer(0), issuer(1), softmax()])
     check(pv_done == set(range(nt)), "P V missing")
+
+
+# ---------------------------------------------------------------------------
+# attn::dec::decode_split_kernel (persistent: a CTA walks several units)
+# ---------------------------------------------------------------------------
+DEC_NSTAGE, DEC_NSTAGE8 = 2, 2
+DECODE_BUGS = ("q_reload_early", "empty_parity", "p_slot_parity", "no_p_wait", "conv_no_empty_wait")
+
+
+def decode(units: list[int], seed: int, fp8: bool = False, bug: str | None = None):
+    """One CTA's units in order; unit n holds units[n] key tiles. A unit
+    streams its K tiles (score MMAs into TMEM), then its V tiles (P V into
+    the output accumulator), through one ring; on the 8-bit path the tiles
+    land in an 8-bit ring and converter warps widen them into the ring."""
+    sim = Sim(seed)
+    NS, NS8 = DEC_NSTAGE, DEC_NSTAGE8
+    for n in ("q_full", "q_empty", "q_conv", "s_full", "o_full", "mma_done"):
+        sim.bar(n, 1)
+    for s in range(NS):
+        sim.bar(f"full{s}", 1)
+        sim.bar(f"empty{s}", 1)
+    for s in range(NS8):
+        sim.bar(f"full8_{s}", 1)
+        sim.bar(f"empty8_{s}", 1)
+    for x in range(2):
+        sim.bar(f"p_full{x}", 1)
+        sim.bar(f"p_empty{x}", 1)
+    st = dict(q=None, qconv=None)
+    ring, ring8, sread, pslot = {}, {}, set(), {}
+    s_tiles, s_exec, pv_exec, o_read, ring_used, ring8_used = {}, set(), set(), set(), {}, {}
+
+    def tiles(n):           # (unit, tile index within the unit's 2 * units[n] ring tiles)
+        return [(n, j) for j in range(2 * units[n])]
+
+    def producer():
+        t = 0
+        for n in range(len(units)):
+            if n > 0 and bug != "q_reload_early":
+                yield from sim.wait("q_empty", (n - 1) & 1)
+            sim.load("q_full", lambda n=n: st.__setitem__("q", n))
+            for tile in tiles(n):
+                if fp8:
+                    s8 = t % NS8
+                    yield from sim.wait(f"empty8_{s8}", ((t // NS8) & 1) ^ 1)
+                    check(ring8.get(s8) is None or ring8_used.get(s8) == ring8[s8], "8-bit stage refilled early", tile)
+                    sim.load(f"full8_{s8}", lambda s8=s8, tile=tile: ring8.__setitem__(s8, tile))
+                else:
+                    s = t % NS
+                    par = ((t // NS) & 1) ^ (0 if bug == "empty_parity" else 1)
+                    yield from sim.wait(f"empty{s}", par)
+                    check(ring.get(s) is None or ring_used.get(s) == ring[s], "ring stage refilled early", tile)
+                    sim.load(f"full{s}", lambda s=s, tile=tile: ring.__setitem__(s, tile))
+                t += 1
+                yield
+
+    def converter():
+        t = 0
+        for n in range(len(units)):
+            yield from sim.wait("q_full", n & 1)
+            check(st["q"] == n, "converter reads the wrong Q", n)
+            st["qconv"] = n
+            sim.bars["q_conv"].arrive()
+            for tile in tiles(n):
+                s8, s = t % NS8, t % NS
+                yield from sim.wait(f"full8_{s8}", (t // NS8) & 1)
+                if bug != "conv_no_empty_wait":
+                    yield from sim.wait(f"empty{s}", ((t // NS) & 1) ^ 1)
+                check(ring8.get(s8) == tile, "converter reads the wrong 8-bit tile", tile)
+                check(ring.get(s) is None or ring_used.get(s) == ring[s], "ring stage overwritten early", tile)
+                ring[s] = tile
+                ring8_used[s8] = tile
+                sim.bars[f"full{s}"].arrive()
+                sim.bars[f"empty8_{s8}"].arrive()
+                t += 1
+                yield
+
+    def mma():
+        t = pc = 0
+        for n, nt in enumerate(units):
+            yield from sim.wait("q_conv" if fp8 else "q_full", n & 1)
+            for j in range(nt):
+                g = t + j
+                s = g % NS
+                yield from sim.wait(f"full{s}", (g // NS) & 1)
+                def ex(n=n, j=j, s=s):
+                    check(ring.get(s) == (n, j), "score MMA reads the wrong K tile", n, j)
+                    check(st["q"] == n and (not fp8 or st["qconv"] == n), "score MMA reads the wrong Q", n)
+                    check(n == 0 or j >= units[n - 1] or (n - 1, j) in sread, "S overwritten while being read", n, j)
+                    ring_used[s] = (n, j)
+                    s_tiles[j] = n
+                    s_exec.add((n, j))
+                sim.mma("mma", ex)
+                sim.commit("mma", f"empty{s}")
+            sim.commit("mma", "q_empty")
+            sim.commit("mma", "s_full")
+            t += nt
+            for j in range(nt):
+                g = t + j
+                s = g % NS
+                yield from sim.wait(f"full{s}", (g // NS) & 1)
+                if bug != "no_p_wait":
+                    yield from sim.wait(f"p_full{pc & 1}", (pc >> 1) & 1)
+                def pv(n=n, j=j, s=s, x=pc & 1, nt=nt):
+                    check(ring.get(s) == (n, nt + j), "P V reads the wrong V tile", n, j)
+                    check(pslot.get(x) == (n, j), "P V reads the wrong P", n, j)
+                    check(j > 0 or n == 0 or (n - 1) in o_read, "O overwritten before it was read", n)
+                    check(j == 0 or (n, j - 1) in pv_exec, "O accumulated out of order", n, j)
+                    ring_used[s] = (n, nt + j)
+                    pv_exec.add((n, j))
+                sim.mma("mma", pv)
+                sim.commit("mma", f"empty{s}")
+                sim.commit("mma", f"p_empty{pc & 1}")
+                pc += 1
+            sim.commit("mma", "o_full")
+            t += nt
+            yield
+        sim.commit("mma", "mma_done")
+        yield from sim.wait("mma_done", 0)
+
+    def softmax():
+        pc = 0
+        for n, nt in enumerate(units):
+            yield from sim.wait("s_full", n & 1)
+            check(all(s_tiles.get(j) == n for j in range(nt)), "softmax reads S of another unit", n)
+            for j in range(nt):
+                check(s_tiles.get(j) == n, "S tile overwritten during pass 2", n, j)
+                sread.add((n, j))
+                par = ((pc >> 1) & 1) ^ (0 if bug == "p_slot_parity" else 1)
+                yield from sim.wait(f"p_empty{pc & 1}", par)
+                prev = pslot.get(pc & 1)
+                check(prev is None or prev in pv_exec, "P slot overwritten before P V read it", n, j)
+                pslot[pc & 1] = (n, j)
+                sim.bars[f"p_full{pc & 1}"].arrive()
+                pc += 1
+                yield
+            yield from sim.wait("o_full", n & 1)
+            check(all((n, j) in pv_exec for j in range(nt)), "output read before the last P V", n)
+            o_read.add(n)
+
+    roles = [producer(), mma(), softmax()] + ([converter()] if fp8 else [])
+    sim.run(roles)
+    check(len(pv_exec) == sum(units), "P V missing")

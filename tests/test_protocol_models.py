@@ -44,3 +44,23 @@ def test_mla_planted_bug_is_caught(bug):
             for tail_partial in (False, True):
                 for seed in range(40):
                     pm.mla(nt, tail_partial, seed, rescale_p=0.5, bug=bug)
+
+
+def _decode_cases():
+    import random
+    rng = random.Random(7)
+    for trial in range(120):
+        yield trial, [rng.randint(1, 5) for _ in range(rng.randint(1, 4))]
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_protocol_hazard_free(fp8):
+    for seed, units in _decode_cases():
+        pm.decode(units, seed, fp8=fp8)
+
+
+@pytest.mark.parametrize("bug", pm.DECODE_BUGS)
+def test_decode_planted_bug_is_caught(bug):
+    with pytest.raises(pm.Hazard):
+        for seed, units in _decode_cases():
+            pm.decode(units, seed, fp8=bug.startswith("conv"), bug=bug)
