@@ -128,12 +128,14 @@ class Sim:
 # attn::pf::prefill_kernel (dense mode)
 # ---------------------------------------------------------------------------
 KSTAGE, VSTAGE, NREL = 2, 3, 3
-PREFILL_BUGS = ("k_release_early", "v_release_early", "s_before_pv", "no_v_wait")
+PREFILL_BUGS = ("k_release_early", "v_release_early", "s_before_pv", "no_v_wait", "no_q_rot_wait")
 
 
-def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = None):
+def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = None, rope: bool = False):
     """Tile t visits key tiles 0 .. nt[t]-1 (the second tile may have one
-    more, as consecutive position blocks do, or none)."""
+    more, as consecutive position blocks do, or none). With `rope`, each
+    softmax warpgroup first rotates its Q tile in place (after Q lands) and
+    the MMA thread waits for that before the tile's first score MMAs."""
     sim = Sim(seed)
     nmax = max(nt)
     sim.bar("q_full", 1)
@@ -147,13 +149,15 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
         sim.bar(f"s_full{t}", 1)
         sim.bar(f"p_full{t}", 1)
         sim.bar(f"o_done{t}", 1)
+        sim.bar(f"q_rot{t}", 1)
     sim.bar("mma_done", 1)
+    qst = {"landed": False, "rotated": set()}
     kst, vst = {}, {}
     s_done, pv_done, sbuf, pbuf = set(), set(), {}, {}
 
     def producer_k():
         if nt[0] or nt[1]:
-            sim.load("q_full", lambda: None)
+            sim.load("q_full", lambda: qst.__setitem__("landed", True))
         for j in range(nmax):
             s = j % KSTAGE
             if j >= KSTAGE:
@@ -180,6 +184,7 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
     def issue_s(t, j):
         def ex():
             check(kst.get(j % KSTAGE) == j, "S reads the wrong K tile", t, j)
+            check(qst["landed"] and (not rope or t in qst["rotated"]), "S reads an unready Q tile", t, j)
             check(pbuf.get(t) is None or (t, pbuf[t]) in pv_done, "S overwrote an unread P", t, j)
             sbuf[t] = j
             s_done.add((t, j))
@@ -202,6 +207,8 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
             yield from sim.wait("k_full0", 0)
             for t in range(2):
                 if nt[t] > 0:
+                    if rope and bug != "no_q_rot_wait":
+                        yield from sim.wait(f"q_rot{t}", 0)
                     issue_s(t, 0)
         for j in range(nmax):
             if bug != "no_v_wait":
@@ -224,6 +231,11 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
         yield from sim.wait("mma_done", 0)
 
     def softmax(t):
+        if rope and nt[t] > 0:
+            yield from sim.wait("q_full", 0)
+            check(qst["landed"], "Q rotated before it landed", t)
+            qst["rotated"].add(t)
+            sim.bars[f"q_rot{t}"].arrive()
         for j in range(nt[t]):
             yield from sim.wait(f"s_full{t}", j & 1)
             check(sbuf.get(t) == j, "softmax reads the wrong S", t, j)

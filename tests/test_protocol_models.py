@@ -16,10 +16,11 @@ def _cases_prefill():
     yield (0, 1)
 
 
-def test_prefill_protocol_hazard_free():
+@pytest.mark.parametrize("rope", [False, True])
+def test_prefill_protocol_hazard_free(rope):
     for nt in _cases_prefill():
         for seed in range(40):
-            pm.prefill(nt, seed, rescale_p=(0.0, 0.3, 1.0)[seed % 3])
+            pm.prefill(nt, seed, rescale_p=(0.0, 0.3, 1.0)[seed % 3], rope=rope)
 
 
 @pytest.mark.parametrize("bug", pm.PREFILL_BUGS)
@@ -27,7 +28,7 @@ def test_prefill_planted_bug_is_caught(bug):
     with pytest.raises(pm.Hazard):
         for nt in _cases_prefill():
             for seed in range(40):
-                pm.prefill(nt, seed, rescale_p=0.5, bug=bug)
+                pm.prefill(nt, seed, rescale_p=0.5, bug=bug, rope=True)
 
 
 def test_mla_protocol_hazard_free():
