@@ -88,6 +88,23 @@ def test_decode_equals_last_prefill_row():
     assert (l_p[:, :, L - 1] - l_d).abs().max() <= 1e-3
 
 
+@pytest.mark.parametrize("L", [2047, 2048, 2049, 4097, 6500])
+def test_decode_independent_of_split_count(L):
+    """The split-KV decode (with 4 query heads per KV head the keys are cut
+    into ceil(L / 2048) chunks: 1, 1, 2, 3 and 4 here, on both sides of a
+    chunk boundary, merged by their log-sum-exp weights) equals the unsplit
+    computation: row L-1 of the causal prefill over the same L tokens."""
+    binding = need_gpu()
+    n_q, n_kv = 32, 8
+    q, k, v = inputs.prefill_inputs(1, L, L, n_q, n_kv, 128, 128, 31 + L, device="cuda")
+    o_p, l_p = binding.attn_fwd(q, k, v, True, 0.08)
+    o_d, l_d = binding.attn_decode(q[:, :, L - 1].contiguous(), k, v,
+                                   torch.tensor([L], dtype=torch.int32, device="cuda"), 0.08)
+    assert binding.device_status() == 0
+    assert (o_p[:, :, L - 1].float() - o_d.float()).abs().max() <= 2e-2
+    assert (l_p[:, :, L - 1] - l_d).abs().max() <= 1e-3
+
+
 def test_decode_zero_length_and_range_status():
     binding = need_gpu()
     B, n_q, n_kv, S_max = 3, 8, 2, 256
