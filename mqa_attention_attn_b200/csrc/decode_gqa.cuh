@@ -104,6 +104,13 @@ template <int GT, bool FP8 = false>
 constexpr size_t smem_bytes() {
     return sizeof(Smem<GT, FP8>) + 1024;  // + alignment slack
 }
+template <bool FP8>
+constexpr bool smem_fits() {   // every head block the launches instantiate
+    return smem_bytes<1, FP8>() <= kMaxSmemPerCta && smem_bytes<2, FP8>() <= kMaxSmemPerCta &&
+           smem_bytes<4, FP8>() <= kMaxSmemPerCta && smem_bytes<8, FP8>() <= kMaxSmemPerCta &&
+           smem_bytes<16, FP8>() <= kMaxSmemPerCta;
+}
+static_assert(smem_fits<false>() && smem_fits<true>(), "decode shared memory exceeds a CTA's");
 
 // FP8 cache scales: element (b, g, j, c) of the cache means
 // e4m3(byte) * k_scale[g] (keys) or * v_scale[g] (values).

@@ -66,6 +66,7 @@ struct Smem {
 };
 
 constexpr size_t smem_bytes() { return sizeof(Smem) + 1024; }
+static_assert(smem_bytes() <= kMaxSmemPerCta, "MLA decode shared memory exceeds a CTA's");
 
 struct Params {
     int B, n_q, S_max;

@@ -121,6 +121,9 @@ constexpr size_t smem_bytes() {
     size_t s = sizeof(Smem<D>) + 1024;
     return s < 118784 ? 118784 : s;
 }
+static_assert(smem_bytes<32>() <= kMaxSmemPerCta && smem_bytes<64>() <= kMaxSmemPerCta &&
+                  smem_bytes<128>() <= kMaxSmemPerCta,
+              "prefill shared memory exceeds a CTA's");
 
 struct Params {
     int B, Sq, Skv, n_q, n_kv, G;

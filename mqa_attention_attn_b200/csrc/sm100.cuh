@@ -28,6 +28,7 @@ __device__ unsigned int g_timeout_site;
 // Upper bound of any single wait inside a kernel. A wait that lasts this
 // long means a lost arrival; the kernel records it and unwinds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr size_t kMaxSmemPerCta = 232448;                    // 227 KB of dynamic shared memory per CTA
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
