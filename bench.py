@@ -7,18 +7,23 @@ One step = one pass of the hot path over synthetic inputs resident in HBM:
     ~U[1024, 32768], 32/8 heads, head dim 128), split-KV + combine;
   * MLA decode: attn_decode on the latent cache (B=64, 4096 rows of 576,
     128 heads, value = first 512 columns).
+The other configurations are timed in a loop of their own after the step:
+the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads) and the tiny
+causal forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency); so are the
+rows built beyond the path (paged, FP8 and RoPE forms), in a third loop.
 `value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
-decode regime is reported in HBM GB/s (algorithmic bytes: the K/V rows below
-each sequence's length, plus q, o and lse) under "regimes". Each kernel is
-timed with CUDA events on its launching stream; L2 (126 MB) is flushed
+decode regimes are reported in HBM GB/s (algorithmic bytes: the K/V rows
+below each sequence's length, plus q, o and lse) under "regimes". Each kernel
+is timed with CUDA events on its launching stream; L2 (126 MB) is flushed
 before every timed launch by writing a 512 MB buffer and then reading a
 256 MB one (so the flush's dirty lines are not written back inside the
 timed launch).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-Multi-GPU: launched by torchrun, one rank per GPU; every rank runs its own
-replica of the workload (independent problems, weak scaling), time is the max
-over ranks, value the sum of all ranks' work over that time.
+Multi-GPU: one rank per GPU (torchrun; `--gpus N` without it starts the N
+ranks itself); every rank runs its own replica of the workload (independent
+problems, weak scaling), time is the max over ranks, value the sum of all
+ranks' work over that time.
 """
 from __future__ import annotations
 
@@ -40,6 +45,12 @@ METRIC = "prefill TFLOP/s & decode HBM GB/s (fraction of B200 peak), 1 GPU"
 HEADLINE = "llama3_8b_prefill"
 DECODE = "gqa_decode"
 MLA = "mla_decode"
+LONG = "llama3_70b_long_prefill"
+TINY = "tiny_prefill"
+# the MLA decode: kernel name, launches per call, key of its per-launch DRAM traffic
+MLA_KERNEL = "attn::mla::mla_decode_kernel (2-CTA cluster)"
+MLA_LAUNCHES = 1
+MLA_TRAFFIC_KEY = "mla_decode_kernel"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -95,7 +106,8 @@ class ClockSampler:
     """SM clocks and throttle reasons sampled during the timed region.
 
     Polls NVML every ~2 ms from a thread (the timed region can be a few
-    milliseconds); falls back to `nvidia-smi -lms 100` if NVML is missing."""
+    milliseconds). Without NVML there is no sample: the summary then reports
+    `samples: 0` and no clock."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
@@ -239,6 +251,47 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 # the CUDA arm
 # ----------------------------------------------------------------------------
+class Regime:
+    """One timed launch sequence of the benchmark: `launch()` enqueues the
+    library call(s) on the bench stream; `launches` is how many of this
+    library's kernels one call runs; `group` is the timed loop it belongs to
+    ("core": the hot-path step; "configs": the other configurations;
+    "next": the rows built beyond the path)."""
+
+    def __init__(self, name, group, launches, launch):
+        self.name, self.group, self.launches, self.launch = name, group, launches, launch
+        self.events = []
+
+    def ms(self):
+        return [a.elapsed_time(b) for a, b in self.events]
+
+    def mean_ms(self):
+        ms = self.ms()
+        return sum(ms) / len(ms) if ms else float("nan")
+
+
+def _oracle_decode_sample(wd, seqlens, qd, kc, vc, n_seq, d_v=None, cache_bytes=None):
+    """The fp64 oracle on the first `n_seq` sequences of a decode workload
+    (every (b, h) row of those, the cache trimmed to their longest length;
+    the tensors may live on the device, only that slice is copied to the
+    host). Returns (seconds, algorithmic bytes of those sequences, threads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    n_seq = min(n_seq, wd.B)
+    sl = seqlens[:n_seq]
+    L = int(sl.max())
+    qx = oracle._f64(qd[:n_seq, :, None, :])
+    kx = oracle._f64(kc[:n_seq, :, :L])
+    vx = kx if vc is kc else oracle._f64(vc[:n_seq, :, :L])
+    t0 = time.perf_counter()
+    oracle.sdpa(qx, kx, vx, False, wd.scale, seqlens=sl.numpy(), d_v=d_v, nthreads=threads)
+    dt = time.perf_counter() - t0
+    rows = float(sl.long().sum())
+    per_row = cache_bytes if cache_bytes is not None else wd.n_kv * (wd.d_qk + wd.d_v) * 2
+    nbytes = rows * per_row + n_seq * wd.n_q * (wd.d_qk * 2 + wd.d_v * 2 + 4)
+    return dt, nbytes, threads
+
+
 def run_ours(args):
     import torch
     ws, rank, local = _dist()
@@ -251,21 +304,10 @@ def run_ours(args):
     from mqa_attention_attn_b200 import binding, build, inputs
     build.build_library()
     binding.lib()
-
-    w = inputs.WORKLOADS[HEADLINE]
-    wd = inputs.WORKLOADS[DECODE]
+    stream = torch.cuda.current_stream(dev)
     gen_seed_shift = 1000 * rank
-    q, k, v = inputs.prefill_inputs(w.B, w.Sq, w.Skv, w.n_q, w.n_kv, w.d_qk, w.d_v, w.seed + gen_seed_shift,
-                                    device=dev)
-    o = torch.empty((w.B, w.n_q, w.Sq, w.d_v), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.B, w.n_q, w.Sq), dtype=torch.float32, device=dev)
-    seqlens, qd, kc, vc = inputs.decode_inputs(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv, wd.seqlen_range,
-                                               wd.seed + gen_seed_shift, device=dev)
-    sl_dev = seqlens.to(dev)
-    od = torch.empty((wd.B, wd.n_q, wd.d_v), dtype=torch.bfloat16, device=dev)
-    ld = torch.empty((wd.B, wd.n_q), dtype=torch.float32, device=dev)
-    wsz = binding.decode_workspace_bytes(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv)
-    work = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    sel = lambda *names: args.only == "all" or args.only in names
+
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     flush_rd = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
@@ -276,58 +318,101 @@ def run_ours(args):
         being written back while it runs."""
         flush.fill_(val)
         torch.sum(flush_rd, dim=0, out=flush_sum)
+
+    regimes = {}
+
+    def add(name, group, launches, fn):
+        regimes[name] = Regime(name, group, launches, fn)
+
+    # ---- the hot-path step: prefill (headline), GQA decode, MLA decode
+    w = inputs.WORKLOADS[HEADLINE]
+    wd = inputs.WORKLOADS[DECODE]
     wm = inputs.WORKLOADS[MLA]
+    q, k, v = inputs.prefill_inputs(w.B, w.Sq, w.Skv, w.n_q, w.n_kv, w.d_qk, w.d_v, w.seed + gen_seed_shift,
+                                    device=dev)
+    o = torch.empty((w.B, w.n_q, w.Sq, w.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.n_q, w.Sq), dtype=torch.float32, device=dev)
+    fl_p, by_p = prefill_flops(w), prefill_bytes(w)
+    if sel("prefill"):
+        add("prefill", "core", 1, lambda: binding.attn_fwd(q, k, v, w.causal, w.scale, o=o, lse=lse, stream=stream))
+
+    seqlens, qd, kc, vc = inputs.decode_inputs(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv, wd.seqlen_range,
+                                               wd.seed + gen_seed_shift, device=dev)
+    sl_dev = seqlens.to(dev)
+    od = torch.empty((wd.B, wd.n_q, wd.d_v), dtype=torch.bfloat16, device=dev)
+    ld = torch.empty((wd.B, wd.n_q), dtype=torch.float32, device=dev)
+    work = torch.empty(binding.decode_workspace_bytes(wd.B, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, wd.Skv),
+                       dtype=torch.uint8, device=dev)
+    by_d, fl_d = decode_bytes(wd, seqlens), decode_flops(wd, seqlens)
+    if sel("decode"):
+        add("decode", "core", 2, lambda: binding.attn_decode(qd, kc, vc, sl_dev, wd.scale, o=od, lse=ld,
+                                                             workspace=work, stream=stream))
+
     slm, qm, cm = inputs.mla_inputs(wm.B, wm.n_q, wm.d_qk, wm.Skv, wm.seqlen_range, wm.seed + gen_seed_shift,
                                     device=dev)
     cm4 = cm[:, None]
     slm_dev = slm.to(dev)
     om = torch.empty((wm.B, wm.n_q, wm.d_v), dtype=torch.bfloat16, device=dev)
     lm = torch.empty((wm.B, wm.n_q), dtype=torch.float32, device=dev)
-    by_m = mla_bytes(wm, slm)
-    fl_m = decode_flops(wm, slm)
+    by_m, fl_m = mla_bytes(wm, slm), decode_flops(wm, slm)
+    mla_ws_n = binding.decode_workspace_bytes(wm.B, wm.n_q, wm.n_kv, wm.d_qk, wm.d_v, wm.Skv)
+    work_m = torch.empty(max(mla_ws_n, 1), dtype=torch.uint8, device=dev)
+    if sel("mla"):
+        add("mla_decode", "core", MLA_LAUNCHES, lambda: binding.attn_decode(
+            qm, cm4, cm4, slm_dev, wm.scale, d_v=wm.d_v, o=om, lse=lm, workspace=work_m, stream=stream))
 
-    stream = torch.cuda.current_stream(dev)
-    fl_p = prefill_flops(w)
-    by_p = prefill_bytes(w)
-    by_d = decode_bytes(wd, seqlens)
-    fl_d = decode_flops(wd, seqlens)
+    # ---- the other configurations: the 70B-shaped long prefill and the tiny one
+    if sel("long"):
+        wl = inputs.WORKLOADS[LONG]
+        ql, kl, vl = inputs.prefill_inputs(wl.B, wl.Sq, wl.Skv, wl.n_q, wl.n_kv, wl.d_qk, wl.d_v,
+                                           wl.seed + gen_seed_shift, device=dev)
+        ol = torch.empty((wl.B, wl.n_q, wl.Sq, wl.d_v), dtype=torch.bfloat16, device=dev)
+        lsel = torch.empty((wl.B, wl.n_q, wl.Sq), dtype=torch.float32, device=dev)
+        add("long_prefill", "configs", 1,
+            lambda: binding.attn_fwd(ql, kl, vl, wl.causal, wl.scale, o=ol, lse=lsel, stream=stream))
+    if sel("tiny"):
+        wt = inputs.WORKLOADS[TINY]
+        qt, kt, vt = inputs.prefill_inputs(wt.B, wt.Sq, wt.Skv, wt.n_q, wt.n_kv, wt.d_qk, wt.d_v,
+                                           wt.seed + gen_seed_shift, device=dev)
+        ot = torch.empty((wt.B, wt.n_q, wt.Sq, wt.d_v), dtype=torch.bfloat16, device=dev)
+        lset = torch.empty((wt.B, wt.n_q, wt.Sq), dtype=torch.float32, device=dev)
+        add("tiny_prefill", "configs", 1,
+            lambda: binding.attn_fwd(qt, kt, vt, wt.causal, wt.scale, o=ot, lse=lset, stream=stream))
 
-    do_p = args.only in ("all", "prefill")
-    do_d = args.only in ("all", "decode")
-    do_m = args.only in ("all", "mla")
-    do_g = args.only in ("all", "paged")
-    do_f = args.only in ("all", "fp8")
-    do_r = args.only in ("all", "rope")
-
-    # rotary position embedding on the prefill and decode workloads (tables
-    # for the Llama-3 base 500000): prefill takes q, k unrotated, decode a
-    # cache that holds rotated keys
+    # ---- the rows built beyond the path, on the same workloads
+    # rotary position embedding (Llama-3 base 500000): prefill takes q, k
+    # unrotated, decode a cache that holds rotated keys
     ROPE_BASE = 500000.0
-    if do_r:
+    if sel("rope"):
         cos_p, sin_p = binding.rope_tables(w.Skv, w.d_qk, ROPE_BASE, device=dev)
         cos_d, sin_d = binding.rope_tables(wd.Skv, wd.d_qk, ROPE_BASE, device=dev)
         k_rot = torch.empty_like(k)
         o_r, lse_r = torch.empty_like(o), torch.empty_like(lse)
         od_r, ld_r = torch.empty_like(od), torch.empty_like(ld)
+        add("rope_prefill", "next", 2, lambda: binding.attn_fwd_rope(
+            q, k, v, w.causal, w.scale, cos_p, sin_p, k_rot=k_rot, o=o_r, lse=lse_r, stream=stream))
+        add("rope_decode", "next", 2, lambda: binding.attn_decode_rope(
+            qd, kc, vc, sl_dev, wd.scale, cos_d, sin_d, o=od_r, lse=ld_r, workspace=work, stream=stream))
 
     # the GQA decode workload with its cache in e4m3, one scale per KV head
-    if do_f:
+    if sel("fp8"):
         def to_e4m3(x):
             amax = x.float().abs().amax(dim=(0, 2, 3)).clamp_min(1e-6)
             sc = (amax / 448.0).float()
             return (x.float() / sc[None, :, None, None]).to(torch.float8_e4m3fn), sc.contiguous()
         k8, ks8 = to_e4m3(kc)
         v8, vs8 = to_e4m3(vc)
-        of8 = torch.empty_like(od)
-        lf8 = torch.empty_like(ld)
+        of8, lf8 = torch.empty_like(od), torch.empty_like(ld)
         work8 = torch.empty(binding.decode_fp8_workspace_bytes(wd.B, wd.n_q, wd.n_kv, wd.Skv), dtype=torch.uint8,
                             device=dev)
         by_f = decode_bytes(wd, seqlens, cache_elem_bytes=1)
+        add("fp8_decode", "next", 2, lambda: binding.attn_decode_fp8(
+            qd, k8, v8, ks8, vs8, sl_dev, wd.scale, o=of8, lse=lf8, workspace=work8, stream=stream))
 
     # the GQA decode workload again, its cache cut into 64-token pages placed
     # in a pool in a seeded random order (the paged-cache serving layout)
     PAGE = 64
-    if do_g:
+    if sel("paged"):
         P = wd.Skv // PAGE
         npg = (seqlens.long() + PAGE - 1) // PAGE
         b_idx = torch.repeat_interleave(torch.arange(wd.B), npg)
@@ -344,74 +429,9 @@ def run_ours(args):
         pool_k[pid_dev] = kview[b_dev, p_dev]
         pool_v[pid_dev] = vview[b_dev, p_dev]
         del pid_dev, b_dev, p_dev
-        og = torch.empty_like(od)
-        lg = torch.empty_like(ld)
-
-    # One step of the hot path = prefill, GQA decode, MLA decode (`core`); the
-    # regimes of the rows built beyond it (paged, FP8, RoPE: `nxt`) are timed
-    # in a loop of their own after it, so that they do not disturb the
-    # headline numbers.
-    def step(times_p, times_d, times_m=None, times_g=None, times_f=None, times_rp=None, times_rd=None,
-             core=True, nxt=True):
-        if do_p and core:
-            cold_l2(1.0)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            binding.attn_fwd(q, k, v, w.causal, w.scale, o=o, lse=lse, stream=stream)
-            e1.record(stream)
-            if times_p is not None:
-                times_p.append((e0, e1))
-        if do_d and core:
-            cold_l2(2.0)
-            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e2.record(stream)
-            binding.attn_decode(qd, kc, vc, sl_dev, wd.scale, o=od, lse=ld, workspace=work, stream=stream)
-            e3.record(stream)
-            if times_d is not None:
-                times_d.append((e2, e3))
-        if do_m and core:
-            cold_l2(3.0)
-            e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e4.record(stream)
-            binding.attn_decode(qm, cm4, cm4, slm_dev, wm.scale, d_v=wm.d_v, o=om, lse=lm, stream=stream)
-            e5.record(stream)
-            if times_m is not None:
-                times_m.append((e4, e5))
-        if do_g and nxt:
-            cold_l2(4.0)
-            e6, e7 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e6.record(stream)
-            binding.attn_decode_paged(qd, pool_k, pool_v, table_dev, sl_dev, wd.scale, o=og, lse=lg,
-                                      workspace=work, stream=stream)
-            e7.record(stream)
-            if times_g is not None:
-                times_g.append((e6, e7))
-        if do_f and nxt:
-            cold_l2(5.0)
-            e8, e9 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e8.record(stream)
-            binding.attn_decode_fp8(qd, k8, v8, ks8, vs8, sl_dev, wd.scale, o=of8, lse=lf8, workspace=work8,
-                                    stream=stream)
-            e9.record(stream)
-            if times_f is not None:
-                times_f.append((e8, e9))
-        if do_r and nxt:
-            cold_l2(6.0)
-            e10, e11 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e10.record(stream)
-            binding.attn_fwd_rope(q, k, v, w.causal, w.scale, cos_p, sin_p, k_rot=k_rot, o=o_r, lse=lse_r,
-                                  stream=stream)
-            e11.record(stream)
-            if times_rp is not None:
-                times_rp.append((e10, e11))
-            cold_l2(7.0)
-            e12, e13 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e12.record(stream)
-            binding.attn_decode_rope(qd, kc, vc, sl_dev, wd.scale, cos_d, sin_d, o=od_r, lse=ld_r, workspace=work,
-                                     stream=stream)
-            e13.record(stream)
-            if times_rd is not None:
-                times_rd.append((e12, e13))
+        og, lg = torch.empty_like(od), torch.empty_like(ld)
+        add("paged_decode", "next", 2, lambda: binding.attn_decode_paged(
+            qd, pool_k, pool_v, table_dev, sl_dev, wd.scale, o=og, lse=lg, workspace=work, stream=stream))
 
     def barrier():
         if ws > 1:
@@ -419,42 +439,39 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    tp, td, tm, tg, tf, trp, trd = [], [], [], [], [], [], []
+    # Each group is warmed up and timed in a loop of its own, so that the
+    # configurations and rows beyond the step do not disturb the headline.
+    # Every timed launch follows an L2 flush and has its own events.
     t_wall = 0.0
     with ClockSampler(torch.cuda.current_device()) as clocks:
-        for core, nxt in ((True, False), (False, True)):
-            if not ((core and (do_p or do_d or do_m)) or (nxt and (do_g or do_f or do_r))):
+        for group in ("core", "configs", "next"):
+            rs = [r for r in regimes.values() if r.group == group]
+            if not rs:
                 continue
+
+            def one_step(timed):
+                for i, r in enumerate(rs):
+                    cold_l2(float(i + 1))
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    r.launch()
+                    e1.record(stream)
+                    if timed:
+                        r.events.append((e0, e1))
+
             for _ in range(max(3, args.warmup)):
-                step(None, None, core=core, nxt=nxt)
+                one_step(False)
             barrier()
             assert binding.device_status(stream) == 0, "device status not clean after warm-up"
             t_wall0 = time.perf_counter()
             for _ in range(args.steps):
-                step(tp, td, tm, tg, tf, trp, trd, core=core, nxt=nxt)
+                one_step(True)
             barrier()
             t_wall += time.perf_counter() - t_wall0
     st = binding.device_status(stream)
     assert st == 0, f"device status {st}"
-    ms_p = [a.elapsed_time(b) for a, b in tp] or [float("nan")]
-    ms_d = [a.elapsed_time(b) for a, b in td] or [float("nan")]
-    ms_m = [a.elapsed_time(b) for a, b in tm] or [float("nan")]
-    ms_g = [a.elapsed_time(b) for a, b in tg] or [float("nan")]
-    mean_g = sum(ms_g) / len(ms_g)
-    ms_f = [a.elapsed_time(b) for a, b in tf] or [float("nan")]
-    mean_f = sum(ms_f) / len(ms_f)
-    mean_m = sum(ms_m) / len(ms_m)
-    mean_p = sum(ms_p) / len(ms_p)
-    mean_d = sum(ms_d) / len(ms_d)
-    ms_rp = [a.elapsed_time(b) for a, b in trp] or [float("nan")]
-    ms_rd = [a.elapsed_time(b) for a, b in trd] or [float("nan")]
-    mean_rp = sum(ms_rp) / len(ms_rp)
-    mean_rd = sum(ms_rd) / len(ms_rd)
-
-    agg_p = aggregate({"time_s": sum(ms_p) / 1e3, "work": fl_p * args.steps}, ws)
-    agg_d = aggregate({"time_s": sum(ms_d) / 1e3, "work": by_d * args.steps}, ws)
-    value = agg_p["work"] / agg_p["time_s"] / 1e12
-    dec_gbs = agg_d["work"] / agg_d["time_s"] / 1e9
+    mean = {n: r.mean_ms() for n, r in regimes.items()}
+    nan = float("nan")
 
     # ---- end to end through the public API with host buffers: every step
     # copies its q, k, v from pinned host memory and reads O and LSE back.
@@ -462,7 +479,7 @@ def run_ours(args):
     # (host-to-device copies of step i+1 and the device-to-host read of step
     # i-1 overlap the attention of step i), the way a serving loop would run.
     e2e = None
-    if not args.no_e2e and do_p:
+    if not args.no_e2e and "prefill" in regimes:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         NB = 2
         dev_in = [tuple(torch.empty_like(t) for t in (q, k, v)) for _ in range(NB)]
@@ -521,93 +538,162 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_bw = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    achieved_tf = fl_p / (mean_p / 1e3) / 1e12
     traffic = load_traffic()
-    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_tf, "traffic": traffic.get("prefill_kernel_128"),
-                "kernel": "attn::pf::prefill_kernel<128>", "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "algorithmic_flops_per_launch": fl_p}
-    dec_achieved = by_d / (mean_d / 1e3) / 1e9
-    regimes = {
-        "prefill": {"workload": w.name, "ms": mean_p, "tflops": achieved_tf,
-                    "frac_of_peak": achieved_tf / peak_tf, "frac_of_nominal_2250": achieved_tf / 2250.0,
-                    "algorithmic_flops": fl_p, "algorithmic_bytes": by_p},
-        "decode": {"workload": wd.name, "ms": mean_d, "gbs": dec_achieved, "aggregate_gbs": dec_gbs,
-                   "frac_of_peak": dec_achieved / peak_bw, "frac_of_nominal_8000": dec_achieved / 8000.0,
-                   "algorithmic_bytes": by_d, "algorithmic_flops": fl_d,
-                   "kernels": "attn::dec::decode_split_kernel<4> + decode_combine_kernel",
-                   "peak": peak_bw, "peak_source": f"{peak_src} hbm_gbs",
-                   "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak_bw, "unit": "GB/s",
-                                "frac": dec_achieved / peak_bw, "traffic": traffic.get("decode_split_kernel_4"),
-                                "note": "achieved over split + merge launches; traffic of the split kernel"}},
-        "mla_decode": {"workload": wm.name, "ms": mean_m, "gbs": by_m / (mean_m / 1e3) / 1e9,
-                       "tflops": fl_m / (mean_m / 1e3) / 1e12,
-                       "frac_of_peak_hbm": by_m / (mean_m / 1e3) / 1e9 / peak_bw,
-                       "roofline_frac": max(by_m / (peak_bw * 1e9), fl_m / (peak_tf * 1e12)) / (mean_m / 1e3),
-                       "algorithmic_bytes": by_m, "algorithmic_flops": fl_m,
-                       "kernel": "attn::mla::mla_decode_kernel (2-CTA cluster)",
-                       "roofline": {"bound": "hbm", "achieved": by_m / (mean_m / 1e3) / 1e9, "peak": peak_bw,
-                                    "unit": "GB/s", "frac": by_m / (mean_m / 1e3) / 1e9 / peak_bw,
-                                    "traffic": traffic.get("mla_decode_kernel"),
-                                    "tensor_frac": fl_m / (mean_m / 1e3) / 1e12 / peak_tf}},
-        "paged_decode": {"workload": f"{wd.name}, {PAGE}-token pages in a shuffled pool", "ms": mean_g,
-                         "gbs": by_d / (mean_g / 1e3) / 1e9, "frac_of_peak": by_d / (mean_g / 1e3) / 1e9 / peak_bw,
-                         "algorithmic_bytes": by_d,
-                         "kernels": "attn::dec::decode_split_kernel<4, paged> + decode_combine_kernel"},
-        "fp8_decode": {"workload": f"{wd.name}, e4m3 cache with one scale per KV head", "ms": mean_f,
-                       "gbs": (by_f / (mean_f / 1e3) / 1e9) if do_f else None,
-                       "frac_of_peak": (by_f / (mean_f / 1e3) / 1e9 / peak_bw) if do_f else None,
-                       "speedup_vs_bf16_cache": (mean_d / mean_f) if (do_f and do_d) else None,
-                       "algorithmic_bytes": by_f if do_f else None,
-                       "kernels": "attn::dec::decode_split_kernel<4, fp8> + decode_combine_kernel",
-                       "roofline": ({"bound": "hbm", "achieved": by_f / (mean_f / 1e3) / 1e9, "peak": peak_bw,
-                                     "unit": "GB/s", "frac": by_f / (mean_f / 1e3) / 1e9 / peak_bw,
-                                     "traffic": traffic.get("decode_split_kernel_4_fp8"),
-                                     "note": "achieved over split + merge launches; traffic of the split kernel"}
-                                    if do_f else None)},
-        "rope_prefill": {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": mean_rp,
-                         "tflops": (fl_p / (mean_rp / 1e3) / 1e12) if do_r else None,
-                         "frac_of_peak": (fl_p / (mean_rp / 1e3) / 1e12 / peak_tf) if do_r else None,
-                         "overhead_vs_attn_fwd": (mean_rp / mean_p - 1.0) if (do_r and do_p) else None,
-                         "kernels": "attn::rope::rope_apply_kernel (keys, once) + attn::pf::prefill_kernel<128, rope> "
-                                    "(queries rotated in shared memory)",
-                         "roofline": ({"bound": "tensor", "achieved": fl_p / (mean_rp / 1e3) / 1e12, "peak": peak_tf,
-                                       "unit": "TFLOP/s", "frac": fl_p / (mean_rp / 1e3) / 1e12 / peak_tf,
-                                       "traffic": traffic.get("prefill_kernel_128_rope"),
-                                       "note": "achieved over both launches; traffic of the attention kernel"}
-                                      if do_r else None)},
-        "rope_decode": {"workload": f"{wd.name}, query rotated at seqlen - 1, cache of rotated keys",
-                        "ms": mean_rd, "gbs": (by_d / (mean_rd / 1e3) / 1e9) if do_r else None,
-                        "frac_of_peak": (by_d / (mean_rd / 1e3) / 1e9 / peak_bw) if do_r else None,
-                        "kernels": "attn::dec::decode_split_kernel<4> (query rotated in the MMA warp) + "
-                                   "decode_combine_kernel"},
-    }
 
-    cpu_baseline = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline and do_p:
-        qc, kc_, vc_ = q.cpu(), k.cpu(), v.cpu()
-        dt, fl, threads = oracle_full(w, qc, kc_, vc_)
-        cpu_baseline = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                        "sample": f"the whole {w.name} workload, all {w.B * w.n_q * w.Sq} query rows "
-                                  f"(fp64 plain definition, OpenMP over rows), {dt:.1f} s"}
+    def tf(flops, ms):
+        return flops / (ms / 1e3) / 1e12
+
+    def gbs(nbytes, ms):
+        return nbytes / (ms / 1e3) / 1e9
+
+    def tensor_roofline(flops, ms, kernel, traffic_key, note=None):
+        a = tf(flops, ms)
+        r = {"bound": "tensor", "achieved": a, "peak": peak_tf, "unit": "TFLOP/s", "frac": a / peak_tf,
+             "traffic": traffic.get(traffic_key), "kernel": kernel,
+             "peak_source": f"{peak_src} bf16_tflops (burst)", "algorithmic_flops_per_launch": flops}
+        if note:
+            r["note"] = note
+        return r
+
+    def hbm_roofline(nbytes, ms, kernel, traffic_key, note=None):
+        a = gbs(nbytes, ms)
+        r = {"bound": "hbm", "achieved": a, "peak": peak_bw, "unit": "GB/s", "frac": a / peak_bw,
+             "traffic": traffic.get(traffic_key), "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs",
+             "algorithmic_bytes_per_launch": nbytes}
+        if note:
+            r["note"] = note
+        return r
+
+    # ---- the oracle on the host cores, per regime (rank 0 of a 1-GPU run only)
+    do_cpu = rank == 0 and ws == 1 and not args.no_cpu_baseline
+    cpu = {}
+    if do_cpu and "prefill" in regimes:
+        dt, fl, threads = oracle_full(w, q.cpu(), k.cpu(), v.cpu())
+        cpu["prefill"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                          "sample": f"the whole {w.name} workload, all {w.B * w.n_q * w.Sq} query rows "
+                                    f"(fp64 plain definition, OpenMP over rows), {dt:.1f} s"}
+    if do_cpu and "decode" in regimes:
+        n_seq = 8
+        dt, nb, threads = _oracle_decode_sample(wd, seqlens, qd, kc, vc, n_seq)
+        cpu["decode"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"the first {n_seq} of the {wd.B} sequences of {wd.name}, every (b, h) row, "
+                                   f"{nb / 1e9:.2f} GB of algorithmic bytes in {dt:.1f} s"}
+    if do_cpu and "mla_decode" in regimes:
+        n_seq = 16
+        dt, nb, threads = _oracle_decode_sample(wm, slm, qm, cm4, cm4, n_seq, d_v=wm.d_v,
+                                                cache_bytes=wm.d_qk * 2)
+        cpu["mla_decode"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"the first {n_seq} of the {wm.B} sequences of {wm.name}, every (b, h) "
+                                       f"row, {nb / 1e6:.0f} MB of algorithmic bytes in {dt:.1f} s"}
+    if do_cpu and "long_prefill" in regimes:
+        n_rows = 2048
+        dt, fl, threads = oracle_sample(wl, ql.cpu(), kl.cpu(), vl.cpu(), n_rows, 4242)
+        rate = fl / dt
+        cpu["long_prefill"] = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                               "sample": f"{n_rows} seeded query rows of {wl.name} ({dt:.1f} s); the whole "
+                                         f"workload extrapolated at that rate: {prefill_flops(wl) / rate:.0f} s",
+                               "extrapolated": True}
+
+    # ---- the JSON line
+    ms_p, ms_d, ms_m = mean.get("prefill", nan), mean.get("decode", nan), mean.get("mla_decode", nan)
+    value = nan
+    if "prefill" in regimes:
+        agg_p = aggregate({"time_s": sum(regimes["prefill"].ms()) / 1e3, "work": fl_p * args.steps}, ws)
+        value = agg_p["work"] / agg_p["time_s"] / 1e12
+    out = {}
+    if "prefill" in regimes:
+        out["prefill"] = {"workload": w.name, "ms": ms_p, "tflops": tf(fl_p, ms_p),
+                          "frac_of_peak": tf(fl_p, ms_p) / peak_tf, "frac_of_nominal_2250": tf(fl_p, ms_p) / 2250.0,
+                          "algorithmic_flops": fl_p, "algorithmic_bytes": by_p, "cpu_baseline": cpu.get("prefill")}
+    if "decode" in regimes:
+        agg_d = aggregate({"time_s": sum(regimes["decode"].ms()) / 1e3, "work": by_d * args.steps}, ws)
+        out["decode"] = {"workload": wd.name, "ms": ms_d, "gbs": gbs(by_d, ms_d),
+                         "aggregate_gbs": agg_d["work"] / agg_d["time_s"] / 1e9,
+                         "frac_of_peak": gbs(by_d, ms_d) / peak_bw, "frac_of_nominal_8000": gbs(by_d, ms_d) / 8000.0,
+                         "algorithmic_bytes": by_d, "algorithmic_flops": fl_d,
+                         "kernels": "attn::dec::decode_split_kernel<4> + decode_combine_kernel",
+                         "roofline": hbm_roofline(by_d, ms_d, "attn::dec::decode_split_kernel<4>",
+                                                  "decode_split_kernel_4",
+                                                  "achieved over split + merge launches; traffic of the split kernel"),
+                         "cpu_baseline": cpu.get("decode")}
+    if "mla_decode" in regimes:
+        t_hbm, t_tc = by_m / (peak_bw * 1e9), fl_m / (peak_tf * 1e12)
+        out["mla_decode"] = {"workload": wm.name, "ms": ms_m, "gbs": gbs(by_m, ms_m), "tflops": tf(fl_m, ms_m),
+                             "frac_of_peak_hbm": gbs(by_m, ms_m) / peak_bw,
+                             "roofline_frac": max(t_hbm, t_tc) / (ms_m / 1e3),
+                             "algorithmic_bytes": by_m, "algorithmic_flops": fl_m, "kernel": MLA_KERNEL,
+                             "roofline": dict(hbm_roofline(by_m, ms_m, MLA_KERNEL, MLA_TRAFFIC_KEY),
+                                              tensor_frac=tf(fl_m, ms_m) / peak_tf),
+                             "cpu_baseline": cpu.get("mla_decode")}
+    if "long_prefill" in regimes:
+        ms_l = mean["long_prefill"]
+        fl_l = prefill_flops(wl)
+        out["long_prefill"] = {"workload": wl.name, "ms": ms_l, "tflops": tf(fl_l, ms_l),
+                               "frac_of_peak": tf(fl_l, ms_l) / peak_tf,
+                               "frac_of_nominal_2250": tf(fl_l, ms_l) / 2250.0,
+                               "algorithmic_flops": fl_l, "algorithmic_bytes": prefill_bytes(wl),
+                               "roofline": tensor_roofline(fl_l, ms_l, "attn::pf::prefill_kernel<128>",
+                                                           "prefill_kernel_128_long"),
+                               "cpu_baseline": cpu.get("long_prefill")}
+    if "tiny_prefill" in regimes:
+        ms_t = mean["tiny_prefill"]
+        fl_t = prefill_flops(wt)
+        lat = sorted(regimes["tiny_prefill"].ms())
+        out["tiny_prefill"] = {"workload": wt.name, "ms": ms_t, "latency_us": 1e3 * ms_t,
+                               "latency_us_median": 1e3 * lat[len(lat) // 2], "tflops": tf(fl_t, ms_t),
+                               "algorithmic_flops": fl_t, "bound": "launch latency (one CTA, one key tile)"}
+    if "paged_decode" in regimes:
+        ms_g = mean["paged_decode"]
+        out["paged_decode"] = {"workload": f"{wd.name}, {PAGE}-token pages in a shuffled pool", "ms": ms_g,
+                               "gbs": gbs(by_d, ms_g), "frac_of_peak": gbs(by_d, ms_g) / peak_bw,
+                               "algorithmic_bytes": by_d,
+                               "kernels": "attn::dec::decode_split_kernel<4, paged> + decode_combine_kernel"}
+    if "fp8_decode" in regimes:
+        ms_f = mean["fp8_decode"]
+        out["fp8_decode"] = {"workload": f"{wd.name}, e4m3 cache with one scale per KV head", "ms": ms_f,
+                             "gbs": gbs(by_f, ms_f), "frac_of_peak": gbs(by_f, ms_f) / peak_bw,
+                             "speedup_vs_bf16_cache": (ms_d / ms_f) if "decode" in regimes else None,
+                             "algorithmic_bytes": by_f,
+                             "kernels": "attn::dec::decode_split_kernel<4, fp8> + decode_combine_kernel",
+                             "roofline": hbm_roofline(by_f, ms_f, "attn::dec::decode_split_kernel<4, fp8>",
+                                                      "decode_split_kernel_4_fp8",
+                                                      "achieved over split + merge launches; traffic of the "
+                                                      "split kernel")}
+    if "rope_prefill" in regimes:
+        ms_rp, ms_rd = mean["rope_prefill"], mean["rope_decode"]
+        out["rope_prefill"] = {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": ms_rp,
+                               "tflops": tf(fl_p, ms_rp), "frac_of_peak": tf(fl_p, ms_rp) / peak_tf,
+                               "overhead_vs_attn_fwd": (ms_rp / ms_p - 1.0) if "prefill" in regimes else None,
+                               "kernels": "attn::rope::rope_apply_kernel (keys, once) + "
+                                          "attn::pf::prefill_kernel<128, rope> (queries rotated in shared memory)",
+                               "roofline": tensor_roofline(fl_p, ms_rp, "attn::pf::prefill_kernel<128, rope>",
+                                                           "prefill_kernel_128_rope",
+                                                           "achieved over both launches; traffic of the attention "
+                                                           "kernel")}
+        out["rope_decode"] = {"workload": f"{wd.name}, query rotated at seqlen - 1, cache of rotated keys",
+                              "ms": ms_rd, "gbs": gbs(by_d, ms_rd), "frac_of_peak": gbs(by_d, ms_rd) / peak_bw,
+                              "kernels": "attn::dec::decode_split_kernel<4> (query rotated in the MMA warp) + "
+                                         "decode_combine_kernel"}
 
     if rank == 0:
+        roofline = (tensor_roofline(fl_p, ms_p, "attn::pf::prefill_kernel<128>", "prefill_kernel_128")
+                    if "prefill" in regimes else None)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": sum(x for x in (mean_p, mean_d, mean_m) if x == x),
+            "warmup": args.warmup, "ms_per_step": sum(x for x in (ms_p, ms_d, ms_m) if x == x),
             "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "S": w.Sq, "n_q": w.n_q, "n_kv": w.n_kv, "d": w.d_qk,
-                       "causal": w.causal, "decode_workload": wd.name,
+                       "causal": w.causal, "decode_workload": wd.name, "mla_workload": wm.name,
                        "l2": "flushed before every timed launch (512 MB write, then 256 MB read)",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
             "roofline": roofline,
-            "regimes": regimes,
-            "cpu_baseline": cpu_baseline,
+            "regimes": out,
+            "cpu_baseline": cpu.get("prefill"),
             "e2e": e2e,
             "clocks": clocks.summary(),
-            "gpu_launches": (int(do_p) + 2 * int(do_d) + int(do_m) + 2 * int(do_g) + 2 * int(do_f) + 4 * int(do_r)) *
-                            args.steps,
+            "gpu_launches": sum(r.launches * len(r.events) for r in regimes.values()) +
+                            (args.steps if e2e is not None else 0),
             "wall_s_timed_region": t_wall,
         }
         print(json.dumps(line), flush=True)
@@ -626,6 +712,20 @@ def load_traffic():
     return {}
 
 
+def relaunch_ranks(args) -> int:
+    """`--gpus N` (N > 1) outside a distributed launch: start N ranks on this
+    node with torch.distributed.run (one process per GPU, rendezvous on
+    127.0.0.1) running this same command, and return their exit status."""
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -636,9 +736,19 @@ def main():
                     help="query rows of the headline workload per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "mla", "paged", "fp8", "rope"],
+    ap.add_argument("--only", default="all",
+                    choices=["all", "prefill", "decode", "mla", "long", "tiny", "paged", "fp8", "rope"],
                     help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" in os.environ:
+        ws = int(os.environ["WORLD_SIZE"])
+        if ws != args.gpus:
+            print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}: launch one rank per GPU", file=sys.stderr)
+            return 2
+    elif args.gpus > 1:
+        return relaunch_ranks(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -40,7 +40,21 @@ def test_reference_arm_json_line():
 def test_reference_arm_other_ranks_do_no_work():
     """Under a multi-rank launch only rank 0 runs the oracle and prints."""
     env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2")
-    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                          "--warmup", "0"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env, capture_output=True, text=True,
+                         timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert not [l for l in out.stdout.splitlines() if l.startswith("{")]
+
+
+def test_gpus_must_match_the_launched_world_size():
+    """Under a distributed launch --gpus N must equal WORLD_SIZE, so that the
+    line's n_gpus is the number of ranks that did the work (both arms)."""
+    env = dict(os.environ, RANK="0", LOCAL_RANK="0", WORLD_SIZE="2")
+    for impl in ("reference", "ours"):
+        out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", impl, "--gpus", "4",
+                              "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env, capture_output=True, text=True,
+                             timeout=300)
+        assert out.returncode == 2, (impl, out.returncode, out.stderr[-2000:])
+        assert "WORLD_SIZE=2" in out.stderr
+        assert not [l for l in out.stdout.splitlines() if l.startswith("{")]
