@@ -283,6 +283,10 @@ int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, c
  * The first call on a device looks up that device's address of the scratch
  * array (cudaGetSymbolAddress); make that first call before any stream
  * capture on the device. Nothing is allocated or freed, then or later.
+ * The address is kept per device together with the CUDA context it belongs
+ * to; after a cudaDeviceReset (a new primary context, in which the library's
+ * module and the array are loaded again) the next call looks it up anew, so
+ * that first call after a reset should also come before any capture.
  * All calls share the one array and it keeps the previous call's contents;
  * no part of it needs to start at zero (every value read is written earlier
  * in the same call). Calls that overlap on the GPU (on different streams, or
@@ -371,6 +375,12 @@ const char *attn_status_string(int status);
  * word of the current device. Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a
  * kernel's bounded wait expired; its outputs are invalid), ATTN_ERR_DEVICE_RANGE,
  * or ATTN_ERR_CUDA if the synchronisation itself failed.
+ * The status word is one per DEVICE, not per stream: it collects the errors of
+ * every kernel of this library on the device, whatever stream launched it,
+ * and only `stream` is synchronised first. With work in flight on other
+ * streams, an error of one of their kernels may be reported to (and cleared
+ * by) this call, or land after it; callers that need per-stream attribution
+ * must synchronise those streams too before calling.
  */
 int attn_device_status(attn_stream_t stream);
 

@@ -5,6 +5,7 @@
 // workspace) belongs to the caller. Validation errors return before any
 // launch; device-side errors land in the status word that
 // attn_device_status() reads.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -68,12 +69,14 @@ bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
+// `done_mask` holds one bit per device; threads that race on the first call
+// of a device both set the (same) attributes, which is harmless.
 template <typename K>
-bool ensure_smem_attr(K kernel, size_t bytes, uint64_t &done_mask) {
+bool ensure_smem_attr(K kernel, size_t bytes, std::atomic<uint64_t> &done_mask) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     const uint64_t bit = 1ull << (dev & 63);
-    if (done_mask & bit) return true;
+    if (done_mask.load(std::memory_order_acquire) & bit) return true;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
     // all of the unified L1 / shared storage as shared memory, so that the
@@ -81,22 +84,23 @@ bool ensure_smem_attr(K kernel, size_t bytes, uint64_t &done_mask) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return false;
-    done_mask |= bit;
+    done_mask.fetch_or(bit, std::memory_order_acq_rel);
     return true;
 }
 inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
-// Number of SMs of the current device (cached per device).
+// Number of SMs of the current device (cached per device; safe to call from
+// several host threads).
 int sm_count() {
-    static int counts[64] = {};
+    static std::atomic<int> counts[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-    if (counts[dev] == 0) {
-        int n = 0;
+    int n = counts[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-        counts[dev] = n;
+        counts[dev].store(n, std::memory_order_relaxed);
     }
-    return counts[dev];
+    return n;
 }
 
 // ---------------------------------------------------------------------------
@@ -179,27 +183,28 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         }
     }
     const size_t smem = attn::pf::smem_bytes<D>();
-    static uint64_t attr_done = 0;  // per template instance, one bit per device
+    static std::atomic<uint64_t> attr_done{0};  // per template instance, one bit per device
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kDense>, smem, attr_done)) return ATTN_ERR_CUDA;
-    static uint64_t attr_done_v = 0, attr_done_w = 0, attr_done_r = 0;
+    static std::atomic<uint64_t> attr_done_v{0}, attr_done_w{0}, attr_done_r{0};
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kVarlen>, smem, attr_done_v)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kWindow>, smem, attr_done_w)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kRope>, smem, attr_done_r)) return ATTN_ERR_CUDA;
     // The kernel rebalances registers between warpgroups (setmaxnreg); that is
     // only safe if it was built with exactly the register count the split
     // assumes, otherwise the increase could never be granted.
-    static int regs_checked = 0;
-    if (regs_checked == 0) {
+    static std::atomic<int> regs_checked{0};   // 0: not yet checked, 1: ok, -1: mismatch
+    if (regs_checked.load(std::memory_order_acquire) == 0) {
         cudaFuncAttributes fa;
         cudaFuncAttributes fv, fw, fr;
         if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D, kDense>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fv, attn::pf::prefill_kernel<D, kVarlen>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fw, attn::pf::prefill_kernel<D, kWindow>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fr, attn::pf::prefill_kernel<D, kRope>) != cudaSuccess) return ATTN_ERR_CUDA;
-        regs_checked = (fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs &&
-                        fw.numRegs == attn::pf::kLaunchRegs && fr.numRegs == attn::pf::kLaunchRegs) ? 1 : -1;
+        regs_checked.store((fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs &&
+                            fw.numRegs == attn::pf::kLaunchRegs && fr.numRegs == attn::pf::kLaunchRegs) ? 1 : -1,
+                           std::memory_order_release);
     }
-    if (regs_checked < 0) return ATTN_ERR_UNSUPPORTED;
+    if (regs_checked.load(std::memory_order_acquire) < 0) return ATTN_ERR_UNSUPPORTED;
     if (vl) {
         // x: (position block, kv head), heaviest causal blocks first; y: sequence
         const long long gx = (long long)p.n_pb * n_kv;
@@ -310,7 +315,7 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
         if (!make_map(&tv, cv.v, 4, dims, vstr, box, 128)) return ATTN_ERR_CUDA;
     }
     const size_t smem = smem_bytes<GT, FP8>();
-    static uint64_t attr_done = 0;
+    static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(decode_split_kernel<GT, PAGED, FP8>, smem, attr_done)) return ATTN_ERR_CUDA;
     float *ws_o = reinterpret_cast<float *>(ws);
     size_t o_bytes = (size_t)B * n_q * n_splits * D * sizeof(float);
@@ -369,7 +374,7 @@ int launch_decode_mla(const void *q, const void *cache, const int32_t *seqlens, 
         if (!make_map(&tc, cache, 3, dims, str, box, 128)) return ATTN_ERR_CUDA;
     }
     const size_t smem = smem_bytes();
-    static uint64_t attr_done = 0;
+    static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(mla_decode_kernel, smem, attr_done)) return ATTN_ERR_CUDA;
     Params p;
     p.B = B;
@@ -818,17 +823,42 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_B
 
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[64] = {};
+CUcontext g_noalloc_ctx[64] = {};   // the context each cached address belongs to
 
-// Device address of the scratch array on the current device (first call on
-// a device does the lookup). Returns nullptr on failure.
+// The current CUDA context, through the runtime's driver entry point (the
+// library does not link the driver library itself). nullptr if unavailable.
+CUcontext current_context() {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    static GetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCurrentFn>(ptr);
+    });
+    CUcontext ctx = nullptr;
+    if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+    return ctx;
+}
+
+// Device address of the scratch array on the current device. The first call
+// on a device does the lookup; so does the first call after the device's
+// context changed (cudaDeviceReset loads the module, and the array, anew).
+// Returns nullptr on failure.
 void *noalloc_scratch_ptr() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    // (no context is current on a thread before its first runtime call that
+    // needs one: the lookup below makes the device's primary context current)
+    const CUcontext ctx = current_context();
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
         g_noalloc_ptr[dev] = ptr;
+        g_noalloc_ctx[dev] = current_context();
     }
     return g_noalloc_ptr[dev];
 }

@@ -143,15 +143,18 @@ def make(w: Workload, device="cpu"):
 
 def sample_rows(n_rows, B, n_q, Sq, seed, must=()):
     """A seeded sample of (b, h, i) row triples for sampled checks at full
-    size: every head appears, first/last rows and 128-row tile boundaries are
-    included, and the rest are uniform. Returns an int32 tensor [n, 3]."""
+    size, stratified: every (b, h) contributes its first and last row, both
+    rows at every 128-row tile boundary (i = 128t - 1 and 128t, each with a
+    seeded (b, h)) are included, and the rest are uniform. The forced rows
+    alone can exceed n_rows at long S; the result then holds all of them.
+    Returns an int32 tensor [n, 3], sorted."""
     g = torch.Generator().manual_seed(int(seed) + 7919)
     picks = set()
     for b in range(B):
         for h in range(n_q):
             picks.add((b, h, 0))
             picks.add((b, h, Sq - 1))
-    for i in list(range(127, Sq, 128))[:64] + list(range(128, Sq, 128))[:64]:
+    for i in list(range(127, Sq, 128)) + list(range(128, Sq, 128)):
         picks.add((int(torch.randint(B, (1,), generator=g)), int(torch.randint(n_q, (1,), generator=g)), i))
     for t in must:
         picks.add(tuple(int(x) for x in t))

@@ -131,9 +131,16 @@ def test_llama3_8b_prefill_sampled():
 
 
 def test_llama3_70b_long_prefill_sampled():
-    """Full-size 70B layout at S=32768: 1200 sampled rows."""
+    """Full-size 70B layout at S=32768: 4096 stratified (b, h, i) triples
+    (every head's first and last row, both sides of all 256 tile boundaries,
+    uniform rest) against the single-row oracle."""
     w = inputs.WORKLOADS["llama3_70b_long_prefill"]
-    _sampled(w, 1200, 12)
+    rows = inputs.sample_rows(4096, w.B, w.n_q, w.Sq, 12)
+    assert len(rows) == 4096
+    i = set(rows[:, 2].tolist())
+    assert all(t in i for t in range(127, w.Sq, 128)) and all(t in i for t in range(128, w.Sq, 128))
+    assert set(rows[:, 1].tolist()) == set(range(w.n_q))
+    _sampled(w, 4096, 12)
 
 
 def test_constant_keys_closed_form_full_size():

@@ -51,10 +51,17 @@ def _check_rope_prefill(o, lse, q, k, v, causal, scale, c, s, what):
     if causal:
         vis = np.arange(Skv)[None, :] <= (np.arange(Sq) + Skv - Sq)[:, None]
         ds = np.where(vis, ds, 0.0)
-    tol = 1e-3 + ds.max(axis=3)
+    widen = ds.max(axis=3)
+    tol = 1e-3 + widen
     lg = lse.double().cpu().numpy()
     assert np.all(np.abs(lg - lse_ref) <= tol), f"{what}: LSE excess {float((np.abs(lg - lse_ref) - tol).max()):.3e}"
-    return int((fq > 0).sum() + (fk > 0).sum())
+    # the widening is a rounding allowance, not a second tolerance: report it,
+    # and keep it well below the 1e-3 it is added to
+    w_max = float(widen.max()) if widen.size else 0.0
+    print(f"{what}: largest per-row LSE widening {w_max:.3e}, rows widened {int((widen > 0).sum())} of {widen.size}, "
+          f"largest |dLSE| {float(np.abs(lg - lse_ref).max()):.3e}")
+    assert w_max <= 5e-4, f"{what}: LSE widening {w_max:.3e} would dominate the 1e-3 tolerance"
+    return int((fq > 0).sum() + (fk > 0).sum()), w_max
 
 
 @pytest.mark.parametrize("n_pos,d,base", [(32768, 128, 500000.0), (4096, 64, 10000.0), (77, 32, 10000.0)])
@@ -164,7 +171,10 @@ def test_llama3_8b_prefill_rope_sampled():
     tol = 1e-3 + w.scale * (np.einsum("nd,nd->n", fq, kabs[g] + fkmax[g]) +
                             np.einsum("nd,nd->n", np.abs(q_rows), fkmax[g]))
     lg = lse[rb.cuda(), rh.cuda(), ri.cuda()].double().cpu().numpy()
-    assert np.all(np.abs(lg - lse_ref) <= tol)
+    dl = np.abs(lg - lse_ref)
+    print(f"llama3_8b_prefill rope: largest per-row LSE widening {float((tol - 1e-3).max()):.3e}, "
+          f"largest |dLSE| {float(dl.max()):.3e}, rows beyond 1e-3 {int((dl > 1e-3).sum())} of {len(dl)}")
+    assert np.all(dl <= tol)
 
 
 @pytest.mark.parametrize("n_q,n_kv", [(32, 8), (64, 4), (8, 8)])

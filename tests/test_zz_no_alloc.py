@@ -6,13 +6,15 @@ by the library, so the caller passes only inputs and outputs.
 
 Checked through the C ABI against attn_decode (which takes a caller-owned
 workspace) on two calls in a row, within the parity tolerances used by every
-GPU test here. This file is collected last on purpose."""
+GPU test here, and on a smaller problem also against the fp64 oracle. This
+file is collected last on purpose."""
 import ctypes
 
 import pytest
 import torch
 
-from gpu_util import LSE_ABS, O_MAX_ABS, need_gpu
+import oracle
+from gpu_util import LSE_ABS, O_MAX_ABS, check_parity, need_gpu
 from mqa_attention_attn_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -61,18 +63,23 @@ def test_noalloc_matches_attn_decode_twice():
 
 def test_noalloc_second_problem_after_first():
     """A smaller problem after a larger one: the leftover scratch contents of
-    the previous call must not leak into the result."""
+    the previous call must not leak into the result. Checked against
+    attn_decode and against the fp64 oracle, on two calls in a row."""
     binding = need_gpu()
     fn = _noalloc_fn(binding)
     seqlens, q, kc, vc = inputs.decode_inputs(3, 16, 4, 128, 128, 3000, (1, 3000), 77, device="cuda")
     sl = seqlens.cuda()
     o_ref, lse_ref = binding.attn_decode(q, kc, vc, sl, 0.1)
-    for _ in range(2):
+    o64, l64 = oracle.sdpa(q[:, :, None, :], kc, vc, False, 0.1, seqlens=seqlens.numpy())
+    for call in range(2):
         o, lse = torch.empty_like(o_ref), torch.empty_like(lse_ref)
-        assert _call_noalloc(fn, q, kc, vc, sl, o, lse, 0.1) == 0
+        rc = _call_noalloc(fn, q, kc, vc, sl, o, lse, 0.1)
+        assert rc == 0, binding.status_string(rc)
         torch.cuda.synchronize()
+        assert binding.device_status() == 0, f"call {call}"
         assert float((o.float() - o_ref.float()).abs().max()) <= O_MAX_ABS
         assert float((lse - lse_ref).abs().max()) <= LSE_ABS
+        check_parity(o, lse, o64[:, :, 0], l64[:, :, 0], f"no-alloc decode, call {call}")
 
 
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
