@@ -351,18 +351,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0, 0);
             const uint32_t idesc_o = umma_idesc_bf16(BM, D, 0, 1);
             bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x21);
+            // Descriptors are built once per operand tile and stepped by
+            // constant offsets in their 16-byte address field: for shared
+            // addresses a, o (multiples of 16, a + o < 2^18, so the 14-bit
+            // field cannot carry) desc(a + o) = desc(a) + (o >> 4). The base
+            // passes through a volatile move so that it is formed where it is
+            // used, not hoisted with all its offsets into registers (this
+            // warp runs on 56).
             auto issue_s = [&](int t, int j) {
                 const int s = j % KSTAGE;
-                const uint32_t qa = smem_u32(sm.q[t]);
-                const uint32_t ka = smem_u32(sm.k[s]);
+                const uint64_t qd0 = pin_u64(umma_smem_desc(smem_u32(sm.q[t]), 16, C::ATOM, C::LAYOUT));
+                const uint64_t kd0 = pin_u64(umma_smem_desc(smem_u32(sm.k[s]), 16, C::ATOM, C::LAYOUT));
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const int kel = ks * 16;
                     const uint32_t off_q = (kel / C::BOXD) * C::QBOX + (kel % C::BOXD) * 2;
                     const uint32_t off_k = (kel / C::BOXD) * C::KBOX + (kel % C::BOXD) * 2;
-                    const uint64_t ad = umma_smem_desc(qa + off_q, 16, C::ATOM, C::LAYOUT);
-                    const uint64_t bd = umma_smem_desc(ka + off_k, 16, C::ATOM, C::LAYOUT);
-                    umma_ss(tmem + C::col_s(t), ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                    // (the varlen instance builds each descriptor in full: with
+                    // the offset form its register allocation spills)
+                    if constexpr (VARLEN)
+                        umma_ss(tmem + C::col_s(t), umma_smem_desc(smem_u32(sm.q[t]) + off_q, 16, C::ATOM, C::LAYOUT),
+                                umma_smem_desc(smem_u32(sm.k[s]) + off_k, 16, C::ATOM, C::LAYOUT), idesc_s, ks > 0 ? 1u : 0u);
+                    else
+                        umma_ss(tmem + C::col_s(t), qd0 + (uint64_t)(off_q >> 4), kd0 + (uint64_t)(off_k >> 4), idesc_s,
+                                ks > 0 ? 1u : 0u);
                 }
                 umma_commit(smem_u32(&sm.s_full[t]));
             };
@@ -370,7 +382,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // warpgroup has written that chunk of P
             auto issue_pv = [&](int t, int j) -> bool {
                 const int s = j % VSTAGE;
-                const uint32_t va = smem_u32(sm.v[s]);
+                const uint64_t vd0 = pin_u64(umma_smem_desc(smem_u32(sm.v[s]), C::KBOX, C::ATOM, C::LAYOUT));
 #pragma unroll
                 for (int c = 0; c < kPChunks; ++c) {
                     if (!mbar_wait(smem_u32(&sm.p_full[t][c]), j & 1, abort_flag, 0x23)) return false;
@@ -378,8 +390,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int kk = 0; kk < kChunkKeys / 16; ++kk) {
                         const int ks = c * (kChunkKeys / 16) + kk;
-                        const uint64_t bd = umma_smem_desc(va + ks * 16 * C::ROWB, C::KBOX, C::ATOM, C::LAYOUT);
-                        umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + ks * 8, bd, idesc_o,
+                        umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + ks * 8,
+                                vd0 + (uint64_t)((uint32_t)(ks * 16 * C::ROWB) >> 4), idesc_o,
                                 (j > 0 || ks > 0) ? 1u : 0u);
                     }
                 }

@@ -289,6 +289,14 @@ __device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo_
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 
+// The value of x, formed at this point of the program: the compiler may not
+// precompute it elsewhere (keeps descriptor arithmetic out of registers).
+__device__ __forceinline__ uint64_t pin_u64(uint64_t x) {
+    uint64_t y;
+    asm volatile("mov.b64 %0, %1;" : "=l"(y) : "l"(x));
+    return y;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulate.
 // a_mn / b_mn select MN-major operands (0 = K-major).
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, int b_mn) {
