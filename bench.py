@@ -8,9 +8,10 @@ One step = one pass of the hot path over synthetic inputs resident in HBM:
   * MLA decode: attn_decode on the latent cache (B=64, 4096 rows of 576,
     128 heads, value = first 512 columns).
 The other configurations are timed in a loop of their own after the step:
-the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads) and the tiny
-causal forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency); so are the
-rows built beyond the path (paged, FP8 and RoPE forms), in a third loop.
+the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads), the tiny causal
+forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency) and two small-batch
+GQA decodes (B=1 at 32768 keys, B=4 at 8192); so are the rows built beyond
+the path (paged, FP8 and RoPE forms), in a third loop.
 `value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
 decode regimes are reported in HBM GB/s (algorithmic bytes: the K/V rows
 below each sequence's length, plus q, o and lse) under "regimes". Each kernel
@@ -379,6 +380,26 @@ def run_ours(args):
         add("tiny_prefill", "configs", 1,
             lambda: binding.attn_fwd(qt, kt, vt, wt.causal, wt.scale, o=ot, lse=lset, stream=stream))
 
+    # small-batch GQA decode (Llama-3-8B heads, full-length caches): one
+    # sequence of 32768 keys and four of 8192, where the split-KV plan must
+    # cut the keys finely enough to reach every SM
+    small_decode = {"decode_b1_32k": (1, 32768), "decode_b4_8k": (4, 8192)}
+    sd = {}
+    if sel("small_decode"):
+        for name, (Bs, Ls) in small_decode.items():
+            sl_s, q_s, k_s, v_s = inputs.decode_inputs(Bs, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, Ls, (Ls, Ls),
+                                                       wd.seed + 100 + Bs + gen_seed_shift, device=dev)
+            ws_s = torch.empty(binding.decode_workspace_bytes(Bs, wd.n_q, wd.n_kv, wd.d_qk, wd.d_v, Ls),
+                               dtype=torch.uint8, device=dev)
+            o_s = torch.empty((Bs, wd.n_q, wd.d_v), dtype=torch.bfloat16, device=dev)
+            l_s = torch.empty((Bs, wd.n_q), dtype=torch.float32, device=dev)
+            sd[name] = (sl_s, decode_bytes(inputs.Workload(name, "decode", B=Bs, n_q=wd.n_q, n_kv=wd.n_kv,
+                                                           d_qk=wd.d_qk, d_v=wd.d_v, seed=0), sl_s))
+            sl_s_dev = sl_s.to(dev)
+            add(name, "configs", 2, (lambda q_s=q_s, k_s=k_s, v_s=v_s, sl_s_dev=sl_s_dev, ws_s=ws_s, o_s=o_s, l_s=l_s:
+                                     binding.attn_decode(q_s, k_s, v_s, sl_s_dev, wd.scale, o=o_s, lse=l_s,
+                                                         workspace=ws_s, stream=stream)))
+
     # ---- the rows built beyond the path, on the same workloads
     # rotary position embedding (Llama-3 base 500000): prefill takes q, k
     # unrotated, decode a cache that holds rotated keys
@@ -642,6 +663,17 @@ def run_ours(args):
         out["tiny_prefill"] = {"workload": wt.name, "ms": ms_t, "latency_us": 1e3 * ms_t,
                                "latency_us_median": 1e3 * lat[len(lat) // 2], "tflops": tf(fl_t, ms_t),
                                "algorithmic_flops": fl_t, "bound": "launch latency (one CTA, one key tile)"}
+    for name in small_decode:
+        if name not in regimes:
+            continue
+        ms_s = mean[name]
+        sl_s, by_s = sd[name]
+        Bs, Ls = small_decode[name]
+        out[name] = {"workload": f"GQA decode, B={Bs}, every cache length {Ls}, n_q={wd.n_q} n_kv={wd.n_kv} d=128",
+                     "ms": ms_s, "gbs": gbs(by_s, ms_s), "frac_of_peak": gbs(by_s, ms_s) / peak_bw,
+                     "algorithmic_bytes": by_s,
+                     "roofline": hbm_roofline(by_s, ms_s, "attn::dec::decode_split_kernel<4>", None,
+                                              "achieved over split + merge launches")}
     if "paged_decode" in regimes:
         ms_g = mean["paged_decode"]
         out["paged_decode"] = {"workload": f"{wd.name}, {PAGE}-token pages in a shuffled pool", "ms": ms_g,
@@ -737,7 +769,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default="all",
-                    choices=["all", "prefill", "decode", "mla", "long", "tiny", "paged", "fp8", "rope"],
+                    choices=["all", "prefill", "decode", "mla", "long", "tiny", "small_decode", "paged", "fp8", "rope"],
                     help="time one regime only (used for profiling captures)")
     args = ap.parse_args()
     if args.gpus < 1:

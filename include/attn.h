@@ -129,7 +129,12 @@ int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float 
 /*
  * attn_decode_workspace_bytes -- scratch size attn_decode needs for these
  * sizes (split-KV partial outputs and their softmax statistics). Writes the
- * byte count to *bytes. The same sizes always give the same answer.
+ * byte count to *bytes. The split of the cached keys into chunks is planned
+ * from the sizes and the SM count of the CURRENT device (a small batch is
+ * cut into more chunks so that it spreads over every SM), so the answer is
+ * the same for the same sizes on the same device; ask with the device
+ * current that the decode will run on. (d_qk selects the shape family: the
+ * (576, 512) MLA form needs no workspace.)
  */
 int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int S_max,
                                 size_t *bytes);
@@ -208,7 +213,8 @@ int attn_decode_window(const void *q, const void *kcache, const void *vcache, co
  * their scales), computed exactly as attn_decode computes it for a bf16
  * cache; half the bytes cross HBM. Supported: head dim 128, n_q / n_kv a
  * power of two. Returns ATTN_OK or an error code (nothing launched on
- * error).
+ * error). attn_decode_fp8_workspace_bytes plans the key chunks as
+ * attn_decode_workspace_bytes does (sizes and the current device's SM count).
  */
 int attn_decode_fp8_workspace_bytes(int B, int n_q, int n_kv, int S_max, size_t *bytes);
 int attn_decode_fp8(const void *q, const void *kcache, const void *vcache, const float *k_scale,

@@ -245,11 +245,57 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
 // ---------------------------------------------------------------------------
 // decode (GQA, head dim 128)
 // ---------------------------------------------------------------------------
-// Query heads per decode work unit (a power of two dividing G) and the
-// number of key chunks of S_max at that block size.
+// Query heads per decode work unit (a power of two dividing G).
 inline int decode_head_block(int G) { return G >= 16 ? 16 : G; }
-inline int decode_n_splits(int G, int S_max) {
-    const int ch = attn::dec::chunk_keys(decode_head_block(G));
+
+// CTAs of the persistent decode grid resident at once on the current device:
+// two per SM while two fit in the SM's 228 KB of shared memory (with 1 KB
+// reserved per CTA; the register budget of two is fixed by the launch
+// bounds), else one.
+template <int GT, bool FP8>
+int decode_slots() {
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return -1;
+    const size_t smem = attn::dec::smem_bytes<GT, FP8>();
+    const int per_sm = (int)(233472 / (smem + 1024)) >= 2 ? 2 : 1;
+    return per_sm * n_sm;
+}
+
+// Keys per decode work unit (the split-KV chunk), planned from the sizes and
+// the SM count: with `slots` resident CTAs and B * n_kv * n_hb units per
+// chunk index, s = slots / (B * n_kv * n_hb) chunks per (sequence, KV head,
+// head block) give every unit of a full-length batch a slot of its own in one
+// wave, so a small batch still reaches every SM; the chunk is S_max / s keys
+// rounded up to the 128-key tile, at most the kernel's largest chunk (2048,
+// or 1024 at 16 heads per unit), which is also what a batch that fills the
+// slots by itself gets. The same sizes on the same device always give the
+// same chunk (the workspace size follows from it).
+template <int GT, bool FP8>
+int decode_chunk_t(int B, int n_kv, int G, int S_max) {
+    constexpr int CH = attn::dec::Cfg<GT, FP8>::CH, KT = attn::dec::KT;
+    const int slots = decode_slots<GT, FP8>();
+    const long long per_split = (long long)B * n_kv * (G / GT);
+    if (slots <= 0 || per_split <= 0) return CH;
+    const long long s = slots / per_split;
+    if (s <= 1) return CH;
+    long long ch = ((S_max + s - 1) / s + KT - 1) / KT * KT;
+    if (ch > CH) ch = CH;
+    if (ch < KT) ch = KT;
+    return (int)ch;
+}
+inline int decode_chunk(int B, int n_kv, int G, int S_max, bool fp8) {
+    switch (decode_head_block(G)) {
+        case 1: return fp8 ? decode_chunk_t<1, true>(B, n_kv, G, S_max) : decode_chunk_t<1, false>(B, n_kv, G, S_max);
+        case 2: return fp8 ? decode_chunk_t<2, true>(B, n_kv, G, S_max) : decode_chunk_t<2, false>(B, n_kv, G, S_max);
+        case 4: return fp8 ? decode_chunk_t<4, true>(B, n_kv, G, S_max) : decode_chunk_t<4, false>(B, n_kv, G, S_max);
+        case 8: return fp8 ? decode_chunk_t<8, true>(B, n_kv, G, S_max) : decode_chunk_t<8, false>(B, n_kv, G, S_max);
+        default:
+            return fp8 ? decode_chunk_t<16, true>(B, n_kv, G, S_max) : decode_chunk_t<16, false>(B, n_kv, G, S_max);
+    }
+}
+// Number of key chunks of S_max (the workspace's split dimension).
+inline int decode_n_splits(int B, int n_kv, int G, int S_max, bool fp8 = false) {
+    const int ch = decode_chunk(B, n_kv, G, S_max, fp8);
     return (S_max + ch - 1) / ch;
 }
 
@@ -280,7 +326,8 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
     using C = Cfg<GT, FP8>;
     const int G = n_q / n_kv;
     const int n_hb = G / GT;
-    const int n_splits = (S_max + C::CH - 1) / C::CH;
+    const int ch = decode_chunk_t<GT, FP8>(B, n_kv, G, S_max);
+    const int n_splits = (S_max + ch - 1) / ch;
     CUtensorMap tq, tk, tv;
     {
         // the group's query rows: [B][n_q][128], box = 64 dims x NH heads
@@ -322,23 +369,19 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
     o_bytes = (o_bytes + 255) & ~size_t(255);
     float2 *ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(ws) + o_bytes);
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
-    // persistent: as many CTAs as fit on the SMs at once (two per SM while
-    // two fit in the SM's 228 KB of shared memory, with 1 KB reserved per
-    // CTA; the register budget of two is fixed by the launch bounds), never
-    // more than the largest possible unit count
-    const int n_sm = sm_count();
-    if (n_sm <= 0) return ATTN_ERR_CUDA;
+    // persistent: as many CTAs as fit on the SMs at once, never more than the
+    // largest possible unit count
+    const int slots = decode_slots<GT, FP8>();
+    if (slots <= 0) return ATTN_ERR_CUDA;
     constexpr int threads = FP8 ? THREADS_FP8 : THREADS;
-    const int per_sm = (int)(233472 / (smem + 1024)) >= 2 ? 2 : 1;
     const long long max_units = (long long)B * n_kv * n_hb * n_splits;
-    const long long resident = (long long)per_sm * n_sm;
-    const int grid = (int)(max_units < resident ? max_units : resident);
+    const int grid = (int)(max_units < slots ? max_units : slots);
     decode_split_kernel<GT, PAGED, FP8><<<grid, threads, smem, stream>>>(tq, tk, tv, seqlens, ws_o, ws_ml, B, n_q,
-                                                                         n_kv, G, n_hb, S_max, n_splits, scale_log2,
-                                                                         cv.pt, cv.win, cv.fs, cv.rt);
+                                                                         n_kv, G, n_hb, S_max, n_splits, ch,
+                                                                         scale_log2, cv.pt, cv.win, cv.fs, cv.rt);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
-        ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, C::CH, cv.win);
+        ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, ch, cv.win);
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -510,7 +553,7 @@ int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int
         return ATTN_OK;
     }
     if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
-    *bytes = decode_ws_bytes(B, n_q, d_v, decode_n_splits(n_q / n_kv, S_max));
+    *bytes = decode_ws_bytes(B, n_q, d_v, decode_n_splits(B, n_kv, n_q / n_kv, S_max));
     return ATTN_OK;
 }
 
@@ -537,7 +580,7 @@ int decode_entry(const void *q, const void *kcache, const void *vcache, const in
         if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
         if ((k_stride_b | k_stride_h | k_stride_s | v_stride_b | v_stride_h | v_stride_s) & 7)
             return ATTN_ERR_MISALIGNED;
-        const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(G, S_max));
+        const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(B, n_kv, G, S_max));
         if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
         CacheView cv{};
@@ -680,8 +723,7 @@ int attn_decode_rope(const void *q, const void *kcache, const void *vcache, cons
 
 int attn_decode_fp8_workspace_bytes(int B, int n_q, int n_kv, int S_max, size_t *bytes) {
     if (!bytes || B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
-    const int ch = attn::dec::chunk_keys(decode_head_block(n_q / n_kv), true);
-    *bytes = decode_ws_bytes(B, n_q, 128, (S_max + ch - 1) / ch);
+    *bytes = decode_ws_bytes(B, n_q, 128, decode_n_splits(B, n_kv, n_q / n_kv, S_max, true));
     return ATTN_OK;
 }
 
@@ -745,7 +787,7 @@ int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, c
     if ((k_stride_page | k_stride_token | k_stride_head | v_stride_page | v_stride_token | v_stride_head) & 7)
         return ATTN_ERR_MISALIGNED;
     const int S_max = page_size * pages_per_seq;
-    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(G, S_max));
+    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(B, n_kv, G, S_max));
     if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
     CacheView cv{};
@@ -873,7 +915,7 @@ extern "C" int attn_decode_noalloc(const void *q, const void *kcache, const void
     if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
     if (B == 0) return ATTN_OK;
     if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
-    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(n_q / n_kv, S_max));
+    const size_t need = decode_ws_bytes(B, n_q, d_v, decode_n_splits(B, n_kv, n_q / n_kv, S_max));
     if (need > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;  // beyond the static maximum
     void *scratch = noalloc_scratch_ptr();
     if (scratch == nullptr) return ATTN_ERR_CUDA;

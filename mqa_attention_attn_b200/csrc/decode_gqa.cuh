@@ -1,7 +1,9 @@
 // decode_gqa.cuh -- single-token GQA decode against a KV cache, split-KV.
 //
 // A work unit is (sequence b, KV head g, a block of GT query heads of that
-// group, one chunk of CH consecutive cached keys, CH = 2048 or 1024). The grid
+// group, one chunk of ch consecutive cached keys: a multiple of 128 up to
+// 2048, or 1024 at 16 heads, chosen at launch from the sizes and the SM
+// count so that small batches too spread over every SM). The grid
 // is persistent (as many CTAs per SM as shared memory allows: two for the
 // bf16 and e4m3 caches at up to 8 heads per block); each CTA walks its share
 // of the units.
@@ -43,9 +45,11 @@ namespace dec {
 
 constexpr int D = 128;            // head dim (keys and values)
 constexpr int KT = 128;           // keys per tile (the MMA's M for S^T)
-// Keys per chunk (one work unit): 2048 while a head block has at most 8
-// heads, 1024 for 16 (the chunk's S^T, 16 or 8 tiles x NH columns, then
-// stays within 256 TMEM columns so that two CTAs share an SM).
+// Largest chunk of keys one work unit takes: 2048 while a head block has at
+// most 8 heads, 1024 for 16 (the chunk's S^T, 16 or 8 tiles x NH columns,
+// then stays within 256 TMEM columns so that two CTAs share an SM). The
+// launch may choose a smaller chunk (a multiple of 128 keys) so that small
+// batches still spread over every SM.
 __host__ __device__ constexpr int chunk_keys(int GT, bool fp8 = false) {
     return (void)fp8, GT <= 8 ? 2048 : 1024;
 }
@@ -71,7 +75,7 @@ constexpr int TILE8_BYTES = KT * D;         // 16 KB: 128 rows x 128 one-byte va
 template <int GT, bool FP8 = false>
 struct Cfg {
     static constexpr int NH = GT < 8 ? 8 : GT;             // MMA N (query-head columns)
-    static constexpr int CH = chunk_keys(GT, FP8);          // keys per unit
+    static constexpr int CH = chunk_keys(GT, FP8);          // most keys per unit
     static constexpr int TPC = CH / KT;                     // tiles per unit
     static constexpr int QBOX = NH * 128;                   // one 64-dim half of the Q rows
     static constexpr int COL_S = 0;                         // S^T: TPC tiles x NH columns
@@ -180,16 +184,14 @@ __device__ __forceinline__ int clamp_seqlen(const int32_t *seqlens, int b, int S
 
 // Advance the cursor to the sequence holding unit i (i never decreases) and
 // decode the unit. Returns false when i is past the last unit.
-template <int CH>
-__device__ __forceinline__ void start_sequence(UnitCursor &cur, const int32_t *seqlens, int S_max, Window w) {
+__device__ __forceinline__ void start_sequence(UnitCursor &cur, const int32_t *seqlens, int S_max, int CH, Window w) {
     cur.seqlen = clamp_seqlen(seqlens, cur.b, S_max);
     cur.plan = chunk_plan(cur.seqlen, CH, w);
     cur.ns = cur.plan.n;
 }
 
-template <int CH>
 __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const int32_t *seqlens, int B, int S_max,
-                                          int n_hb, int units_per_chunk, Window w, Unit &u) {
+                                          int CH, int n_hb, int units_per_chunk, Window w, Unit &u) {
     while (cur.b < B) {
         const long long n = (long long)units_per_chunk * cur.ns;
         if (i < cur.base + n) {
@@ -207,7 +209,7 @@ __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const in
         }
         cur.base += n;
         ++cur.b;
-        if (cur.b < B) start_sequence<CH>(cur, seqlens, S_max, w);
+        if (cur.b < B) start_sequence(cur, seqlens, S_max, CH, w);
     }
     return false;
 }
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(FP8 ? THREADS_FP8 : THREADS, (FP8 && GT >= 16)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ seqlens,
                     float *__restrict__ ws_o, float2 *__restrict__ ws_ml, int B, int n_q, int n_kv, int G, int n_hb,
-                    int S_max, int n_splits, float scale_log2, const PageTable pt, const Window win,
+                    int S_max, int n_splits, int ch, float scale_log2, const PageTable pt, const Window win,
                     const Fp8Scales fs, const rope::Tables rt) {
     using C = Cfg<GT, FP8>;
     constexpr int NH = C::NH;
@@ -283,7 +285,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     volatile int *abort_flag = &sm.abort_flag;
 
     UnitCursor cur;
-    if (B > 0) start_sequence<C::CH>(cur, seqlens, S_max, win);
+    if (B > 0) start_sequence(cur, seqlens, S_max, ch, win);
     Unit u;
 
     if (warp == PRODUCER_WARP) {
@@ -294,7 +296,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_prefetch_desc(&tm_v);
             int t = 0, n = 0;   // ring tiles issued, units started
             bool ok = true;
-            for (long long i = blockIdx.x; ok && next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
+            for (long long i = blockIdx.x; ok && next_unit(cur, i, seqlens, B, S_max, ch, n_hb, units_per_chunk, win, u);
                  i += gridDim.x, ++n) {
                 // the single Q buffer is free once the previous unit's S^T MMAs completed
                 if (n > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n - 1) & 1, abort_flag, 0x101)) break;
@@ -369,7 +371,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         constexpr uint32_t idesc_s = FP8 ? umma_idesc_f16(KT, NH, 0, 0) : umma_idesc_bf16(KT, NH, 0, 0);
         constexpr uint32_t idesc_o = FP8 ? umma_idesc_f16(D, NH, 1, 1) : umma_idesc_bf16(D, NH, 1, 1);
         int t = 0, n = 0, pc = 0;   // ring tiles, units, P tiles handed over
-        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
+        for (long long i = blockIdx.x; next_unit(cur, i, seqlens, B, S_max, ch, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             if (!mbar_wait(smem_u32(FP8 ? &sm.q_conv : &sm.q_full), n & 1, abort_flag, 0x201)) break;
             if (!FP8 && rt.cos != nullptr) {
@@ -470,7 +472,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int cw = (int)warp - CONV_WARP0;
         int t = 0, n = 0;
         bool ok = true;
-        for (long long i = blockIdx.x; ok && next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
+        for (long long i = blockIdx.x; ok && next_unit(cur, i, seqlens, B, S_max, ch, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             // the unit's Q rows, bf16 -> f16 in place (same byte positions)
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.q_full), n & 1, abort_flag, 0x401));
@@ -539,7 +541,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int tid = threadIdx.x;                       // key row of each tile; dim row of O^T
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
         int n = 0, pc = 0;   // units, P tiles handed over
-        for (long long i = blockIdx.x; next_unit<C::CH>(cur, i, seqlens, B, S_max, n_hb, units_per_chunk, win, u);
+        for (long long i = blockIdx.x; next_unit(cur, i, seqlens, B, S_max, ch, n_hb, units_per_chunk, win, u);
              i += gridDim.x, ++n) {
             const int h0 = u.kvh * G + u.hb * GT;
             // FP8: the key scale of this KV head scales every score

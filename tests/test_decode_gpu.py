@@ -90,9 +90,9 @@ def test_decode_equals_last_prefill_row():
 
 @pytest.mark.parametrize("L", [2047, 2048, 2049, 4097, 6500])
 def test_decode_independent_of_split_count(L):
-    """The split-KV decode (with 4 query heads per KV head the keys are cut
-    into ceil(L / 2048) chunks: 1, 1, 2, 3 and 4 here, on both sides of a
-    chunk boundary, merged by their log-sum-exp weights) equals the unsplit
+    """The split-KV decode (one sequence of 8 KV heads: the keys are cut into
+    as many chunks as it takes to reach every SM, chunk lengths of whole
+    128-key tiles, merged by their log-sum-exp weights) equals the unsplit
     computation: row L-1 of the causal prefill over the same L tokens."""
     binding = need_gpu()
     n_q, n_kv = 32, 8
@@ -173,3 +173,55 @@ def test_timeout_path_reports_status():
     assert binding.device_status() == 0
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum()) == 8.0
+
+
+def _planned_splits(B, n_kv, G, S_max):
+    """The split count the launch plans for a bf16 cache (two CTAs per SM at
+    up to 8 heads per unit): every unit of a full-length batch gets a slot of
+    the persistent grid when the batch alone does not fill it."""
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    GT = min(G, 16)
+    largest = 2048 if GT <= 8 else 1024
+    s = (2 * n_sm) // (B * n_kv * (G // GT))
+    ch = largest if s <= 1 else min(largest, -(-(-(-S_max // s)) // 128) * 128)
+    return -(-S_max // ch)
+
+
+@pytest.mark.parametrize("B,L,seqlens", [
+    (1, 32768, [32768]),                   # one long sequence: chunks over every SM
+    (4, 8192, [8192, 8192, 5000, 1]),     # a small batch, ragged
+])
+def test_small_batch_decode_spreads_over_the_sms(B, L, seqlens):
+    """Llama-3-8B heads (32 / 8), a batch too small to fill the GPU by whole
+    sequences: the keys are cut into enough chunks that every SM gets work
+    (the workspace has that many splits), and the result matches the oracle."""
+    binding = need_gpu()
+    n_q, n_kv = 32, 8
+    splits = _planned_splits(B, n_kv, n_q // n_kv, L)
+    assert splits > L // 2048, splits          # more chunks than the largest chunk gives
+    rows = B * n_q * splits
+    assert binding.decode_workspace_bytes(B, n_q, n_kv, 128, 128, L) == ((rows * 512 + 255) // 256) * 256 + rows * 8
+    seq = torch.tensor(seqlens, dtype=torch.int32)
+    g = torch.Generator(device="cuda").manual_seed(B * 7 + L)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(B, n_kv, L, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(B, n_kv, L, 128, generator=g, device="cuda").to(torch.bfloat16)
+    _decode_and_check(seq, q, kc, vc, 1 / math.sqrt(128), f"small-batch decode B={B} L={L}")
+
+
+def test_large_batch_decode_keeps_the_largest_chunk():
+    """A batch that fills every slot of the persistent grid by itself keeps
+    the largest chunk (2048 keys at 4 query heads per KV head); lengths on
+    both sides of chunk boundaries, against the oracle."""
+    binding = need_gpu()
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    n_q, n_kv, S_max = 32, 8, 6500
+    B = -(-2 * n_sm // n_kv)                       # B * n_kv >= the resident CTAs
+    assert _planned_splits(B, n_kv, n_q // n_kv, S_max) == 4
+    base = [2047, 2048, 2049, 4096, 4097, 6500, 1, 128, 129]
+    seq = torch.tensor([base[b % len(base)] for b in range(B)], dtype=torch.int32)
+    g = torch.Generator(device="cuda").manual_seed(77)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
+    _decode_and_check(seq, q, kc, vc, 1 / math.sqrt(128), f"large-batch decode B={B}")

@@ -75,7 +75,8 @@ def test_window_decode_skips_unread_chunks():
     vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
     for b, L in enumerate(seq.tolist()):
         # whole 2048-key spans between the sinks' chunk and the window's first
-        # chunk (chunks hold 2048 keys at this group size): never read
+        # chunk: never read, whatever chunk length (a whole number of 128-key
+        # tiles up to 2048) the launch plans
         lo = (L - W) // 2048 * 2048
         kc[b, :, 2048:lo] = float("nan")
         vc[b, :, 2048:lo] = float("nan")
