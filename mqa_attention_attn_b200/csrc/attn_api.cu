@@ -380,8 +380,20 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
                                                                          n_kv, G, n_hb, S_max, n_splits, ch,
                                                                          scale_log2, cv.pt, cv.win, cv.fs, cv.rt);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    decode_combine_kernel<<<dim3(n_q, B), COMBINE_THREADS, 0, stream>>>(
-        ws_o, ws_ml, seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, ch, cv.win);
+    // the merge, as a programmatic dependent of the split kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_q, B);
+    cfg.blockDim = dim3(COMBINE_THREADS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, (const float *)ws_o, (const float2 *)ws_ml, seqlens,
+                           reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, ch, cv.win) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

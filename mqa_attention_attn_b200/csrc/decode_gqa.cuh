@@ -239,6 +239,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const Fp8Scales fs, const rope::Tables rt) {
     using C = Cfg<GT, FP8>;
     constexpr int NH = C::NH;
+    // the merge kernel (launched as a programmatic dependent) may be scheduled
+    // now; it waits for this grid to complete before it reads the workspace
+    griddep_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     Smem<GT, FP8> &sm =
         *reinterpret_cast<Smem<GT, FP8> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -653,6 +656,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
 // Merge the chunks of each (b, h) (head dim D): M = max m_s, w_s = 2^(m_s - M),
 // O = sum w_s o_s / sum w_s l_s, LSE = (M + log2 sum w_s l_s) * ln 2.
+// Launched as a programmatic dependent of the split kernel, so that its launch
+// overlaps that kernel's tail; it waits for the partials before reading them.
 // One CTA per (h, b), 128 threads = 4 groups of 32; a group takes the
 // chunks s = g (mod 4), a lane 4 consecutive output dims per 128 (16-byte
 // loads), and the four groups' sums meet in shared memory.
@@ -672,6 +677,9 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
     const int ns = plan.n;   // chunks written for this sequence: splits plan.split(0 .. ns-1)
     const size_t row = (size_t)b * n_q + h;
     const float2 *ml = ws_ml + row * n_splits;
+    // launched as a programmatic dependent of the split kernel: its partials
+    // are complete and visible past this point
+    griddep_wait();
     if (ns == 0) {
         for (int d = tid; d < D; d += COMBINE_THREADS) o[row * D + d] = __float2bfloat16_rn(0.f);
         if (tid == 0 && lse) lse[row] = -INFINITY;
