@@ -9,9 +9,10 @@ One step = one pass of the hot path over synthetic inputs resident in HBM:
     128 heads, value = first 512 columns).
 The other configurations are timed in a loop of their own after the step:
 the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads), the tiny causal
-forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency) and two small-batch
-GQA decodes (B=1 at 32768 keys, B=4 at 8192); so are the rows built beyond
-the path (paged, FP8 and RoPE forms), in a third loop.
+forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency), two small-batch
+GQA decodes (B=1 at 32768 keys, B=4 at 8192) and two small-batch MLA decodes
+(B=1 and B=4 at 4096 keys); so are the rows built beyond the path (paged,
+FP8 and RoPE forms), in a third loop.
 `value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
 decode regimes are reported in HBM GB/s (algorithmic bytes: the K/V rows
 below each sequence's length, plus q, o and lse) under "regimes". Each kernel
@@ -400,6 +401,28 @@ def run_ours(args):
                                      binding.attn_decode(q_s, k_s, v_s, sl_s_dev, wd.scale, o=o_s, lse=l_s,
                                                          workspace=ws_s, stream=stream)))
 
+    # small-batch MLA decode (the MLA workload's shape with 1 and 4
+    # sequences): the keys of each sequence are cut into chunks over the SMs
+    small_mla = {"mla_decode_b1": 1, "mla_decode_b4": 4}
+    smla = {}
+    if sel("small_decode"):
+        for name, Bm in small_mla.items():
+            sl_m, q_m, c_m = inputs.mla_inputs(Bm, wm.n_q, wm.d_qk, wm.Skv, (wm.Skv, wm.Skv),
+                                               wm.seed + 100 + Bm + gen_seed_shift, device=dev)
+            nws = binding.decode_workspace_bytes(Bm, wm.n_q, wm.n_kv, wm.d_qk, wm.d_v, wm.Skv)
+            ws_m = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+            o_m = torch.empty((Bm, wm.n_q, wm.d_v), dtype=torch.bfloat16, device=dev)
+            l_m = torch.empty((Bm, wm.n_q), dtype=torch.float32, device=dev)
+            smla[name] = (mla_bytes(inputs.Workload(name, "mla_decode", B=Bm, n_q=wm.n_q, n_kv=1, d_qk=wm.d_qk,
+                                                    d_v=wm.d_v, seed=0), sl_m),
+                          decode_flops(inputs.Workload(name, "mla_decode", B=Bm, n_q=wm.n_q, n_kv=1, d_qk=wm.d_qk,
+                                                       d_v=wm.d_v, seed=0), sl_m), nws > 0)
+            c_m4, sl_m_dev = c_m[:, None], sl_m.to(dev)
+            add(name, "configs", 2 if nws > 0 else 1,
+                (lambda q_m=q_m, c_m4=c_m4, sl_m_dev=sl_m_dev, ws_m=ws_m, o_m=o_m, l_m=l_m:
+                 binding.attn_decode(q_m, c_m4, c_m4, sl_m_dev, wm.scale, d_v=wm.d_v, o=o_m, lse=l_m, workspace=ws_m,
+                                     stream=stream)))
+
     # ---- the rows built beyond the path, on the same workloads
     # rotary position embedding (Llama-3 base 500000): prefill takes q, k
     # unrotated, decode a cache that holds rotated keys
@@ -674,6 +697,19 @@ def run_ours(args):
                      "algorithmic_bytes": by_s,
                      "roofline": hbm_roofline(by_s, ms_s, "attn::dec::decode_split_kernel<4>", None,
                                               "achieved over split + merge launches")}
+    for name, Bm in small_mla.items():
+        if name not in regimes:
+            continue
+        ms_s = mean[name]
+        by_s, fl_s, split = smla[name]
+        t_hbm, t_tc = by_s / (peak_bw * 1e9), fl_s / (peak_tf * 1e12)
+        out[name] = {"workload": f"MLA absorbed decode, B={Bm}, S=4096, 128 heads, key 576 / value 512",
+                     "ms": ms_s, "gbs": gbs(by_s, ms_s), "tflops": tf(fl_s, ms_s),
+                     "roofline_frac": max(t_hbm, t_tc) / (ms_s / 1e3), "split_kv": split,
+                     "algorithmic_bytes": by_s, "algorithmic_flops": fl_s,
+                     "roofline": dict(hbm_roofline(by_s, ms_s, MLA_KERNEL, None,
+                                                   "achieved over split + merge launches" if split else None),
+                                      tensor_frac=tf(fl_s, ms_s) / peak_tf)}
     if "paged_decode" in regimes:
         ms_g = mean["paged_decode"]
         out["paged_decode"] = {"workload": f"{wd.name}, {PAGE}-token pages in a shuffled pool", "ms": ms_g,

@@ -160,7 +160,9 @@ int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int
  *           bytes, 256-byte aligned; its contents on entry do not matter.
  *           Calls that share a workspace must be ordered on one stream.
  *           (128, 128): split-KV partial outputs and statistics; (576, 512):
- *           none is needed (0 bytes; the pointer may be NULL).
+ *           the same for the key chunks when the batch is too small to fill
+ *           the GPU by whole sequences, and none otherwise (0 bytes; the
+ *           pointer may then be NULL).
  * Supported: (d_qk, d_v) = (128, 128) with n_q / n_kv in {1, 2, 4, 8, 16, ...}
  * (any power of two); (576, 512) with n_kv = 1 (MLA absorbed decode, the
  * scale usually 1/sqrt(128 + 64)). Cache rows at or past a sequence's length

@@ -391,7 +391,7 @@ int launch_decode_gqa(const void *q, const CacheView &cv, const int32_t *seqlens
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, (const float *)ws_o, (const float2 *)ws_ml, seqlens,
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, (const float *)ws_o, (const float2 *)ws_ml, seqlens,
                            reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, n_splits, S_max, ch, cv.win) != cudaSuccess)
         return ATTN_ERR_CUDA;
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -412,8 +412,32 @@ int dispatch_decode_gqa(int G, const void *q, const CacheView &cv, const int32_t
 // ---------------------------------------------------------------------------
 // MLA decode (latent row of 576 = key, its first 512 columns = value)
 // ---------------------------------------------------------------------------
+// Split-KV plan of the MLA decode: a 2-CTA cluster per (sequence, head
+// block, key chunk), one CTA per SM. With c = SMs / 2 clusters resident and
+// B * n_hb of them per chunk index, s = c / (B * n_hb) chunks per sequence
+// give a full-length batch one wave over every SM; chunks hold at least two
+// 64-key tiles (every chunk's cluster loads the whole query block). A batch
+// that fills the clusters by itself gets one chunk per sequence, and then no
+// workspace: the clusters write O and LSE themselves.
+int mla_n_splits(int B, int n_q, int S_max, int *chunk) {
+    constexpr int KT = attn::mla::KT, MIN_CHUNK = 2 * KT;
+    const int n_sm = sm_count();
+    const long long per_split = (long long)B * (n_q / attn::mla::M);
+    long long s = (n_sm > 0 && per_split > 0) ? (n_sm / 2) / per_split : 1;
+    const long long most = (S_max + MIN_CHUNK - 1) / MIN_CHUNK;
+    if (s > most) s = most;
+    if (s < 1) s = 1;
+    const int ch = (int)(((S_max + s - 1) / s + KT - 1) / KT * KT);
+    if (chunk) *chunk = ch;
+    return (S_max + ch - 1) / ch;
+}
+size_t mla_ws_bytes(int B, int n_q, int S_max) {
+    const int n_splits = mla_n_splits(B, n_q, S_max, nullptr);
+    return n_splits > 1 ? decode_ws_bytes(B, n_q, attn::mla::DV, n_splits) : 0;
+}
+
 int launch_decode_mla(const void *q, const void *cache, const int32_t *seqlens, void *o, float *lse, int B, int n_q,
-                      int S_max, int64_t stride_b, int64_t stride_s, float scale, cudaStream_t stream) {
+                      int S_max, int64_t stride_b, int64_t stride_s, float scale, void *ws, cudaStream_t stream) {
     using namespace attn::mla;
     CUtensorMap tq, tc;
     {
@@ -439,8 +463,18 @@ int launch_decode_mla(const void *q, const void *cache, const int32_t *seqlens, 
     p.o = reinterpret_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.n_splits = mla_n_splits(B, n_q, S_max, &p.ch);
+    p.ws_o = nullptr;
+    p.ws_ml = nullptr;
+    if (p.n_splits > 1) {
+        size_t o_bytes = (size_t)B * n_q * p.n_splits * DV * sizeof(float);
+        o_bytes = (o_bytes + 255) & ~size_t(255);
+        p.ws_o = reinterpret_cast<float *>(ws);
+        p.ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(ws) + o_bytes);
+    }
+    if ((long long)2 * B * p.n_splits > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * B, n_q / M, 1);
+    cfg.gridDim = dim3(2 * B * p.n_splits, n_q / M, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -452,6 +486,22 @@ int launch_decode_mla(const void *q, const void *cache, const int32_t *seqlens, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, mla_decode_kernel, tq, tc, p) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (p.n_splits == 1) return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    // the merge of the chunks (as for the GQA decode), a programmatic dependent
+    cudaLaunchConfig_t mcfg = {};
+    mcfg.gridDim = dim3(n_q, B);
+    mcfg.blockDim = dim3(attn::dec::COMBINE_THREADS);
+    mcfg.dynamicSmemBytes = 0;
+    mcfg.stream = stream;
+    cudaLaunchAttribute mattr[1];
+    mattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    mattr[0].val.programmaticStreamSerializationAllowed = 1;
+    mcfg.attrs = mattr;
+    mcfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&mcfg, attn::dec::decode_combine_kernel<DV>, (const float *)p.ws_o, (const float2 *)p.ws_ml,
+                           seqlens, reinterpret_cast<__nv_bfloat16 *>(o), lse, n_q, p.n_splits, S_max, p.ch,
+                           attn::dec::Window{0, 0}) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -560,8 +610,9 @@ int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float 
 
 int attn_decode_workspace_bytes(int B, int n_q, int n_kv, int d_qk, int d_v, int S_max, size_t *bytes) {
     if (!bytes || B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
-    if (d_qk == 576 && d_v == 512 && n_kv == 1) {  // the MLA kernel keeps everything on chip
-        *bytes = 0;
+    if (d_qk == 576 && d_v == 512 && n_kv == 1) {  // 0 when one chunk per sequence is planned
+        if (n_q % attn::mla::M != 0) return ATTN_ERR_UNSUPPORTED;
+        *bytes = mla_ws_bytes(B, n_q, S_max);
         return ATTN_OK;
     }
     if (!(d_qk == 128 && d_v == 128)) return ATTN_ERR_UNSUPPORTED;
@@ -613,7 +664,13 @@ int decode_entry(const void *q, const void *kcache, const void *vcache, const in
         if (!aligned16(q) || !aligned16(kcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
         if ((k_stride_b | k_stride_s) & 7) return ATTN_ERR_MISALIGNED;
         if (B > 32767) return ATTN_ERR_UNSUPPORTED;
-        return launch_decode_mla(q, kcache, seqlens, o, lse, B, n_q, S_max, k_stride_b, k_stride_s, scale, s);
+        const size_t need = mla_ws_bytes(B, n_q, S_max);
+        if (need > 0) {
+            if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+            if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+        }
+        return launch_decode_mla(q, kcache, seqlens, o, lse, B, n_q, S_max, k_stride_b, k_stride_s, scale, workspace,
+                                 s);
     }
     return ATTN_ERR_UNSUPPORTED;
 }

@@ -654,8 +654,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 }
 
-// Merge the chunks of each (b, h) (head dim D): M = max m_s, w_s = 2^(m_s - M),
-// O = sum w_s o_s / sum w_s l_s, LSE = (M + log2 sum w_s l_s) * ln 2.
+// Merge the chunks of each (b, h) (value width DV: 128, or the MLA form's 512):
+// M = max m_s, w_s = 2^(m_s - M), O = sum w_s o_s / sum w_s l_s,
+// LSE = (M + log2 sum w_s l_s) * ln 2.
 // Launched as a programmatic dependent of the split kernel, so that its launch
 // overlaps that kernel's tail; it waits for the partials before reading them.
 // One CTA per (h, b), 128 threads = 4 groups of 32; a group takes the
@@ -663,11 +664,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 // loads), and the four groups' sums meet in shared memory.
 constexpr int COMBINE_THREADS = 128;
 
+template <int DV>
 __global__ void __launch_bounds__(COMBINE_THREADS)
 decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__ ws_ml,
                       const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o,
                       float *__restrict__ lse, int n_q, int n_splits, int S_max, int chunk, Window win) {
-    __shared__ float red[4][D];
+    static_assert(DV % 128 == 0, "value width");
+    constexpr int NQ = DV / 128;   // float4 loads per lane and chunk
+    __shared__ float red[4][DV];
     __shared__ float part[4];
     const int h = blockIdx.x, b = blockIdx.y;
     const int tid = threadIdx.x, g = tid >> 5, lane = tid & 31;
@@ -681,7 +685,7 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
     // are complete and visible past this point
     griddep_wait();
     if (ns == 0) {
-        for (int d = tid; d < D; d += COMBINE_THREADS) o[row * D + d] = __float2bfloat16_rn(0.f);
+        for (int d = tid; d < DV; d += COMBINE_THREADS) o[row * DV + d] = __float2bfloat16_rn(0.f);
         if (tid == 0 && lse) lse[row] = -INFINITY;
         return;
     }
@@ -694,29 +698,35 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
     __syncthreads();
     M = fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3]));
     // this group's weighted sum of o_s over its chunks, and of l_s
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc[NQ];
+#pragma unroll
+    for (int qi = 0; qi < NQ; ++qi) acc[qi] = make_float4(0.f, 0.f, 0.f, 0.f);
     float L = 0.f;
-    const float *base = ws_o + row * n_splits * (size_t)D + lane * 4;
+    const float *base = ws_o + row * n_splits * (size_t)DV + lane * 4;
 #pragma unroll 4
     for (int c = g; c < ns; c += 4) {
         const int s = plan.split(c);
         const float2 m_l = ml[s];
         const float w = ex2(m_l.x - M);
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(base + (size_t)s * D));
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(base + (size_t)s * DV + qi * 128));
+            acc[qi].x = fmaf(w, v.x, acc[qi].x);
+            acc[qi].y = fmaf(w, v.y, acc[qi].y);
+            acc[qi].z = fmaf(w, v.z, acc[qi].z);
+            acc[qi].w = fmaf(w, v.w, acc[qi].w);
+        }
         L = fmaf(w, m_l.y, L);
     }
-    *reinterpret_cast<float4 *>(&red[g][lane * 4]) = acc;
+#pragma unroll
+    for (int qi = 0; qi < NQ; ++qi) *reinterpret_cast<float4 *>(&red[g][qi * 128 + lane * 4]) = acc[qi];
     __syncthreads();   // part[] reads above are done before it is reused
     if (lane == 0) part[g] = L;
     __syncthreads();
     const float Lt = part[0] + part[1] + part[2] + part[3];
     const float inv = 1.f / Lt;
-    for (int d = tid; d < D; d += COMBINE_THREADS)
-        o[row * D + d] = __float2bfloat16_rn((red[0][d] + red[1][d] + red[2][d] + red[3][d]) * inv);
+    for (int d = tid; d < DV; d += COMBINE_THREADS)
+        o[row * DV + d] = __float2bfloat16_rn((red[0][d] + red[1][d] + red[2][d] + red[3][d]) * inv);
     if (tid == 0 && lse) lse[row] = (M + log2f(Lt)) * 0.6931471805599453f;
 }
 

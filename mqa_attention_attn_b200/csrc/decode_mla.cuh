@@ -25,6 +25,14 @@
 // The score MMAs are done twice (1.5x the algorithmic FLOPs in all); in
 // exchange the two SMs never wait on each other. TMA loads are plain (no
 // multicast).
+// Split-KV (the decode against the cache of "Attention deep dive", section 5,
+// cut across SMs): a batch too small to occupy every SM by whole sequences
+// has each sequence's keys cut into chunks, one cluster per chunk; each
+// cluster then writes its unnormalised partial output and (m, l) to the
+// workspace, and the merge kernel of the GQA decode combines the chunks by
+// their log-sum-exp weights (the section 4 recurrence of "Attention
+// Engineering" across chunks). A batch that fills the SMs keeps one chunk per
+// sequence and writes O and LSE directly.
 #pragma once
 
 #include "sm100.cuh"
@@ -74,6 +82,14 @@ struct Params {
     __nv_bfloat16 *o;      // [B, n_q, 512]
     float *lse;            // [B, n_q] or null
     float scale_log2;
+    // Split-KV: cluster c takes keys [s * ch, (s + 1) * ch) of sequence
+    // c / n_splits, s = c % n_splits. With one split the cluster writes O and
+    // LSE; with more it writes its unnormalised partial output o_s (fp32,
+    // [B, n_q, n_splits, 512]) and (m_s, l_s) ([B, n_q, n_splits], log2
+    // units) for the merge kernel.
+    int n_splits, ch;
+    float *ws_o;
+    float2 *ws_ml;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -89,14 +105,18 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t warp = warp_id(), lane = lane_id();
     const uint32_t rank = cluster_rank();            // which half of the output
-    const int b = blockIdx.x / 2;
+    const int b = (int)(blockIdx.x / 2) / p.n_splits;
+    const int split = (int)(blockIdx.x / 2) % p.n_splits;
     const int hb = blockIdx.y;                        // block of 128 heads
-    int nkeys = p.seqlens[b];
-    if (nkeys > p.S_max) {
-        if (threadIdx.x == 0 && rank == 0 && hb == 0) atomicOr(&g_status, kStatusRange);
-        nkeys = p.S_max;
+    int seqlen = p.seqlens[b];
+    if (seqlen > p.S_max) {
+        if (threadIdx.x == 0 && rank == 0 && hb == 0 && split == 0) atomicOr(&g_status, kStatusRange);
+        seqlen = p.S_max;
     }
-    if (nkeys < 0) nkeys = 0;
+    if (seqlen < 0) seqlen = 0;
+    // this cluster's keys: key0 .. key0 + nkeys - 1 of the sequence
+    const int key0 = split * p.ch;
+    const int nkeys = max(0, min(p.ch, seqlen - key0));
     const int nt = (nkeys + KT - 1) / KT;
     const int tail = nt > 0 ? nkeys - (nt - 1) * KT : KT;   // valid rows of the last tile
 
@@ -156,7 +176,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint32_t fb = smem_u32(&sm.kv_full[s][g]);
                     mbar_arrive_expect_tx(fb, (uint32_t)(NB / NG * KBOX));
                     for (int bx = g * (NB / NG); bx < (g + 1) * (NB / NG); ++bx)
-                        tma_load_3d(smem_u32(sm.k[s][bx]), &tm_c, fb, 64 * bx, j * KT, b);
+                        tma_load_3d(smem_u32(sm.k[s][bx]), &tm_c, fb, 64 * bx, key0 + j * KT, b);
                 }
                 ++issued;
             }
@@ -367,34 +387,58 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncwarp();
         tc_fence_after();
         const int head = hb * M + r;
-        if (head < p.n_q && nt == 0) {
-            uint4 *orow = reinterpret_cast<uint4 *>(p.o + ((size_t)b * p.n_q + head) * DV + 256 * rank);
-            for (int c = 0; c < 256 / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
-        }
-        if (nt > 0) {
-            const float inv_l = 1.f / l_run;
+        if (p.n_splits > 1) {
+            // partial output of this chunk for the merge kernel: unnormalised O
+            // (this CTA's 256 columns) and, from rank 0, (m, l); a chunk with
+            // no key writes nothing (the merge reads only the chunks below the
+            // sequence's length)
+            if (nt > 0) {
+                const size_t prow = ((size_t)b * p.n_q + head) * p.n_splits + split;
 #pragma unroll 1
-            for (int c = 0; c < 256 / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(trow + COL_O + 32 * c, o);
-                tmem_wait_ld();
-                if (head < p.n_q) {
-                    uint4 *dst =
-                        reinterpret_cast<uint4 *>(p.o + ((size_t)b * p.n_q + head) * DV + 256 * rank + 32 * c);
+                for (int c = 0; c < 256 / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(trow + COL_O + 32 * c, o);
+                    tmem_wait_ld();
+                    if (head < p.n_q) {
+                        float4 *dst = reinterpret_cast<float4 *>(p.ws_o + prow * DV + 256 * rank + 32 * c);
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        uint4 w;
-                        w.x = f2_to_bf2(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
-                        w.y = f2_to_bf2(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
-                        w.z = f2_to_bf2(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
-                        w.w = f2_to_bf2(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
-                        dst[q8] = w;
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
+                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+                    }
+                }
+                if (rank == 0 && head < p.n_q) p.ws_ml[prow] = make_float2(m_run, l_run);
+            }
+        } else {
+            if (head < p.n_q && nt == 0) {
+                uint4 *orow = reinterpret_cast<uint4 *>(p.o + ((size_t)b * p.n_q + head) * DV + 256 * rank);
+                for (int c = 0; c < 256 / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
+            }
+            if (nt > 0) {
+                const float inv_l = 1.f / l_run;
+#pragma unroll 1
+                for (int c = 0; c < 256 / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(trow + COL_O + 32 * c, o);
+                    tmem_wait_ld();
+                    if (head < p.n_q) {
+                        uint4 *dst =
+                            reinterpret_cast<uint4 *>(p.o + ((size_t)b * p.n_q + head) * DV + 256 * rank + 32 * c);
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            uint4 w;
+                            w.x = f2_to_bf2(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
+                            w.y = f2_to_bf2(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
+                            w.z = f2_to_bf2(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
+                            w.w = f2_to_bf2(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
+                            dst[q8] = w;
+                        }
                     }
                 }
             }
+            if (rank == 0 && head < p.n_q && p.lse != nullptr)
+                p.lse[(size_t)b * p.n_q + head] = nt > 0 ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
         }
-        if (rank == 0 && head < p.n_q && p.lse != nullptr)
-            p.lse[(size_t)b * p.n_q + head] = nt > 0 ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
     }
 
     // ---- teardown

@@ -98,3 +98,33 @@ def test_mla_rejects_unaliased_value():
     with pytest.raises(binding.AttnError) as e:
         binding.attn_decode(q, c, v, torch.ones(1, dtype=torch.int32, device="cuda"), 0.1, d_v=512)
     assert e.value.code == -2
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_mla_small_batch_split_over_the_sms(B):
+    """A batch too small to fill the GPU by whole sequences (S=4096, 128
+    heads): the keys are cut into chunks, each a 2-CTA cluster of its own
+    writing a partial output to the workspace, merged by their log-sum-exp
+    weights; every output row against the oracle."""
+    binding = need_gpu()
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    S = 4096
+    ws = binding.decode_workspace_bytes(B, 128, 1, 576, 512, S)
+    # clusters of two SMs; at least two 64-key tiles per chunk
+    s = min((n_sm // 2) // B, S // 128)
+    ch = -(-(-(-S // s)) // 64) * 64
+    splits = -(-S // ch)
+    assert splits > 1
+    rows = B * 128 * splits
+    assert ws == ((rows * 512 * 4 + 255) // 256) * 256 + rows * 8, (ws, splits)
+    seqlens, q, cache = inputs.mla_inputs(B, 128, 576, S, (S, S), 40 + B, device="cuda")
+    _run(seqlens, q, cache, 1 / math.sqrt(192), f"mla split B={B}")
+
+
+def test_mla_full_batch_needs_no_workspace():
+    """The MLA workload's batch (64 sequences) fills the clusters by itself:
+    one chunk per sequence, no workspace."""
+    binding = need_gpu()
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    B = max(64, n_sm // 2)
+    assert binding.decode_workspace_bytes(B, 128, 1, 576, 512, 4096) == 0
