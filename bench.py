@@ -11,8 +11,8 @@ The other configurations are timed in a loop of their own after the step:
 the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads), the tiny causal
 forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency), two small-batch
 GQA decodes (B=1 at 32768 keys, B=4 at 8192) and two small-batch MLA decodes
-(B=1 and B=4 at 4096 keys); so are the rows built beyond the path (paged,
-FP8 and RoPE forms), in a third loop.
+(B=1 and B=4 at 4096 keys); so are the rows built beyond the path (paged
+prefill and decode, FP8 and RoPE forms), in a third loop.
 `value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
 decode regimes are reported in HBM GB/s (algorithmic bytes: the K/V rows
 below each sequence's length, plus q, o and lse) under "regimes". Each kernel
@@ -453,6 +453,27 @@ def run_ours(args):
         add("fp8_decode", "next", 2, lambda: binding.attn_decode_fp8(
             qd, k8, v8, ks8, vs8, sl_dev, wd.scale, o=of8, lse=lf8, workspace=work8, stream=stream))
 
+    # the Llama-3-8B prefill with its keys and values in 64-token pages placed
+    # in a pool in a seeded random order (chunked-prefill serving layout)
+    if sel("paged"):
+        PPAGE = 64
+        Pp = w.Skv // PPAGE
+        perm_p = torch.randperm(Pp, generator=torch.Generator().manual_seed(w.seed + 78)).to(torch.int32)
+        table_p = perm_p[None].to(dev)
+        kd_p = k[0].permute(1, 0, 2).reshape(Pp, PPAGE, w.n_kv, w.d_qk)
+        vd_p = v[0].permute(1, 0, 2).reshape(Pp, PPAGE, w.n_kv, w.d_v)
+        pool_kp, pool_vp = torch.empty_like(kd_p), torch.empty_like(vd_p)
+        pool_kp[perm_p.long().to(dev)] = kd_p
+        pool_vp[perm_p.long().to(dev)] = vd_p
+        del kd_p, vd_p
+        q_packed = q[0].permute(1, 0, 2).contiguous()
+        cu_qp = torch.tensor([0, w.Sq], dtype=torch.int32, device=dev)
+        sk_p = torch.tensor([w.Skv], dtype=torch.int32, device=dev)
+        o_pp = torch.empty_like(q_packed)
+        l_pp = torch.empty((w.n_q, w.Sq), dtype=torch.float32, device=dev)
+        add("paged_prefill", "next", 1, lambda: binding.attn_fwd_paged(
+            q_packed, pool_kp, pool_vp, table_p, cu_qp, sk_p, w.Sq, w.causal, w.scale, o=o_pp, lse=l_pp, stream=stream))
+
     # the GQA decode workload again, its cache cut into 64-token pages placed
     # in a pool in a seeded random order (the paged-cache serving layout)
     PAGE = 64
@@ -716,6 +737,12 @@ def run_ours(args):
                                "gbs": gbs(by_d, ms_g), "frac_of_peak": gbs(by_d, ms_g) / peak_bw,
                                "algorithmic_bytes": by_d,
                                "kernels": "attn::dec::decode_split_kernel<4, paged> + decode_combine_kernel"}
+    if "paged_prefill" in regimes:
+        ms_pp = mean["paged_prefill"]
+        out["paged_prefill"] = {"workload": f"{w.name}, keys and values in 64-token pages in a shuffled pool",
+                                "ms": ms_pp, "tflops": tf(fl_p, ms_pp), "frac_of_peak": tf(fl_p, ms_pp) / peak_tf,
+                                "kernel": "attn::pf::prefill_kernel<128, paged>",
+                                "roofline": tensor_roofline(fl_p, ms_pp, "attn::pf::prefill_kernel<128, paged>", None)}
     if "fp8_decode" in regimes:
         ms_f = mean["fp8_decode"]
         out["fp8_decode"] = {"workload": f"{wd.name}, e4m3 cache with one scale per KV head", "ms": ms_f,

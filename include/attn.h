@@ -269,6 +269,49 @@ int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, c
                       float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_fwd_paged -- prefill (or chunked prefill) of a packed batch whose keys
+ * and values live in a paged KV cache. Source: "Attention deep dive"
+ * (askaiml.pages.dev), section 5 (production engines keep the KV cache in
+ * fixed-size pages addressed through a page table, and batch sequences of
+ * different lengths); the attention of each sequence is that of attn_fwd_varlen
+ * over its first seqlens_k[b] cached tokens, only where those tokens live
+ * changes. The cached tokens include the new ones (the caller writes the new
+ * keys and values into the cache before the call), so a chunk of Sq_b new
+ * queries sits at the end of its sequence: query i of sequence b is position
+ * seqlens_k[b] - Sq_b + i.
+ *
+ *   q            [total_q, n_q, d_qk] bf16, contiguous (the queries of all
+ *                sequences, packed); o [total_q, n_q, d_v] bf16 (written);
+ *                lse [n_q, total_q] fp32 (written; may be NULL)
+ *   cu_seqlens_q [B + 1] int32 on the device: sequence b owns query rows
+ *                cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 (non-decreasing)
+ *   seqlens_k    [B] int32 on the device: cached tokens of sequence b
+ *                (values above pages_per_seq * page_size are clamped and
+ *                reported as ATTN_ERR_DEVICE_RANGE by attn_device_status)
+ *   k_pages, v_pages, block_table, page_size, pages_per_seq, num_pages and
+ *                the page / token / head strides (in ELEMENTS): as for
+ *                attn_decode_paged (head dim d_qk = d_v instead of 128; token
+ *                stride >= d). Only table entries of tokens below seqlens_k[b]
+ *                are read; a page id outside [0, num_pages) reads as zeros
+ *                and is reported as ATTN_ERR_DEVICE_RANGE.
+ *   max_seqlen_q an upper bound of every Sq_b (sizes the grid).
+ *   causal       query i sees key j iff j <= i + (seqlens_k[b] - Sq_b); a row
+ *                that sees no key gets O = 0, LSE = -inf.
+ * Supported: d_qk == d_v in {32, 64, 128}; n_q / n_kv a power of two <= 256;
+ * page_size 16, 32, 64 or a power of two >= 128; B <= 65535. Malformed
+ * cu_seqlens_q entries skip the sequence and are reported as
+ * ATTN_ERR_DEVICE_RANGE. Returns ATTN_OK or an error code (nothing launched
+ * on error).
+ */
+int attn_fwd_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
+                   const int32_t *cu_seqlens_q, const int32_t *seqlens_k, void *o, float *lse,
+                   int B, int max_seqlen_q, int total_q, int n_q, int n_kv, int d_qk, int d_v,
+                   int page_size, int pages_per_seq, int num_pages,
+                   int64_t k_stride_page, int64_t k_stride_token, int64_t k_stride_head,
+                   int64_t v_stride_page, int64_t v_stride_token, int64_t v_stride_head,
+                   int causal, float scale, attn_stream_t stream);
+
+/*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
  * memory.
  *

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_fp8.restype = _i
         L.attn_decode_paged.argtypes = ([_vp] * 7 + [_i] * 8 + [_i64] * 6 +
                                         [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_fwd_paged.argtypes = [_vp] * 8 + [_i] * 10 + [_i64] * 6 + [_i, ctypes.c_float, _vp]
+        L.attn_fwd_paged.restype = _i
         L.attn_decode_paged.restype = _i
         L.attn_rope_tables.argtypes = [_vp, _vp, _i, _i, ctypes.c_double, _vp]
         L.attn_rope_tables.restype = _i
@@ -309,6 +311,37 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float, o
                                  _ptr(lse), B, n_q, n_kv, d, d, page_size, pages_per_seq, num_pages, *ks, *vs,
                                  float(scale), _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_decode_paged")
+    return o, lse
+
+
+def attn_fwd_paged(q, k_pages, v_pages, block_table, cu_seqlens_q, seqlens_k, max_seqlen_q: int, causal: bool,
+                   scale: float, o=None, lse=None, stream=None, want_lse=True):
+    """Prefill of a packed batch against a paged cache. q [total_q,n_q,d] bf16
+    contiguous; k_pages/v_pages indexed [page, token in page, kv head, dim]
+    (any strides with a unit inner stride); block_table int32 [B,
+    pages_per_seq], cu_seqlens_q int32 [B+1] and seqlens_k int32 [B] on the
+    device. Returns (o [total_q,n_q,d] bf16, lse [n_q,total_q] fp32 or None)."""
+    total_q, n_q, d = q.shape
+    num_pages, page_size, n_kv, d_k = k_pages.shape
+    B, pages_per_seq = block_table.shape
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    for t in (block_table, cu_seqlens_q, seqlens_k):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("block_table, cu_seqlens_q and seqlens_k must be contiguous int32 CUDA tensors")
+    if cu_seqlens_q.numel() != B + 1 or seqlens_k.numel() != B:
+        raise ValueError("cu_seqlens_q needs B + 1 offsets and seqlens_k B lengths")
+    ks, vs = _elem_strides(k_pages), _elem_strides(v_pages)
+    d_v = v_pages.shape[3]
+    if o is None:
+        o = torch.empty((total_q, n_q, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((n_q, total_q), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(cu_seqlens_q),
+                              _ptr(seqlens_k), _ptr(o), _ptr(lse), B, int(max_seqlen_q), total_q, n_q, n_kv, d, d_v,
+                              page_size, pages_per_seq, num_pages, *ks, *vs, int(bool(causal)), float(scale),
+                              ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_fwd_paged")
     return o, lse
 
 

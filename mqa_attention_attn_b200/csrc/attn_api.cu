@@ -110,6 +110,11 @@ int sm_count() {
 struct VarlenArgs {
     const int32_t *cu_q, *cu_k;
     int max_q, total_q, total_k;
+    // paged keys and values (attn_fwd_paged): cu_k is unused, the pools are
+    // [page][token][kv head][dim] with these element strides
+    const int32_t *block_table = nullptr, *seqlens_k = nullptr;
+    int page_size = 0, pages_per_seq = 0, num_pages = 0;
+    int64_t ks[3] = {0, 0, 0}, vs[3] = {0, 0, 0};   // page, token, head
 };
 
 template <int D>
@@ -117,6 +122,7 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
                    int n_q, int n_kv, int causal, float scale, cudaStream_t stream, const VarlenArgs *vl = nullptr,
                    int window = 0, int n_sink = 0, const attn::rope::Tables *rope = nullptr) {
     using attn::pf::kDense;
+    using attn::pf::kPaged;
     using attn::pf::kRope;
     using attn::pf::kVarlen;
     using attn::pf::kWindow;
@@ -160,12 +166,30 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         const uint32_t qb[3] = {(uint32_t)C::BOXD, (uint32_t)p.Ht, (uint32_t)p.Pt};
         if (!make_map(&tq, q, 3, qd, qs, qb, C::ROWB)) return ATTN_ERR_CUDA;
         if (!make_map(&to, o, 3, qd, qs, qb, C::ROWB)) return ATTN_ERR_CUDA;
-        // k, v [total_k][n_kv][D]: box = BOXD dims x 1 head x BN keys
-        const uint64_t kd[3] = {(uint64_t)D, (uint64_t)n_kv, (uint64_t)vl->total_k};
-        const uint64_t ks[2] = {(uint64_t)D * 2, (uint64_t)n_kv * D * 2};
-        const uint32_t kb[3] = {(uint32_t)C::BOXD, 1u, (uint32_t)attn::pf::BN};
-        if (!make_map(&tk, k, 3, kd, ks, kb, C::ROWB)) return ATTN_ERR_CUDA;
-        if (!make_map(&tv, v, 3, kd, ks, kb, C::ROWB)) return ATTN_ERR_CUDA;
+        if (vl->block_table) {
+            // page pools [page][token][kv head][D]: box = BOXD dims x box_rows tokens
+            p.block_table = vl->block_table;
+            p.seqlens_k = vl->seqlens_k;
+            p.pages_per_seq = vl->pages_per_seq;
+            p.num_pages = vl->num_pages;
+            int shift = 0;
+            while ((1 << shift) < vl->page_size) ++shift;
+            p.page_shift = shift;
+            p.box_rows = vl->page_size < attn::pf::BN ? vl->page_size : attn::pf::BN;
+            const uint64_t pd[4] = {(uint64_t)D, (uint64_t)vl->page_size, (uint64_t)n_kv, (uint64_t)vl->num_pages};
+            const uint32_t pbx[4] = {(uint32_t)C::BOXD, (uint32_t)p.box_rows, 1u, 1u};
+            const uint64_t kst[3] = {(uint64_t)vl->ks[1] * 2, (uint64_t)vl->ks[2] * 2, (uint64_t)vl->ks[0] * 2};
+            const uint64_t vst[3] = {(uint64_t)vl->vs[1] * 2, (uint64_t)vl->vs[2] * 2, (uint64_t)vl->vs[0] * 2};
+            if (!make_map(&tk, k, 4, pd, kst, pbx, C::ROWB)) return ATTN_ERR_CUDA;
+            if (!make_map(&tv, v, 4, pd, vst, pbx, C::ROWB)) return ATTN_ERR_CUDA;
+        } else {
+            // k, v [total_k][n_kv][D]: box = BOXD dims x 1 head x BN keys
+            const uint64_t kd[3] = {(uint64_t)D, (uint64_t)n_kv, (uint64_t)vl->total_k};
+            const uint64_t ks[2] = {(uint64_t)D * 2, (uint64_t)n_kv * D * 2};
+            const uint32_t kb[3] = {(uint32_t)C::BOXD, 1u, (uint32_t)attn::pf::BN};
+            if (!make_map(&tk, k, 3, kd, ks, kb, C::ROWB)) return ATTN_ERR_CUDA;
+            if (!make_map(&tv, v, 3, kd, ks, kb, C::ROWB)) return ATTN_ERR_CUDA;
+        }
     } else {
         {
             const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * n_q};
@@ -185,8 +209,9 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     const size_t smem = attn::pf::smem_bytes<D>();
     static std::atomic<uint64_t> attr_done{0};  // per template instance, one bit per device
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kDense>, smem, attr_done)) return ATTN_ERR_CUDA;
-    static std::atomic<uint64_t> attr_done_v{0}, attr_done_w{0}, attr_done_r{0};
+    static std::atomic<uint64_t> attr_done_v{0}, attr_done_w{0}, attr_done_r{0}, attr_done_p{0};
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kVarlen>, smem, attr_done_v)) return ATTN_ERR_CUDA;
+    if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kPaged>, smem, attr_done_p)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kWindow>, smem, attr_done_w)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kRope>, smem, attr_done_r)) return ATTN_ERR_CUDA;
     // The kernel rebalances registers between warpgroups (setmaxnreg); that is
@@ -195,13 +220,15 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     static std::atomic<int> regs_checked{0};   // 0: not yet checked, 1: ok, -1: mismatch
     if (regs_checked.load(std::memory_order_acquire) == 0) {
         cudaFuncAttributes fa;
-        cudaFuncAttributes fv, fw, fr;
+        cudaFuncAttributes fv, fw, fr, fp;
         if (cudaFuncGetAttributes(&fa, attn::pf::prefill_kernel<D, kDense>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fv, attn::pf::prefill_kernel<D, kVarlen>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fw, attn::pf::prefill_kernel<D, kWindow>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fr, attn::pf::prefill_kernel<D, kRope>) != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaFuncGetAttributes(&fp, attn::pf::prefill_kernel<D, kPaged>) != cudaSuccess) return ATTN_ERR_CUDA;
         regs_checked.store((fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs &&
-                            fw.numRegs == attn::pf::kLaunchRegs && fr.numRegs == attn::pf::kLaunchRegs) ? 1 : -1,
+                            fw.numRegs == attn::pf::kLaunchRegs && fr.numRegs == attn::pf::kLaunchRegs &&
+                            fp.numRegs == attn::pf::kLaunchRegs) ? 1 : -1,
                            std::memory_order_release);
     }
     if (regs_checked.load(std::memory_order_acquire) < 0) return ATTN_ERR_UNSUPPORTED;
@@ -210,8 +237,12 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         const long long gx = (long long)p.n_pb * n_kv;
         if (gx <= 0 || B <= 0) return ATTN_OK;
         if (gx > 0x7fffffffLL || B > 65535) return ATTN_ERR_UNSUPPORTED;
-        attn::pf::prefill_kernel<D, kVarlen><<<dim3((unsigned)gx, (unsigned)B), attn::pf::THREADS, smem, stream>>>(
-            tq, tk, tv, to, p);
+        if (vl->block_table)
+            attn::pf::prefill_kernel<D, kPaged><<<dim3((unsigned)gx, (unsigned)B), attn::pf::THREADS, smem, stream>>>(
+                tq, tk, tv, to, p);
+        else
+            attn::pf::prefill_kernel<D, kVarlen><<<dim3((unsigned)gx, (unsigned)B), attn::pf::THREADS, smem, stream>>>(
+                tq, tk, tv, to, p);
     } else {
         const long long grid = (long long)p.n_pb * B * n_kv;
         if (grid <= 0) return ATTN_OK;
@@ -605,6 +636,50 @@ int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float 
         case 32: return launch_prefill<32>(q, kk, vv, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
         case 64: return launch_prefill<64>(q, kk, vv, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
         default: return launch_prefill<128>(q, kk, vv, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
+    }
+}
+
+int attn_fwd_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
+                   const int32_t *cu_seqlens_q, const int32_t *seqlens_k, void *o, float *lse, int B, int max_seqlen_q,
+                   int total_q, int n_q, int n_kv, int d_qk, int d_v, int page_size, int pages_per_seq, int num_pages,
+                   int64_t k_stride_page, int64_t k_stride_token, int64_t k_stride_head, int64_t v_stride_page,
+                   int64_t v_stride_token, int64_t v_stride_head, int causal, float scale, attn_stream_t stream) {
+    if (B < 0 || max_seqlen_q < 0 || total_q < 0 || n_q < 1 || n_kv < 1 || d_qk < 1 || d_v < 1)
+        return ATTN_ERR_INVALID_ARG;
+    if (n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (page_size < 1 || pages_per_seq < 1 || num_pages < 1) return ATTN_ERR_INVALID_ARG;
+    if ((long long)page_size * pages_per_seq > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    if (k_stride_page < 0 || k_stride_token < 0 || k_stride_head < 0 || v_stride_page < 0 || v_stride_token < 0 ||
+        v_stride_head < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+    if (!q || !o || !k_pages || !v_pages || !block_table || !cu_seqlens_q || !seqlens_k) return ATTN_ERR_INVALID_ARG;
+    if (d_qk != d_v || (d_qk != 32 && d_qk != 64 && d_qk != 128)) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G) || G > 256) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    // a page is whole TMA boxes of up to 128 rows: 16, 32, 64 or a power of two >= 128 tokens
+    if (!(page_size == 16 || page_size == 32 || page_size == 64 || (page_size % 128 == 0 && is_pow2(page_size))))
+        return ATTN_ERR_UNSUPPORTED;
+    if (k_stride_token < d_qk || v_stride_token < d_v) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o) || !aligned16(k_pages) || !aligned16(v_pages)) return ATTN_ERR_MISALIGNED;
+    if ((k_stride_page | k_stride_token | k_stride_head | v_stride_page | v_stride_token | v_stride_head) & 7)
+        return ATTN_ERR_MISALIGNED;
+    VarlenArgs vl{cu_seqlens_q, nullptr, max_seqlen_q, total_q, 1};
+    vl.block_table = block_table;
+    vl.seqlens_k = seqlens_k;
+    vl.page_size = page_size;
+    vl.pages_per_seq = pages_per_seq;
+    vl.num_pages = num_pages;
+    vl.ks[0] = k_stride_page, vl.ks[1] = k_stride_token, vl.ks[2] = k_stride_head;
+    vl.vs[0] = v_stride_page, vl.vs[1] = v_stride_token, vl.vs[2] = v_stride_head;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (d_qk) {
+        case 32: return launch_prefill<32>(q, k_pages, v_pages, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
+        case 64: return launch_prefill<64>(q, k_pages, v_pages, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
+        default: return launch_prefill<128>(q, k_pages, v_pages, o, lse, B, 0, 0, n_q, n_kv, causal, scale, s, &vl);
     }
 }
 

@@ -109,6 +109,7 @@ struct Smem {
     uint64_t p_full[2][kPChunks];  // one per hand-off chunk of P
     uint64_t o_done[2];
     uint64_t mma_done;
+    uint64_t v_tail;               // PAGED: the copy of the tile holding the last key (cleared past it)
     uint64_t q_rot[2];             // ROPE: Q tile t rotated in place
     uint32_t tmem_base;
     int abort_flag;
@@ -145,6 +146,13 @@ struct Params {
     int window, n_sink;
     // Rotary tables (the ROPE kernel): cos/sin [n_pos][D/2], n_pos >= Skv.
     rope::Tables rope;
+    // Paged cache (the PAGED kernel: queries packed as in VARLEN): sequence b
+    // has seqlens_k[b] cached tokens; token j lives in row j % page_size of
+    // page block_table[b * pages_per_seq + j / page_size] of the pools the K
+    // and V tensor maps address ([page][token][kv head][dim]); a 128-key tile
+    // is 128 / box_rows TMA boxes, box_rows = min(page_size, 128).
+    const int32_t *block_table, *seqlens_k;
+    int pages_per_seq, page_shift, box_rows, num_pages;
     __nv_bfloat16 *o;      // varlen: rows of a tile that ends past its sequence are stored directly
 };
 
@@ -162,8 +170,36 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // MODE: kDense (BHSD batch), kVarlen (packed batch), kWindow (BHSD, causal
-// sliding window with sink keys), kRope (BHSD batch, queries rotated here).
-enum : int { kDense = 0, kVarlen = 1, kWindow = 2, kRope = 3 };
+// sliding window with sink keys), kRope (BHSD batch, queries rotated here),
+// kPaged (packed queries, keys and values in a paged cache).
+enum : int { kDense = 0, kVarlen = 1, kWindow = 2, kRope = 3, kPaged = 4 };
+
+// One 128-key tile of a paged K or V pool into shared memory (the PAGED
+// kernel): box x of the tile holds keys key0 + x * box_rows .. + box_rows - 1,
+// read from their page through the block table. Boxes at or past the
+// sequence's length read an out-of-range page, which TMA fills with zeros,
+// so every row of the tile holds finite values (rows past the length get
+// weight 0, and 0 * NaN would not be 0); a page id outside the pool reads as
+// zeros too and is reported. The barrier expects the whole tile.
+template <int NBOX, int BOXD, int KBOX, int ROWB>
+__device__ __forceinline__ void load_paged_tile(uint32_t dst, const CUtensorMap *tm, uint32_t bar, const Params &p,
+                                                int b, int kvh, int key0, int Skv) {
+    const int nbox = BN / p.box_rows;
+    const uint32_t box_bytes = (uint32_t)p.box_rows * ROWB;
+    const int32_t *row_pages = p.block_table + (size_t)b * p.pages_per_seq;
+    for (int x = 0; x < nbox; ++x) {
+        const int key = key0 + x * p.box_rows;
+        int page = p.num_pages;                        // past the length: zeros
+        if (key < Skv) {
+            page = row_pages[key >> p.page_shift];
+            if ((unsigned)page >= (unsigned)p.num_pages) atomicOr(&g_status, kStatusRange);
+        }
+        const int prow = key & ((1 << p.page_shift) - 1);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_4d(dst + bx * KBOX + x * box_bytes, tm, bar, bx * BOXD, prow, kvh, page);
+    }
+}
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -172,6 +208,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const Params p) {
     using C = Cfg<D>;
     constexpr bool VARLEN = MODE == kVarlen;
+    constexpr bool PAGED = MODE == kPaged;
+    constexpr bool PACKED = VARLEN || PAGED;      // queries packed [total_q][n_q][D]
     constexpr bool WINDOW = MODE == kWindow;
     constexpr bool ROPE = MODE == kRope;
     extern __shared__ uint8_t smem_raw[];
@@ -182,16 +220,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ---- work unit: (b, kv head, position block), heaviest causal blocks first
     int b, kvh, pb;
     int Sq = p.Sq, Skv = p.Skv, q0 = 0, k0 = 0;   // this sequence's sizes and first rows (varlen)
-    if (VARLEN) {
+    if (PACKED) {
         b = blockIdx.y;
         kvh = blockIdx.x % p.n_kv;
         pb = p.n_pb - 1 - (int)(blockIdx.x / p.n_kv);
         q0 = p.cu_q[b];
-        k0 = p.cu_k[b];
         Sq = p.cu_q[b + 1] - q0;
-        Skv = p.cu_k[b + 1] - k0;
-        if (q0 < 0 || k0 < 0 || Sq < 0 || Skv < 0 || q0 + Sq > p.total_q || k0 + Skv > p.total_k ||
-            Sq > p.n_pb * (p.pair_by_heads ? p.Pt : 2 * p.Pt)) {
+        bool bad = q0 < 0 || Sq < 0 || q0 + Sq > p.total_q || Sq > p.n_pb * (p.pair_by_heads ? p.Pt : 2 * p.Pt);
+        if (VARLEN) {
+            k0 = p.cu_k[b];
+            Skv = p.cu_k[b + 1] - k0;
+            bad = bad || k0 < 0 || Skv < 0 || k0 + Skv > p.total_k;
+        } else {
+            // the cached tokens of the sequence, at most what its pages hold
+            Skv = p.seqlens_k[b];
+            const int cap = p.pages_per_seq << p.page_shift;
+            if (Skv > cap) {
+                if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_status, kStatusRange);
+                Skv = cap;
+            }
+            if (Skv < 0) Skv = 0;
+        }
+        if (bad) {
             if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&g_status, kStatusRange);
             Sq = 0;   // malformed offsets: this sequence is skipped
         }
@@ -250,6 +300,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(smem_u32(&sm.o_done[t]), 1);
         }
         mbar_init(smem_u32(&sm.mma_done), 1);
+        mbar_init(smem_u32(&sm.v_tail), 1);
         for (int t = 0; t < 2; ++t) mbar_init(smem_u32(&sm.q_rot[t]), 128);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -285,7 +336,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int t = 0; t < 2; ++t) {
                 if (nt[t] == 0) continue;
                 for (int bx = 0; bx < C::NBOX; ++bx)
-                    if (VARLEN)
+                    if (PACKED)
                         tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, h0[t],
                                     q0 + p0[t]);
                     else
@@ -306,6 +357,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     break;
                 const uint32_t fb = smem_u32(&sm.k_full[s]);
                 mbar_arrive_expect_tx(fb, C::KBYTES);
+                if (PAGED)
+                    load_paged_tile<C::NBOX, C::BOXD, C::KBOX, C::ROWB>(smem_u32(sm.k[s]), &tm_k, fb, p, b, kvh, j * BN,
+                                                                      Skv);
+                else
                 for (int bx = 0; bx < C::NBOX; ++bx)
                     if (VARLEN)
                         tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, kvh, k0 + j * BN);
@@ -322,8 +377,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
     } else if (warp == 2) {
         // ======================= TMA producer (V tiles) =======================
+        // PAGED: the visited tile that ends past the last cached key (-1: none)
+        const int tail_tile = (PAGED && Skv % BN != 0 && (Skv - 1) / BN < nmax) ? (Skv - 1) / BN : -1;
+        int issued = 0;
         if (lane == 0) {
-            int issued = 0;
             for (int j = 0; j < nmax; ++j) {
                 const int s = j % VSTAGE;
                 // V tile j - VSTAGE is free once iteration j - VSTAGE is released
@@ -331,8 +388,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (j >= VSTAGE &&
                     !mbar_wait(smem_u32(&sm.rel[it % NREL]), (it / NREL) & 1, abort_flag, 0x14))
                     break;
-                const uint32_t fb = smem_u32(&sm.v_full[s]);
+                // PAGED: the tile holding the last key lands on v_tail instead;
+                // v_full of its stage is completed below, after the clearing
+                const uint32_t fb = smem_u32((PAGED && j == tail_tile) ? &sm.v_tail : &sm.v_full[s]);
                 mbar_arrive_expect_tx(fb, C::KBYTES);
+                if (PAGED)
+                    load_paged_tile<C::NBOX, C::BOXD, C::KBOX, C::ROWB>(smem_u32(sm.v[s]), &tm_v, fb, p, b, kvh, j * BN,
+                                                                      Skv);
+                else
                 for (int bx = 0; bx < C::NBOX; ++bx)
                     if (VARLEN)
                         tma_load_3d(smem_u32(sm.v[s]) + bx * C::KBOX, &tm_v, fb, bx * C::BOXD, kvh, k0 + j * BN);
@@ -341,8 +404,36 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                     b * p.n_kv + kvh);
                 ++issued;
             }
+        }
+        issued = __shfl_sync(0xffffffffu, issued, 0);
+        if constexpr (PAGED) {
+            // The tile holding the sequence's last key may hold rows past the
+            // length (a page's unused slots, whatever they contain): they get
+            // weight 0, but 0 * (NaN or Inf) is not 0, so this warp clears
+            // them once the tile has landed, then completes the stage's v_full
+            // (a plain arrival: the copy's bytes were counted on v_tail).
+            const int jt = tail_tile;
+            if (jt >= 0 && jt < issued) {
+                const int s = jt % VSTAGE;
+                const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.v_tail), 0, abort_flag, 0x16));
+                if (ok) {
+                    const int rows = Skv - jt * BN;             // valid rows of the tile
+                    constexpr int CPR = C::ROWB / 16;             // 16-byte chunks per box row
+                    for (int e = rows * CPR + (int)lane; e < BN * CPR; e += 32)
+#pragma unroll
+                        for (int bx = 0; bx < C::NBOX; ++bx)
+                            sts128(smem_u32(sm.v[s]) + bx * C::KBOX + (uint32_t)e * 16u, make_uint4(0u, 0u, 0u, 0u));
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0 && ok) mbar_arrive(smem_u32(&sm.v_full[s]));
+            }
+        }
+        if (lane == 0) {
+            // never leave copies in flight into this CTA's shared memory
             for (int j = issued - 1; j >= 0 && j >= issued - VSTAGE; --j)
-                mbar_wait(smem_u32(&sm.v_full[j % VSTAGE]), (j / VSTAGE) & 1, nullptr, 0x15);
+                mbar_wait(smem_u32((PAGED && j == tail_tile) ? &sm.v_tail : &sm.v_full[j % VSTAGE]),
+                          (PAGED && j == tail_tile) ? 0 : (j / VSTAGE) & 1, nullptr, 0x15);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -369,7 +460,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const uint32_t off_k = (kel / C::BOXD) * C::KBOX + (kel % C::BOXD) * 2;
                     // (the varlen instance builds each descriptor in full: with
                     // the offset form its register allocation spills)
-                    if constexpr (VARLEN)
+                    if constexpr (PACKED)
                         umma_ss(tmem + C::col_s(t), umma_smem_desc(smem_u32(sm.q[t]) + off_q, 16, C::ATOM, C::LAYOUT),
                                 umma_smem_desc(smem_u32(sm.k[s]) + off_k, 16, C::ATOM, C::LAYOUT), idesc_s, ks > 0 ? 1u : 0u);
                     else
@@ -442,8 +533,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t quad = warp & 3u;
         const int r = (int)(quad * 32 + lane);          // row of the tile = TMEM lane
         if (p0[t] < Sq) {
-            const int hl = VARLEN ? r % p.Ht : r / p.Pt;
-            const int pl = VARLEN ? r / p.Ht : r % p.Pt;
+            const int hl = PACKED ? r % p.Ht : r / p.Pt;
+            const int pl = PACKED ? r / p.Ht : r % p.Pt;
             const int pos = p0[t] + pl;
             const int head = h0[t] + hl;
             if constexpr (ROPE) {
@@ -544,7 +635,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // is off by default.
                 // a row with no visible key yet keeps m = -inf: exponentiate
                 // against 0 instead (every p is then 0)
-                const float m_use = ((VARLEN || WINDOW) && m_run == -INFINITY) ? 0.f : m_run;
+                const float m_use = ((PACKED || WINDOW) && m_run == -INFINITY) ? 0.f : m_run;
                 const float2 nm2 = make_float2(-m_use, -m_use);
                 float2 rs = make_float2(0.f, 0.f);
                 // one chunk of exponentials; which pairs take the FMA-pipe
@@ -592,11 +683,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             tc_fence_after();
             // a row that saw no key: O = 0, LSE = -inf (the empty sum)
-            const float inv_l = (!VARLEN || l_run > 0.f) ? 1.f / l_run : 0.f;
+            const float inv_l = (!PACKED || l_run > 0.f) ? 1.f / l_run : 0.f;
             const uint32_t stage = smem_u32(sm.q[t]);
             // varlen: a tile reaching past its sequence's last query is stored
             // row by row (TMA would write into the next sequence's rows)
-            const bool direct = VARLEN && p0[t] + p.Pt > Sq;
+            const bool direct = PACKED && p0[t] + p.Pt > Sq;
             {
                 uint32_t o[D];
                 if (ntt > 0) {
@@ -627,8 +718,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             if (p.lse != nullptr && pos < Sq) {
-                const float lse_v = (!VARLEN || l_run > 0.f) ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
-                if (VARLEN)
+                const float lse_v = (!PACKED || l_run > 0.f) ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+                if (PACKED)
                     p.lse[(size_t)head * p.total_q + q0 + pos] = lse_v;
                 else
                     p.lse[((size_t)b * p.n_q + head) * p.Sq + pos] = lse_v;
@@ -637,7 +728,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             named_bar_sync(2 + t, 128);
             if (r == 0 && ok && !direct) {
                 for (int bx = 0; bx < C::NBOX; ++bx) {
-                    if (VARLEN)
+                    if (PACKED)
                         tma_store_3d(&tm_o, stage + bx * C::QBOX, bx * C::BOXD, h0[t], q0 + p0[t]);
                     else
                         tma_store_3d(&tm_o, stage + bx * C::QBOX, bx * C::BOXD, p0[t], b * p.n_q + h0[t]);

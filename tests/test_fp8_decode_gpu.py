@@ -75,10 +75,12 @@ def test_fp8_decode_nan_past_the_length():
     assert torch.isfinite(o.float()).all()
 
 
-def test_fp8_decode_gqa_workload_sampled_against_bf16_path():
-    """The GQA decode workload quantized to e4m3: equals attn_decode on the
-    dequantized cache (rounded back to bf16, exact for e4m3 values times a
-    power-of-two scale) within the parity tolerances."""
+def test_fp8_decode_gqa_workload_against_oracle_and_bf16_path():
+    """The GQA decode workload quantized to e4m3: every row equals attn_decode
+    on the dequantized cache (rounded back to bf16, exact for e4m3 values
+    times a power-of-two scale) within the parity tolerances, and the rows of
+    four of its sequences (every head, the shortest and longest lengths
+    among them) equal the fp64 oracle on the dequantized cache."""
     binding = need_gpu()
     w = inputs.WORKLOADS["gqa_decode"]
     seqlens, q, kc, vc = inputs.make(w, device="cuda")
@@ -96,6 +98,14 @@ def test_fp8_decode_gqa_workload_sampled_against_bf16_path():
     assert binding.device_status() == 0
     assert float((o8.float() - ob.float()).abs().max()) <= 2e-2
     assert float((l8 - lb).abs().max()) <= 1e-3
+    order = torch.argsort(seqlens)
+    pick = sorted({int(order[0]), int(order[-1]), 1, 2})
+    for b in pick:
+        L = int(seqlens[b])
+        kq = oracle.dequant_e4m3(k8[b:b + 1, :, :L].view(torch.uint8), ks)
+        vq = oracle.dequant_e4m3(v8[b:b + 1, :, :L].view(torch.uint8), vs)
+        o_ref, l_ref = oracle.sdpa(q[b:b + 1, :, None, :], kq, vq, False, w.scale)
+        check_parity(o8[b:b + 1], l8[b:b + 1], o_ref[:, :, 0], l_ref[:, :, 0], f"fp8 gqa_decode sequence {b} (L={L})")
 
 
 def test_fp8_decode_rejects_bad_arguments():
