@@ -19,7 +19,9 @@ refilled before its last reader ran, P overwritten before P V read it, O
 touched while a P V may still run, a wait that can never complete -- raises
 ``Hazard``. The kernels modelled: ``attn::pf::prefill_kernel`` (dense mode:
 two ping-pong query tiles, K ring of 2, V ring of 3, three release
-barriers), ``attn::mla::mla_decode_kernel`` (two issuing threads taking
+barriers; in the paged mode the tile holding the last key landing on its own
+barrier and cleared past the length before its stage counts as full),
+``attn::mla::mla_decode_kernel`` (two issuing threads taking
 even and odd tiles, per-group arrival barriers, the Q staging in ring
 stage 1, the tail clearing) and ``attn::dec::decode_split_kernel``
 (persistent over units, one ring for K then V tiles, two P slots, the
@@ -128,10 +130,12 @@ class Sim:
 # attn::pf::prefill_kernel (dense mode)
 # ---------------------------------------------------------------------------
 KSTAGE, VSTAGE, NREL = 2, 3, 3
-PREFILL_BUGS = ("k_release_early", "v_release_early", "s_before_pv", "no_v_wait", "no_q_rot_wait")
+PREFILL_BUGS = ("k_release_early", "v_release_early", "s_before_pv", "no_v_wait", "no_q_rot_wait",
+                "tail_lands_on_v_full")
 
 
-def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = None, rope: bool = False):
+def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = None, rope: bool = False,
+            paged_tail: bool = False):
     """Tile t visits key tiles 0 .. nt[t]-1 (the second tile may have one
     more, as consecutive position blocks do, or none). With `rope`, each
     softmax warpgroup first rotates its Q tile in place (after Q lands) and
@@ -151,6 +155,8 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
         sim.bar(f"o_done{t}", 1)
         sim.bar(f"q_rot{t}", 1)
     sim.bar("mma_done", 1)
+    sim.bar("v_tail", 1)
+    cleared = set()
     qst = {"landed": False, "rotated": set()}
     kst, vst = {}, {}
     s_done, pv_done, sbuf, pbuf = set(), set(), {}, {}
@@ -178,8 +184,23 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
                     yield from sim.wait(f"rel{it % NREL}", (it // NREL) & 1)
                 for t in range(2):
                     check(j - VSTAGE >= nt[t] or (t, j - VSTAGE) in pv_done, "V stage refilled early", j)
-            sim.load(f"v_full{s}", lambda s=s, j=j: vst.__setitem__(s, j))
+            if paged_tail and j == nmax - 1 and bug != "tail_lands_on_v_full":
+                # the tile holding the last key lands on v_tail; its rows past
+                # the length are cleared before v_full of the stage completes
+                sim.load("v_tail", lambda s=s, j=j: vst.__setitem__(s, j))
+            else:
+                sim.load(f"v_full{s}", lambda s=s, j=j: vst.__setitem__(s, j))
             yield
+        if paged_tail and nmax > 0:
+            st = (nmax - 1) % VSTAGE
+            if bug == "tail_lands_on_v_full":
+                yield from sim.wait(f"v_full{st}", ((nmax - 1) // VSTAGE) & 1)
+            else:
+                yield from sim.wait("v_tail", 0)
+            check(vst.get(st) == nmax - 1, "tail cleared before it landed")
+            cleared.add(nmax - 1)
+            if bug != "tail_lands_on_v_full":
+                sim.bars[f"v_full{st}"].arrive()
 
     def issue_s(t, j):
         def ex():
@@ -196,6 +217,7 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
         def ex():
             check(pbuf.get(t) == j, "P V reads the wrong P", t, j)
             check(vst.get(j % VSTAGE) == j, "P V reads the wrong V tile", t, j)
+            check(not paged_tail or j != nmax - 1 or j in cleared, "P V reads an uncleared tail tile", t, j)
             pv_done.add((t, j))
         sim.mma("mma", ex)
         if j == nt[t] - 1:

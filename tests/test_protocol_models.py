@@ -16,11 +16,11 @@ def _cases_prefill():
     yield (0, 1)
 
 
-@pytest.mark.parametrize("rope", [False, True])
-def test_prefill_protocol_hazard_free(rope):
+@pytest.mark.parametrize("rope,paged_tail", [(False, False), (True, False), (False, True)])
+def test_prefill_protocol_hazard_free(rope, paged_tail):
     for nt in _cases_prefill():
         for seed in range(40):
-            pm.prefill(nt, seed, rescale_p=(0.0, 0.3, 1.0)[seed % 3], rope=rope)
+            pm.prefill(nt, seed, rescale_p=(0.0, 0.3, 1.0)[seed % 3], rope=rope, paged_tail=paged_tail)
 
 
 @pytest.mark.parametrize("bug", pm.PREFILL_BUGS)
@@ -28,7 +28,7 @@ def test_prefill_planted_bug_is_caught(bug):
     with pytest.raises(pm.Hazard):
         for nt in _cases_prefill():
             for seed in range(40):
-                pm.prefill(nt, seed, rescale_p=0.5, bug=bug, rope=True)
+                pm.prefill(nt, seed, rescale_p=0.5, bug=bug, rope=True, paged_tail=True)
 
 
 def test_mla_protocol_hazard_free():
