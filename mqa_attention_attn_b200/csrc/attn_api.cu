@@ -141,6 +141,7 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     p.window = window;
     p.n_sink = n_sink;
     if (rope) p.rope = *rope;
+    p.o = reinterpret_cast<__nv_bfloat16 *>(o);
     const int Sq_plan = vl ? vl->max_q : Sq;   // position blocks cover the longest sequence
     if (G >= 2) {
         p.Ht = G / 2;
@@ -247,6 +248,9 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         const long long grid = (long long)p.n_pb * B * n_kv;
         if (grid <= 0) return ATTN_OK;
         if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+        // one CTA per SM: the CTA one wave later gets its Q tiles prefetched
+        const int n_sm = sm_count();
+        p.l2_ahead = (n_sm > 0 && grid > n_sm) ? n_sm : 0;
         if (rope) {
             // launched as a programmatic dependent of the key rotation: the
             // prologue (barriers, TMEM, Q load and rotation) overlaps it and

@@ -73,6 +73,20 @@ constexpr int kPChunks = ATTN_PF_P_CHUNKS;
 constexpr int kPolyEvery = ATTN_PF_POLY_EVERY;
 constexpr int kChunkKeys = BN / kPChunks;
 static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P hand-off chunks");
+#ifndef ATTN_PF_EARLY_LOADS
+#define ATTN_PF_EARLY_LOADS 1
+#endif
+#ifndef ATTN_PF_L2_PREFETCH
+#define ATTN_PF_L2_PREFETCH 1
+#endif
+// kEarlyLoads: the thread that initialises the barriers issues the Q tiles and
+// the first K tiles at once, before the block-wide setup barrier and the TMEM
+// allocation. kL2Prefetch: it also prefetches into L2 the Q tiles of the CTA
+// one wave later (dense batches). Measured on B200 at the Llama-3-8B prefill
+// shape, the two take 3 % off the kernel time; storing O straight from
+// registers instead of through shared memory and a TMA store was slower.
+constexpr bool kEarlyLoads = ATTN_PF_EARLY_LOADS != 0;
+constexpr bool kL2Prefetch = ATTN_PF_L2_PREFETCH != 0;
 constexpr int kLaunchRegs = 168;            // registers per thread the kernel must be built with
 constexpr int kRegsLow = 56;               // producer / MMA warpgroup after setmaxnreg.dec
 constexpr int kRegsHigh = 224;              // softmax warpgroups after setmaxnreg.inc
@@ -154,6 +168,10 @@ struct Params {
     const int32_t *block_table, *seqlens_k;
     int pages_per_seq, page_shift, box_rows, num_pages;
     __nv_bfloat16 *o;      // varlen: rows of a tile that ends past its sequence are stored directly
+    // Dense batch: the CTA this many launch slots later has its Q tiles
+    // prefetched into L2 by this one (0: none). With one CTA per SM and the
+    // grid taken in index order, that CTA starts once this wave drains.
+    int l2_ahead;
 };
 
 template <bool B>
@@ -252,16 +270,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         b = bh / p.n_kv;
         kvh = bh % p.n_kv;
     }
+    // query tile t of a unit: first head and first position
+    auto tile_origin = [&](int kvh_, int pb_, int t, int &h0_, int &p0_) {
+        if (p.pair_by_heads) {
+            h0_ = kvh_ * p.G + t * p.Ht;
+            p0_ = pb_ * p.Pt;
+        } else {
+            h0_ = kvh_;  // G == 1: query head == KV head
+            p0_ = pb_ * 2 * p.Pt + t * p.Pt;
+        }
+    };
     int h0[2], p0[2], nt[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        if (p.pair_by_heads) {
-            h0[t] = kvh * p.G + t * p.Ht;
-            p0[t] = pb * p.Pt;
-        } else {
-            h0[t] = kvh;  // G == 1: query head == KV head
-            p0[t] = pb * 2 * p.Pt + t * p.Pt;
-        }
+        tile_origin(kvh, pb, t, h0[t], p0[t]);
         if (p0[t] >= Sq) {
             nt[t] = 0;
         } else {
@@ -286,6 +308,47 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto key_tile = [&](int j) { return (WINDOW && j >= nsk) ? jw0 + (j - nsk) : j; };
     const int nmax = max(nt[0], nt[1]);
 
+    // Q tiles of this unit, all on q_full
+    auto load_q = [&]() {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_o);
+        uint32_t qbytes = 0;
+        for (int t = 0; t < 2; ++t)
+            if (nt[t] > 0) qbytes += C::QBYTES;
+        const uint32_t qbar = smem_u32(&sm.q_full);
+        mbar_arrive_expect_tx(qbar, qbytes);
+        for (int t = 0; t < 2; ++t) {
+            if (nt[t] == 0) continue;
+            for (int bx = 0; bx < C::NBOX; ++bx)
+                if (PACKED)
+                    tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, h0[t], q0 + p0[t]);
+                else
+                    tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
+                                b * p.n_q + h0[t]);
+        }
+    };
+    // K tile of iteration j into its stage (the stage must be free)
+    auto load_k = [&](int j) {
+        const int s = j % KSTAGE;
+        const uint32_t fb = smem_u32(&sm.k_full[s]);
+        mbar_arrive_expect_tx(fb, C::KBYTES);
+        if (PAGED)
+            load_paged_tile<C::NBOX, C::BOXD, C::KBOX, C::ROWB>(smem_u32(sm.k[s]), &tm_k, fb, p, b, kvh, j * BN, Skv);
+        else
+            for (int bx = 0; bx < C::NBOX; ++bx)
+                if (VARLEN)
+                    tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, kvh, k0 + j * BN);
+                else
+                    tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, key_tile(j) * BN,
+                                b * p.n_kv + kvh);
+    };
+    // K tiles issued during setup (ROPE: the rotated keys come from the grid
+    // launched just before this one, so its K tiles wait in the producer;
+    // PAGED: the page lookups issued here spill in the producer's registers)
+    const int k_early = (kEarlyLoads && !ROPE && !PAGED) ? min(KSTAGE, nmax) : 0;
+
     // ---- setup: barriers (warp 0), TMEM (warp 1)
     if (warp == 0 && lane == 0) {
         mbar_init(smem_u32(&sm.q_full), 1);
@@ -304,6 +367,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int t = 0; t < 2; ++t) mbar_init(smem_u32(&sm.q_rot[t]), 128);
         sm.abort_flag = 0;
         fence_mbar_init();
+        if constexpr (kEarlyLoads) {
+            load_q();
+            for (int j = 0; j < k_early; ++j) load_k(j);
+        }
+        if (kL2Prefetch && !PACKED && p.l2_ahead > 0 && blockIdx.x + (unsigned)p.l2_ahead < gridDim.x) {
+            // Q tiles of a unit that starts later, into L2
+            const unsigned f = blockIdx.x + (unsigned)p.l2_ahead;
+            const int nbh = p.B * p.n_kv;
+            const int fbh = (int)(f % (unsigned)nbh);
+            const int fpb = p.n_pb - 1 - (int)(f / (unsigned)nbh);
+            for (int t = 0; t < 2; ++t) {
+                int fh0, fp0;
+                tile_origin(fbh % p.n_kv, fpb, t, fh0, fp0);
+                if (fp0 >= Sq) continue;
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_prefetch_l2_3d(&tm_q, bx * C::BOXD, fp0, (fbh / p.n_kv) * p.n_q + fh0);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm.tmem_base), C::TMEM_COLS);
@@ -324,49 +405,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == 0) {
         // ======================= TMA producer =======================
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            tma_prefetch_desc(&tm_o);
-            uint32_t qbytes = 0;
-            for (int t = 0; t < 2; ++t)
-                if (nt[t] > 0) qbytes += C::QBYTES;
             const uint32_t qbar = smem_u32(&sm.q_full);
-            mbar_arrive_expect_tx(qbar, qbytes);
-            for (int t = 0; t < 2; ++t) {
-                if (nt[t] == 0) continue;
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    if (PACKED)
-                        tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, h0[t],
-                                    q0 + p0[t]);
-                    else
-                        tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, p0[t],
-                                    b * p.n_q + h0[t]);
-            }
+            if constexpr (!kEarlyLoads) load_q();
             // K tiles (V tiles are loaded by warp 2). ROPE: the rotated keys come
             // from the grid launched just before this one
             if (ROPE) griddep_wait();
-            int issued = 0;
-            for (int j = 0; j < nmax; ++j) {
-                const int s = j % KSTAGE;
+            int issued = k_early;
+            for (int j = k_early; j < nmax; ++j) {
                 // K tile j - KSTAGE is free once iteration j - KSTAGE - 1 is released
                 // (K tile 0 with iteration 0)
                 const int it = j - KSTAGE - 1 < 0 ? 0 : j - KSTAGE - 1;
                 if (j >= KSTAGE &&
                     !mbar_wait(smem_u32(&sm.rel[it % NREL]), (it / NREL) & 1, abort_flag, 0x11))
                     break;
-                const uint32_t fb = smem_u32(&sm.k_full[s]);
-                mbar_arrive_expect_tx(fb, C::KBYTES);
-                if (PAGED)
-                    load_paged_tile<C::NBOX, C::BOXD, C::KBOX, C::ROWB>(smem_u32(sm.k[s]), &tm_k, fb, p, b, kvh, j * BN,
-                                                                      Skv);
-                else
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    if (VARLEN)
-                        tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, kvh, k0 + j * BN);
-                    else
-                        tma_load_3d(smem_u32(sm.k[s]) + bx * C::KBOX, &tm_k, fb, bx * C::BOXD, key_tile(j) * BN,
-                                    b * p.n_kv + kvh);
+                load_k(j);
                 ++issued;
             }
             // never leave copies in flight into this CTA's shared memory
