@@ -50,8 +50,14 @@ constexpr int NBS = NB - NBT;     // Q boxes 4-8 (columns 256-575) in shared mem
 constexpr int QBOX = M * 128;     // one 64-column box of Q: 128 rows x 128 B
 constexpr int KBOX = KT * 128;    // one 64-column box of a key tile: 64 rows x 128 B
 constexpr int NSTAGE = 2;
-constexpr int NG = 3;             // arrival groups of a ring stage: boxes 0-2, 3-5, 6-8
-constexpr int THREADS = 256;      // warp 0 TMA, warps 1-2 MMAs (even / odd tiles), warps 4-7 softmax
+// A ring stage is filled in two groups with their own barriers: group A, the
+// boxes only the score MMAs read (for CTA r: the five boxes outside its value
+// columns 256r .. 256r+255), freed once the tile's score MMAs complete, and
+// group B, its four value boxes 4r .. 4r+3, freed once the tile's P.V
+// completes. Group A of tile j+2 so loads while tile j's softmax and P.V run.
+constexpr int NA = 5, NBV = 4;    // boxes of group A and of group B
+constexpr int THREADS = 256;      // warp 0 TMA (group A), warps 1-2 MMAs (even / odd tiles), warp 3 TMA
+                                  // (group B), warps 4-7 softmax
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_S1 = 64;   // S double buffer (P over its first half)
@@ -62,7 +68,7 @@ struct Smem {
     uint8_t q[NBS][QBOX];                  // 80 KB
     uint8_t k[NSTAGE][NB][KBOX];           // 144 KB; stage 1 first stages Q boxes 0-3
     uint64_t q_full;
-    uint64_t kv_full[NSTAGE][NG], kv_empty[NSTAGE];
+    uint64_t kv_full[NSTAGE][2], kv_empty[NSTAGE][2];   // [stage][group A, group B]
     uint64_t s_full[2], p_full[2];
     uint64_t s_done[2];                    // every MMA of issuing thread t has completed
     uint64_t qt_ready;                     // Q columns 0-255 copied into TMEM
@@ -123,8 +129,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) {
         mbar_init(smem_u32(&sm.q_full), 1);
         for (int s = 0; s < NSTAGE; ++s) {
-            for (int g = 0; g < NG; ++g) mbar_init(smem_u32(&sm.kv_full[s][g]), 1);
-            mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+            for (int g = 0; g < 2; ++g) {
+                mbar_init(smem_u32(&sm.kv_full[s][g]), 1);
+                mbar_init(smem_u32(&sm.kv_empty[s][g]), 1);
+            }
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.s_full[i]), 1);
@@ -150,51 +158,57 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort_flag;
 
-    if (warp == 0) {
-        // ======================= TMA producer =======================
+    // box bx of a 576-column row belongs to group B of this CTA iff it is one
+    // of its value boxes
+    auto box_of = [rank](int g, int i) -> int {
+        // group A: the other CTA's value boxes, then box 8; group B: own value boxes
+        return g == 0 ? (i < NBV ? 4 * (1 - (int)rank) + i : 8) : 4 * (int)rank + i;
+    };
+    if (warp == 0 || warp == 3) {
+        // ============ TMA producers: warp 0 group A (and Q), warp 3 group B ============
+        const int g = warp == 0 ? 0 : 1;
+        const int nbox = g == 0 ? NA : NBV;
         if (lane == 0 && nt > 0) {
-            tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_c);
-            // Q: boxes 4-8 to their home, boxes 0-3 staged in ring stage 1
             const uint32_t qbar = smem_u32(&sm.q_full);
-            mbar_arrive_expect_tx(qbar, (uint32_t)(NB * QBOX));
-            for (int bx = 0; bx < NB; ++bx) {
-                const uint32_t dst = bx < NBT ? smem_u32(sm.k[1][0]) + bx * QBOX : smem_u32(sm.q[bx - NBT]);
-                tma_load_3d(dst, &tm_q, qbar, 64 * bx, hb * M, b);
+            if (g == 0) {
+                tma_prefetch_desc(&tm_q);
+                // Q: boxes 4-8 to their home, boxes 0-3 staged in ring stage 1
+                mbar_arrive_expect_tx(qbar, (uint32_t)(NB * QBOX));
+                for (int bx = 0; bx < NB; ++bx) {
+                    const uint32_t dst = bx < NBT ? smem_u32(sm.k[1][0]) + bx * QBOX : smem_u32(sm.q[bx - NBT]);
+                    tma_load_3d(dst, &tm_q, qbar, 64 * bx, hb * M, b);
+                }
             }
             bool ok = true;
             int issued = 0;
             for (int j = 0; ok && j < nt; ++j) {
                 const int s = j % NSTAGE;
-                if (j == 1) ok = mbar_wait(smem_u32(&sm.qt_ready), 0, abort_flag, 0x410);  // staging free
+                // Q boxes 0-3 (4 x 16 KB) are staged over boxes 0-7 of stage 1
+                if (j == 1) ok = mbar_wait(smem_u32(&sm.qt_ready), 0, abort_flag, 0x410);
                 if (ok && j >= NSTAGE)
-                    ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((j / NSTAGE) + 1) & 1, abort_flag, 0x411);
+                    ok = mbar_wait(smem_u32(&sm.kv_empty[s][g]), ((j / NSTAGE) + 1) & 1, abort_flag, 0x411);
                 if (!ok) break;
-                // one barrier per group of three boxes, so that the score MMAs
-                // of a group start while the later groups are still in flight
-                for (int g = 0; g < NG; ++g) {
-                    const uint32_t fb = smem_u32(&sm.kv_full[s][g]);
-                    mbar_arrive_expect_tx(fb, (uint32_t)(NB / NG * KBOX));
-                    for (int bx = g * (NB / NG); bx < (g + 1) * (NB / NG); ++bx)
-                        tma_load_3d(smem_u32(sm.k[s][bx]), &tm_c, fb, 64 * bx, key0 + j * KT, b);
+                const uint32_t fb = smem_u32(&sm.kv_full[s][g]);
+                mbar_arrive_expect_tx(fb, (uint32_t)(nbox * KBOX));
+                for (int i = 0; i < nbox; ++i) {
+                    const int bx = box_of(g, i);
+                    tma_load_3d(smem_u32(sm.k[s][bx]), &tm_c, fb, 64 * bx, key0 + j * KT, b);
                 }
                 ++issued;
             }
-            mbar_wait(qbar, 0, nullptr, 0x412);
+            if (g == 0) mbar_wait(qbar, 0, nullptr, 0x412);
             for (int j = issued - 1; j >= 0 && j >= issued - NSTAGE; --j)
-                for (int g = 0; g < NG; ++g)
-                    mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE][g]), (j / NSTAGE) & 1, nullptr, 0x413);
+                mbar_wait(smem_u32(&sm.kv_full[j % NSTAGE][g]), (j / NSTAGE) & 1, nullptr, 0x413);
         }
         __syncwarp();
-        if (tail < KT) {
+        if (g == 1 && tail < KT) {
             // Rows past the length get weight 0, but 0 * (NaN or Inf) is not
             // 0: clear this CTA's value columns of those rows so that whatever
             // the cache holds there cannot reach the output. Done before the
-            // last tile's MMAs are issued (they wait for tail_ready).
+            // last tile's group-B score MMAs are issued (they wait for tail_ready).
             const int s = (nt - 1) % NSTAGE;
-            bool ok = true;
-            for (int g = 0; ok && g < NG; ++g)
-                ok = mbar_wait(smem_u32(&sm.kv_full[s][g]), ((nt - 1) / NSTAGE) & 1, abort_flag, 0x414);
+            bool ok = mbar_wait(smem_u32(&sm.kv_full[s][1]), ((nt - 1) / NSTAGE) & 1, abort_flag, 0x414);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 for (int e = tail * 8 + (int)lane; e < KT * 8; e += 32) {
@@ -232,33 +246,55 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int s = j % NSTAGE;   // == par
                 const uint32_t ph = (uint32_t)(j / NSTAGE) & 1u;
                 ok = mbar_wait(smem_u32(&sm.kv_full[s][0]), ph, abort_flag, 0x422);
-                if (ok && j == nt - 1 && tail < KT) ok = mbar_wait(smem_u32(&sm.tail_ready), 0, abort_flag, 0x426);
                 if (!ok) break;
                 tc_fence_after();
                 // the 36 score MMAs fully unrolled, each descriptor the tile's (or
                 // Q's) base descriptor plus a constant offset in its 16-byte
                 // address field (at N = 64 an MMA finishes in fewer cycles than
-                // a loop iteration of the issuing thread would take); boxes
-                // 3-5 and 6-8 are waited for just before their MMAs
+                // a loop iteration of the issuing thread would take): group A's
+                // boxes first, then, once they have landed, group B's. The two
+                // CTAs add the nine boxes in different orders, so their scores
+                // may differ in the last bits; each normalises its own half of
+                // O by its own sums, and the LSE is the first CTA's.
                 const uint64_t kd0 = umma_smem_desc(smem_u32(sm.k[s][0]), 16, 1024, 2);
-#pragma unroll
-                for (int bx = 0; bx < NB; ++bx) {
-                    if (bx > 0 && bx % (NB / NG) == 0) {
-                        ok = mbar_wait(smem_u32(&sm.kv_full[s][bx / (NB / NG)]), ph, abort_flag, 0x429);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
+                auto score_box = [&](int bx, bool first) {
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         if (bx < NBT)
                             umma_ts(dcol, tmem + COL_QT + 32 * bx + 8 * k4, kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4),
-                                    idesc_s, (bx > 0 || k4 > 0) ? 1u : 0u);
+                                    idesc_s, (first && k4 == 0) ? 0u : 1u);
                         else
                             umma_ss(dcol, qd0 + (uint64_t)(((bx - NBT) * QBOX + 32 * k4) >> 4),
-                                    kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4), idesc_s, 1u);
+                                    kd0 + (uint64_t)((bx * KBOX + 32 * k4) >> 4), idesc_s, (first && k4 == 0) ? 0u : 1u);
                     }
+                };
+                // group B landed (and, on the last tile, its rows past the
+                // length cleared: the clearing writes those boxes)
+                auto group_b = [&]() -> bool {
+                    if (!mbar_wait(smem_u32(&sm.kv_full[s][1]), ph, abort_flag, 0x429)) return false;
+                    if (j == nt - 1 && tail < KT && !mbar_wait(smem_u32(&sm.tail_ready), 0, abort_flag, 0x426))
+                        return false;
+                    tc_fence_after();
+                    return true;
+                };
+                if (rank == 0) {
+#pragma unroll
+                    for (int bx = 4; bx < 9; ++bx) score_box(bx, bx == 4);
+                    ok = group_b();
+                    if (!ok) break;
+#pragma unroll
+                    for (int bx = 0; bx < 4; ++bx) score_box(bx, false);
+                } else {
+#pragma unroll
+                    for (int bx = 0; bx < 4; ++bx) score_box(bx, bx == 0);
+                    score_box(8, false);
+                    ok = group_b();
+                    if (!ok) break;
+#pragma unroll
+                    for (int bx = 4; bx < 8; ++bx) score_box(bx, false);
                 }
-                if (!ok) break;
+                // group A of this stage is free once these MMAs complete
+                umma_commit(smem_u32(&sm.kv_empty[s][0]));
                 umma_commit(smem_u32(&sm.s_full[j & 1]));
                 // O_r += P(j) V_j, V = this CTA's 256 columns of the tile, after
                 // the P.V of tile j - 1 (the other thread's) has completed
@@ -271,7 +307,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int ks = 0; ks < KT / 16; ++ks)
                     umma_ts(tmem + COL_O, dcol + ks * 8, vd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
                             (j > 0 || ks > 0) ? 1u : 0u);
-                umma_commit(smem_u32(&sm.kv_empty[s]));
+                umma_commit(smem_u32(&sm.kv_empty[s][1]));
                 umma_commit(smem_u32(&sm.pv_done[par]));
                 if (j == nt - 1) umma_commit(smem_u32(&sm.o_done));   // O final (tile nt-2's P.V already done)
             }

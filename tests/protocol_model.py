@@ -22,8 +22,9 @@ two ping-pong query tiles, K ring of 2, V ring of 3, three release
 barriers; in the paged mode the tile holding the last key landing on its own
 barrier and cleared past the length before its stage counts as full),
 ``attn::mla::mla_decode_kernel`` (two issuing threads taking
-even and odd tiles, per-group arrival barriers, the Q staging in ring
-stage 1, the tail clearing) and ``attn::dec::decode_split_kernel``
+even and odd tiles, each ring stage filled in a score-only group and a value
+group with their own producers and releases, the Q staging in ring stage 1,
+the tail clearing) and ``attn::dec::decode_split_kernel``
 (persistent over units, one ring for K then V tiles, two P slots, the
 8-bit path's converter warps between an 8-bit ring and the ring). ``bug``
 plants one protocol mistake, so that tests can show a model catches it.
@@ -278,8 +279,11 @@ def prefill(nt: tuple[int, int], seed: int, rescale_p: float, bug: str | None = 
 # ---------------------------------------------------------------------------
 # attn::mla::mla_decode_kernel
 # ---------------------------------------------------------------------------
-NG = 3
-MLA_BUGS = ("kv_empty_parity", "no_qt_ready", "no_tail_ready", "no_group_wait", "pv_unordered")
+# A ring stage is filled in two groups: A (the boxes only the score MMAs read),
+# freed when the tile's score MMAs complete, and B (this CTA's value boxes),
+# freed when its P.V completes; each group has its own producer thread.
+MLA_BUGS = ("kv_empty_parity", "no_qt_ready", "no_qt_ready_b", "no_tail_ready", "no_group_wait", "pv_unordered",
+            "a_release_early")
 
 
 def mla(nt: int, tail_partial: bool, seed: int, rescale_p: float, bug: str | None = None):
@@ -287,42 +291,44 @@ def mla(nt: int, tail_partial: bool, seed: int, rescale_p: float, bug: str | Non
     for n in ("q_full", "qt_ready", "tail_ready", "o_done"):
         sim.bar(n, 1)
     for s in range(2):
-        sim.bar(f"kv_empty{s}", 1)
-        for g in range(NG):
+        for g in range(2):
+            sim.bar(f"kv_empty{s}_{g}", 1)
             sim.bar(f"kv_full{s}_{g}", 1)
     for i in range(2):
         for n in ("s_full", "p_full", "pv_done", "s_done"):
             sim.bar(f"{n}{i}", 1)
-    stage = {(s, g): None for s in range(2) for g in range(NG)}
-    stage[(1, 0)] = stage[(1, 1)] = "Q"      # Q columns 0-255 staged in ring stage 1
+    stage = {(s, g): None for s in range(2) for g in range(2)}
+    stage[(1, 0)] = stage[(1, 1)] = "Q"      # Q columns 0-255 staged over both groups of ring stage 1
     st = dict(q_copied=False, tail_cleared=False)
-    s_done, pv_done, sbuf, pbuf = set(), set(), {}, {}
+    scores_done, pv_done, sbuf, pbuf = set(), set(), {}, {}
 
-    def producer():
-        sim.load("q_full", lambda: None)
+    def producer(g):
+        if g == 0:
+            sim.load("q_full", lambda: None)
         for j in range(nt):
             s = j % 2
-            if j == 1 and bug != "no_qt_ready":
+            if j == 1 and not (bug == "no_qt_ready" and g == 0) and not (bug == "no_qt_ready_b" and g == 1):
                 yield from sim.wait("qt_ready", 0)
             if j >= 2:
                 par = ((j // 2) + (0 if bug == "kv_empty_parity" else 1)) & 1
-                yield from sim.wait(f"kv_empty{s}", par)
-                check((j - 2) in s_done and (j - 2) in pv_done, "ring stage refilled early", j)
-            for g in range(NG):
-                sim.load(f"kv_full{s}_{g}", lambda s=s, g=g, j=j: stage.__setitem__((s, g), j))
+                yield from sim.wait(f"kv_empty{s}_{g}", par)
+                if g == 0:
+                    check((j - 2) in scores_done, "group A refilled before its score MMAs completed", j)
+                else:
+                    check((j - 2) in pv_done, "group B refilled before its P V completed", j)
+            check(stage[(s, g)] != "Q" or st["q_copied"], "Q staging overwritten before the copy", j, g)
+            sim.load(f"kv_full{s}_{g}", lambda s=s, g=g, j=j: stage.__setitem__((s, g), j))
             yield
-        if nt > 0 and tail_partial:            # rows past the length cleared in the last tile
+        if g == 1 and nt > 0 and tail_partial:  # value rows past the length cleared in the last tile
             s = (nt - 1) % 2
-            for g in range(NG):
-                yield from sim.wait(f"kv_full{s}_{g}", ((nt - 1) // 2) & 1)
-            check(all(stage[(s, g)] == nt - 1 for g in range(NG)), "tail cleared before its tile landed")
+            yield from sim.wait(f"kv_full{s}_1", ((nt - 1) // 2) & 1)
+            check(stage[(s, 1)] == nt - 1, "tail cleared before its tile landed")
             st["tail_cleared"] = True
             sim.bars["tail_ready"].arrive()
 
     def qcopy():
         if nt > 0:
             yield from sim.wait("q_full", 0)
-            check(stage[(1, 0)] == "Q" and stage[(1, 1)] == "Q", "Q staging overwritten before the copy")
             st["q_copied"] = True
             sim.bars["qt_ready"].arrive()
 
@@ -335,30 +341,36 @@ def mla(nt: int, tail_partial: bool, seed: int, rescale_p: float, bug: str | Non
         for j in range(par, nt, 2):
             s, ph = j % 2, (j // 2) & 1
             yield from sim.wait(f"kv_full{s}_0", ph)
-            if j == nt - 1 and tail_partial and bug != "no_tail_ready":
-                yield from sim.wait("tail_ready", 0)
-            for g in range(NG):
-                if g > 0 and bug != "no_group_wait":
-                    yield from sim.wait(f"kv_full{s}_{g}", ph)
+            if bug == "a_release_early":
+                sim.commit(th, f"kv_empty{s}_0")
+            for g in range(2):
+                if g == 1:
+                    if bug != "no_group_wait":
+                        yield from sim.wait(f"kv_full{s}_1", ph)
+                    if j == nt - 1 and tail_partial and bug != "no_tail_ready":
+                        yield from sim.wait("tail_ready", 0)
                 def ex(j=j, s=s, g=g):
                     check(stage[(s, g)] == j, "score MMA reads the wrong tile", j, g)
-                    check(not (j == nt - 1 and tail_partial) or st["tail_cleared"], "tail read before cleared", j)
+                    check(g == 0 or not (j == nt - 1 and tail_partial) or st["tail_cleared"],
+                          "tail read before cleared", j)
                     check(g > 0 or pbuf.get(j & 1) is None or pbuf[j & 1] in pv_done, "S overwrote an unread P", j)
-                    if g == NG - 1:
+                    if g == 1:
                         sbuf[j & 1] = j
-                        s_done.add(j)
+                        scores_done.add(j)
                 sim.mma(th, ex)
+            if bug != "a_release_early":
+                sim.commit(th, f"kv_empty{s}_0")
             sim.commit(th, f"s_full{j & 1}")
             yield from sim.wait(f"p_full{j & 1}", (j >> 1) & 1)
             if j > 0 and bug != "pv_unordered":
                 yield from sim.wait(f"pv_done{par ^ 1}", ((j - 1) >> 1) & 1)
             def pv(j=j, s=s):
                 check(pbuf.get(j & 1) == j, "P V reads the wrong P", j)
-                check(all(stage[(s, g)] == j for g in range(NG)), "P V reads the wrong tile", j)
+                check(stage[(s, 1)] == j, "P V reads the wrong tile", j)
                 check(j == 0 or (j - 1) in pv_done, "O accumulated out of order", j)
                 pv_done.add(j)
             sim.mma(th, pv)
-            sim.commit(th, f"kv_empty{s}")
+            sim.commit(th, f"kv_empty{s}_1")
             sim.commit(th, f"pv_done{par}")
             if j == nt - 1:
                 sim.commit(th, "o_done")
@@ -380,7 +392,7 @@ def mla(nt: int, tail_partial: bool, seed: int, rescale_p: float, bug: str | Non
             yield from sim.wait("o_done", 0)
             check(pv_done == set(range(nt)), "epilogue before the last P V")
 
-    sim.run([producer(), qcopy(), issuer(0), issuer(1), softmax()])
+    sim.run([producer(0), producer(1), qcopy(), issuer(0), issuer(1), softmax()])
     check(pv_done == set(range(nt)), "P V missing")
 
 
