@@ -7,12 +7,12 @@ One step = one pass of the hot path over synthetic inputs resident in HBM:
     ~U[1024, 32768], 32/8 heads, head dim 128), split-KV + combine;
   * MLA decode: attn_decode on the latent cache (B=64, 4096 rows of 576,
     128 heads, value = first 512 columns).
-The other configurations are timed in a loop of their own after the step:
-the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads), the tiny causal
-forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency), two small-batch
-GQA decodes (B=1 at 32768 keys, B=4 at 8192) and two small-batch MLA decodes
-(B=1 and B=4 at 4096 keys); so are the rows built beyond the path (paged
-prefill and decode, FP8 and RoPE forms), in a third loop.
+The other configurations are timed after the step, each in a loop of its
+own: the 70B-shaped long prefill (B=1, S=32768, 64 / 8 heads), the tiny
+causal forward (B=1, S=64, 4 / 2 heads, head dim 32, a latency), two
+small-batch GQA decodes (B=1 at 32768 keys, B=4 at 8192) and two small-batch
+MLA decodes (B=1 and B=4 at 4096 keys); so are the rows built beyond the
+path (paged prefill and decode, FP8 and RoPE forms).
 `value` is prefill TFLOP/s (algorithmic FLOPs: causal pairs only); the
 decode regimes are reported in HBM GB/s (algorithmic bytes: the K/V rows
 below each sequence's length, plus q, o and lse) under "regimes". Each kernel
@@ -504,13 +504,16 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    # Each group is warmed up and timed in a loop of its own, so that the
-    # configurations and rows beyond the step do not disturb the headline.
-    # Every timed launch follows an L2 flush and has its own events.
+    # The step (the hot path's regimes, one after another) is warmed up and
+    # timed in a loop of its own; every other regime gets a loop of its own
+    # too, so that neither disturbs the headline nor the others (power and
+    # clock state carry over from one kernel to the next). Every timed launch
+    # follows an L2 flush and has its own events.
     t_wall = 0.0
+    loops = [[r for r in regimes.values() if r.group == "core"]]
+    loops += [[r] for g in ("configs", "next") for r in regimes.values() if r.group == g]
     with ClockSampler(torch.cuda.current_device()) as clocks:
-        for group in ("core", "configs", "next"):
-            rs = [r for r in regimes.values() if r.group == group]
+        for rs in loops:
             if not rs:
                 continue
 
