@@ -748,7 +748,8 @@ def run_ours(args):
         out["paged_prefill"] = {"workload": f"{w.name}, keys and values in 64-token pages in a shuffled pool",
                                 "ms": ms_pp, "tflops": tf(fl_p, ms_pp), "frac_of_peak": tf(fl_p, ms_pp) / peak_tf,
                                 "kernel": "attn::pf::prefill_kernel<128, paged>",
-                                "roofline": tensor_roofline(fl_p, ms_pp, "attn::pf::prefill_kernel<128, paged>", None)}
+                                "roofline": tensor_roofline(fl_p, ms_pp, "attn::pf::prefill_kernel<128, paged>",
+                                                            "prefill_kernel_128_paged")}
     if "fp8_decode" in regimes:
         ms_f = mean["fp8_decode"]
         out["fp8_decode"] = {"workload": f"{wd.name}, e4m3 cache with one scale per KV head", "ms": ms_f,
