@@ -269,6 +269,32 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(smem_u32(&sm.mma_done), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
+        if constexpr (!FP8 && !PAGED) {
+            // The first unit's Q rows and first ring tiles go out now, before
+            // the setup barrier and the TMEM allocation (the producer warp
+            // skips them): every stage is free at the start.
+            UnitCursor c0;
+            Unit u0;
+            if (B > 0) start_sequence(c0, seqlens, S_max, ch, win);
+            if (B > 0 && next_unit(c0, blockIdx.x, seqlens, B, S_max, ch, n_hb, n_kv * n_hb, win, u0)) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+                const int h0 = u0.kvh * G + u0.hb * GT;
+                mbar_arrive_expect_tx(smem_u32(&sm.q_full), 2 * C::QBOX);
+                tma_load_3d(smem_u32(sm.q[0]), &tm_q, smem_u32(&sm.q_full), 0, h0, u0.b);
+                tma_load_3d(smem_u32(sm.q[1]), &tm_q, smem_u32(&sm.q_full), 64, h0, u0.b);
+                const int pre = min(NSTAGE, 2 * u0.ntiles);
+                for (int j = 0; j < pre; ++j) {
+                    const CUtensorMap *tm = (j < u0.ntiles) ? &tm_k : &tm_v;
+                    const int krow = u0.key0 + (j < u0.ntiles ? j : j - u0.ntiles) * KT;
+                    const uint32_t full = smem_u32(&sm.full[j]);
+                    mbar_arrive_expect_tx(full, TILE_BYTES);
+                    tma_load_4d(smem_u32(sm.ring[j]), tm, full, 0, krow, u0.kvh, u0.b);
+                    tma_load_4d(smem_u32(sm.ring[j]) + BOX_BYTES, tm, full, 64, krow, u0.kvh, u0.b);
+                }
+            }
+        }
         // values above S_max are clamped; report it once per launch
         if (blockIdx.x == 0)
             for (int b = 0; b < B; ++b)
@@ -304,10 +330,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // the single Q buffer is free once the previous unit's S^T MMAs completed
                 if (n > 0 && !mbar_wait(smem_u32(&sm.q_empty), (n - 1) & 1, abort_flag, 0x101)) break;
                 const int h0 = u.kvh * G + u.hb * GT;
-                mbar_arrive_expect_tx(smem_u32(&sm.q_full), 2 * C::QBOX);
-                tma_load_3d(smem_u32(sm.q[0]), &tm_q, smem_u32(&sm.q_full), 0, h0, u.b);
-                tma_load_3d(smem_u32(sm.q[1]), &tm_q, smem_u32(&sm.q_full), 64, h0, u.b);
-                for (int j = 0; j < 2 * u.ntiles; ++j, ++t) {
+                // the first unit's Q and first ring tiles were issued during setup
+                const int pre = (!FP8 && !PAGED && n == 0) ? min(NSTAGE, 2 * u.ntiles) : 0;
+                if (pre == 0) {
+                    mbar_arrive_expect_tx(smem_u32(&sm.q_full), 2 * C::QBOX);
+                    tma_load_3d(smem_u32(sm.q[0]), &tm_q, smem_u32(&sm.q_full), 0, h0, u.b);
+                    tma_load_3d(smem_u32(sm.q[1]), &tm_q, smem_u32(&sm.q_full), 64, h0, u.b);
+                }
+                t += pre;
+                for (int j = pre; j < 2 * u.ntiles; ++j, ++t) {
                     const CUtensorMap *tm = (j < u.ntiles) ? &tm_k : &tm_v;
                     const int krow = u.key0 + (j < u.ntiles ? j : j - u.ntiles) * KT;
                     if constexpr (FP8) {
@@ -659,10 +690,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 // LSE = (M + log2 sum w_s l_s) * ln 2.
 // Launched as a programmatic dependent of the split kernel, so that its launch
 // overlaps that kernel's tail; it waits for the partials before reading them.
-// One CTA per (h, b), 128 threads = 4 groups of 32; a group takes the
-// chunks s = g (mod 4), a lane 4 consecutive output dims per 128 (16-byte
-// loads), and the four groups' sums meet in shared memory.
-constexpr int COMBINE_THREADS = 128;
+// One CTA per (h, b), 256 threads = 8 groups of 32; a group takes the chunks
+// s = g (mod 8) and folds them with a running maximum of its own (each
+// chunk's (m_s, l_s) and partial output are loaded together, so a group's
+// loads all go out at once), a lane 4 consecutive output dims per 128
+// (16-byte loads); the eight groups' sums meet in shared memory, rescaled to
+// the overall maximum.
+constexpr int COMBINE_THREADS = 256;
+constexpr int COMBINE_GROUPS = COMBINE_THREADS / 32;
 
 template <int DV>
 __global__ void __launch_bounds__(COMBINE_THREADS)
@@ -671,8 +706,9 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
                       float *__restrict__ lse, int n_q, int n_splits, int S_max, int chunk, Window win) {
     static_assert(DV % 128 == 0, "value width");
     constexpr int NQ = DV / 128;   // float4 loads per lane and chunk
-    __shared__ float red[4][DV];
-    __shared__ float part[4];
+    constexpr int NG = COMBINE_GROUPS;
+    __shared__ float red[NG][DV];
+    __shared__ float part_m[NG], part_l[NG];
     const int h = blockIdx.x, b = blockIdx.y;
     const int tid = threadIdx.x, g = tid >> 5, lane = tid & 31;
     int seqlen = seqlens[b];
@@ -689,44 +725,58 @@ decode_combine_kernel(const float *__restrict__ ws_o, const float2 *__restrict__
         if (tid == 0 && lse) lse[row] = -INFINITY;
         return;
     }
-    // M = max over chunks
-    float M = -INFINITY;
-    for (int c = tid; c < ns; c += COMBINE_THREADS) M = fmaxf(M, ml[plan.split(c)].x);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) part[g] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3]));
-    // this group's weighted sum of o_s over its chunks, and of l_s
+    // this group's chunks folded against its own running maximum Mg:
+    // acc = sum 2^(m_s - Mg) o_s, L = sum 2^(m_s - Mg) l_s
     float4 acc[NQ];
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) acc[qi] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float L = 0.f;
+    float Mg = -INFINITY, L = 0.f;
     const float *base = ws_o + row * n_splits * (size_t)DV + lane * 4;
-#pragma unroll 4
-    for (int c = g; c < ns; c += 4) {
+#pragma unroll 8
+    for (int c = g; c < ns; c += NG) {
         const int s = plan.split(c);
         const float2 m_l = ml[s];
-        const float w = ex2(m_l.x - M);
+        float4 v[NQ];
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) v[qi] = __ldg(reinterpret_cast<const float4 *>(base + (size_t)s * DV + qi * 128));
+        const float m_new = fmaxf(Mg, m_l.x);
+        const float a = Mg == -INFINITY ? 0.f : ex2(Mg - m_new);   // rescale of what came before
+        const float w = ex2(m_l.x - m_new);
 #pragma unroll
         for (int qi = 0; qi < NQ; ++qi) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(base + (size_t)s * DV + qi * 128));
-            acc[qi].x = fmaf(w, v.x, acc[qi].x);
-            acc[qi].y = fmaf(w, v.y, acc[qi].y);
-            acc[qi].z = fmaf(w, v.z, acc[qi].z);
-            acc[qi].w = fmaf(w, v.w, acc[qi].w);
+            acc[qi].x = fmaf(w, v[qi].x, acc[qi].x * a);
+            acc[qi].y = fmaf(w, v[qi].y, acc[qi].y * a);
+            acc[qi].z = fmaf(w, v[qi].z, acc[qi].z * a);
+            acc[qi].w = fmaf(w, v[qi].w, acc[qi].w * a);
         }
-        L = fmaf(w, m_l.y, L);
+        L = fmaf(w, m_l.y, L * a);
+        Mg = m_new;
     }
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) *reinterpret_cast<float4 *>(&red[g][qi * 128 + lane * 4]) = acc[qi];
-    __syncthreads();   // part[] reads above are done before it is reused
-    if (lane == 0) part[g] = L;
+    if (lane == 0) {
+        part_m[g] = Mg;
+        part_l[g] = L;
+    }
     __syncthreads();
-    const float Lt = part[0] + part[1] + part[2] + part[3];
+    // the groups' sums rescaled to M = max over all chunks (a group without
+    // chunks has Mg = -inf and weight 0)
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) M = fmaxf(M, part_m[k]);
+    float sc[NG], Lt = 0.f;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+        sc[k] = part_m[k] == -INFINITY ? 0.f : ex2(part_m[k] - M);
+        Lt = fmaf(sc[k], part_l[k], Lt);
+    }
     const float inv = 1.f / Lt;
-    for (int d = tid; d < DV; d += COMBINE_THREADS)
-        o[row * DV + d] = __float2bfloat16_rn((red[0][d] + red[1][d] + red[2][d] + red[3][d]) * inv);
+    for (int d = tid; d < DV; d += COMBINE_THREADS) {
+        float x = 0.f;
+#pragma unroll
+        for (int k = 0; k < NG; ++k) x = fmaf(sc[k], red[k][d], x);
+        o[row * DV + d] = __float2bfloat16_rn(x * inv);
+    }
     if (tid == 0 && lse) lse[row] = (M + log2f(Lt)) * 0.6931471805599453f;
 }
 
