@@ -19,6 +19,7 @@ Functions:
   sdpa_varlen(q, k, v, cu_q, cu_k, causal, scale) -> (o, lse)  packed batch, one sdpa per sequence
   sdpa_window(q, k, v, causal, window, n_sink, scale, seqlens=None) -> (o, lse) sliding window + sinks
   dequant_e4m3(bytes, scale)                     -> fp64      FP8 (e4m3) cache values
+  dequant_e4m3_tiles(bytes, scales, tile)        -> fp64      the same with one scale per token tile
   rope_tables(n_pos, d, base)                    -> (cos, sin) rotary tables [n_pos, d/2]
   rope(x, cos, sin, positions)                   -> fp64      rotary position embedding
   sdpa_rope(q, k, v, causal, scale, cos, sin)    -> (o, lse)  sdpa on rotated (bf16) queries and keys
@@ -313,6 +314,19 @@ def dequant_e4m3(raw, scale=None, head_axis=1):
         shape[head_axis] = -1
         val = val * sc.reshape(shape)
     return val
+
+
+def dequant_e4m3_tiles(raw, scales, tile: int = 128):
+    """Values of an e4m3 cache [B, n_kv, S, d] with one scale per tile of
+    `tile` consecutive tokens of each (sequence, KV head) ("Flash Attention 3
+    and Multi-Headed Latent Attention", FP8 section: per-tile scaling
+    factors): token j of (b, g) is e4m3(byte) * scales[b, g, j // tile].
+    `scales` [B, n_kv, ceil(S / tile)]. Returns float64."""
+    val = dequant_e4m3(raw)
+    sc = np.asarray(scales.cpu().numpy() if hasattr(scales, "cpu") else scales, dtype=np.float64)
+    S = val.shape[2]
+    tok_tile = np.arange(S) // tile                      # tile of each token
+    return val * sc[:, :, tok_tile][..., None]
 
 
 def rope_tables(n_pos: int, d: int, base: float, lib=None):

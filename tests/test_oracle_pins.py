@@ -124,6 +124,22 @@ def test_dequant_e4m3_matches_an_independent_decoder():
     assert np.array_equal(oracle.dequant_e4m3(x, [1.0, 0.5, 2.0])[0, :, 0], [1.0, 0.5, 2.0])
 
 
+def test_dequant_e4m3_tiles():
+    """Per-tile scales: a hand case (1.0 bytes over two tiles of two tokens
+    scaled by 2 and 3; a NaN byte stays NaN), and constant scales per
+    (sequence, KV head) reduce to the per-head form."""
+    x = np.full((1, 1, 4, 2), 0x38, np.uint8)
+    x[0, 0, 3, 1] = 0x7F
+    got = oracle.dequant_e4m3_tiles(x, [[[2.0, 3.0]]], tile=2)
+    assert np.array_equal(got[0, 0, :3], [[2.0, 2.0], [2.0, 2.0], [3.0, 3.0]])
+    assert got[0, 0, 3, 0] == 3.0 and np.isnan(got[0, 0, 3, 1])
+    rng = np.random.default_rng(4)
+    raw = rng.integers(0, 126, size=(2, 3, 300, 8)).astype(np.uint8)   # no NaN patterns
+    per_head = np.array([0.5, 2.0, 0.125])
+    tiles = np.broadcast_to(per_head[None, :, None], (2, 3, 3))
+    assert np.array_equal(oracle.dequant_e4m3_tiles(raw, tiles), oracle.dequant_e4m3(raw, per_head))
+
+
 def test_round_bf16_matches_torch():
     """The oracle's bf16 rounding against torch's fp32 -> bf16 conversion
     (round to nearest even) on fp32 values, ties and near-ties included."""
