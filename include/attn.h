@@ -227,6 +227,29 @@ int attn_decode_fp8(const void *q, const void *kcache, const void *vcache, const
                     float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_decode_fp8_tiles -- attn_decode_fp8 with one key scale and one value
+ * scale per 128-key tile of each (sequence, KV head) instead of per KV head.
+ * Source: "Flash Attention 3 and Multi-Headed Latent Attention"
+ * (misar.blog), FP8 section (e4m3 operands with per-tile scaling factors).
+ *
+ *   k_scales, v_scales: [B, n_kv, ceil(S_max / 128)] fp32 on the device,
+ *            contiguous; key j of (b, g) is e4m3(bytes) * k_scales[b, g, j / 128],
+ *            value likewise with v_scales (finite, > 0)
+ *   every other argument, the workspace (attn_decode_fp8_workspace_bytes)
+ *   and the error behaviour as attn_decode_fp8.
+ * The key scale of a tile multiplies its scores, the value scale the
+ * softmax weights of its keys before they meet the values (so the weights
+ * stay below the value scale in f16); the row sums take the unscaled
+ * weights.
+ */
+int attn_decode_fp8_tiles(const void *q, const void *kcache, const void *vcache, const float *k_scales,
+                          const float *v_scales, const int32_t *seqlens, void *o, float *lse,
+                          int B, int n_q, int n_kv, int S_max,
+                          int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                          int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s,
+                          float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_paged -- attn_decode against a paged KV cache.
  * Source: "Attention deep dive" (askaiml.pages.dev), section 5 (production
  * engines keep the KV cache in fixed-size pages addressed through a page

@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.attn_decode_fp8.argtypes = ([_vp] * 8 + [_i] * 4 + [_i64] * 6 +
                                       [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_decode_fp8.restype = _i
+        L.attn_decode_fp8_tiles.argtypes = ([_vp] * 8 + [_i] * 4 + [_i64] * 6 +
+                                            [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
+        L.attn_decode_fp8_tiles.restype = _i
         L.attn_decode_paged.argtypes = ([_vp] * 7 + [_i] * 8 + [_i64] * 6 +
                                         [ctypes.c_float, _vp, ctypes.c_size_t, _vp])
         L.attn_fwd_paged.argtypes = [_vp] * 8 + [_i] * 10 + [_i64] * 6 + [_i, ctypes.c_float, _vp]
@@ -282,6 +285,37 @@ def attn_decode_fp8(q, kcache, vcache, k_scale, v_scale, seqlens, scale: float, 
                                _ptr(o), _ptr(lse), B, n_q, n_kv, S_max, *ks, *vs, float(scale), _ptr(workspace),
                                workspace.numel(), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_decode_fp8")
+    return o, lse
+
+
+def attn_decode_fp8_tiles(q, kcache, vcache, k_scales, v_scales, seqlens, scale: float, o=None, lse=None,
+                          workspace=None, stream=None, want_lse=True):
+    """attn_decode_fp8 with one scale per 128-key tile: k_scales/v_scales
+    contiguous fp32 [B, n_kv, ceil(S_max / 128)] on the device."""
+    B, n_q, d = q.shape
+    _, n_kv, S_max, _ = kcache.shape
+    if not (q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous()):
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    for t in (kcache, vcache):
+        if t.element_size() != 1 or not t.is_cuda:
+            raise ValueError("the FP8 cache must be a one-byte-per-element CUDA tensor")
+    n_tiles = (S_max + 127) // 128
+    for t in (k_scales, v_scales):
+        if (t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous()
+                or tuple(t.shape) != (B, n_kv, n_tiles)):
+            raise ValueError("k_scales / v_scales must be contiguous fp32 CUDA tensors [B, n_kv, ceil(S_max/128)]")
+    ks, vs = _elem_strides(kcache), _elem_strides(vcache)
+    if o is None:
+        o = torch.empty((B, n_q, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(decode_fp8_workspace_bytes(B, n_q, n_kv, S_max), 1), dtype=torch.uint8,
+                                device=q.device)
+    rc = lib().attn_decode_fp8_tiles(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(k_scales), _ptr(v_scales),
+                                     _ptr(seqlens), _ptr(o), _ptr(lse), B, n_q, n_kv, S_max, *ks, *vs, float(scale),
+                                     _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_decode_fp8_tiles")
     return o, lse
 
 

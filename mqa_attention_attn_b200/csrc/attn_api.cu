@@ -908,6 +908,40 @@ int attn_decode_fp8(const void *q, const void *kcache, const void *vcache, const
                                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+int attn_decode_fp8_tiles(const void *q, const void *kcache, const void *vcache, const float *k_scales,
+                          const float *v_scales, const int32_t *seqlens, void *o, float *lse, int B, int n_q, int n_kv,
+                          int S_max, int64_t k_stride_b, int64_t k_stride_h, int64_t k_stride_s,
+                          int64_t v_stride_b, int64_t v_stride_h, int64_t v_stride_s, float scale, void *workspace,
+                          size_t workspace_bytes, attn_stream_t stream) {
+    if (B < 0 || n_q < 1 || n_kv < 1 || S_max < 1 || n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0) return ATTN_OK;
+    if (!q || !kcache || !vcache || !k_scales || !v_scales || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (k_stride_b < 0 || k_stride_h < 0 || k_stride_s < 0 || v_stride_b < 0 || v_stride_h < 0 || v_stride_s < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (k_stride_s < 128 || v_stride_s < 128) return ATTN_ERR_INVALID_ARG;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+    if ((k_stride_b | k_stride_h | k_stride_s | v_stride_b | v_stride_h | v_stride_s) & 15)
+        return ATTN_ERR_MISALIGNED;   // one-byte elements: strides in multiples of 16 bytes
+    size_t need = 0;
+    attn_decode_fp8_workspace_bytes(B, n_q, n_kv, S_max, &need);
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+    CacheView cv{};
+    cv.k = kcache;
+    cv.v = vcache;
+    cv.ks[0] = k_stride_b, cv.ks[1] = k_stride_h, cv.ks[2] = k_stride_s;
+    cv.vs[0] = v_stride_b, cv.vs[1] = v_stride_h, cv.vs[2] = v_stride_s;
+    cv.fs.k_scale = k_scales;
+    cv.fs.v_scale = v_scales;
+    cv.fs.tile_stride = (S_max + attn::dec::KT - 1) / attn::dec::KT;
+    return dispatch_decode_gqa<false, true>(G, q, cv, seqlens, o, lse, B, n_q, n_kv, S_max, scale, workspace,
+                                            reinterpret_cast<cudaStream_t>(stream));
+}
+
 int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
                       const int32_t *seqlens, void *o, float *lse, int B, int n_q, int n_kv, int d_qk, int d_v,
                       int page_size, int pages_per_seq, int num_pages, int64_t k_stride_page,

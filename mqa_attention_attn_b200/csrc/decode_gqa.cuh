@@ -119,7 +119,10 @@ static_assert(smem_fits<false>() && smem_fits<true>(), "decode shared memory exc
 // FP8 cache scales: element (b, g, j, c) of the cache means
 // e4m3(byte) * k_scale[g] (keys) or * v_scale[g] (values).
 struct Fp8Scales {
-    const float *k_scale, *v_scale;   // [n_kv]; null on the bf16 path
+    const float *k_scale, *v_scale;   // null on the bf16 path
+    // 0: one scale per KV head ([n_kv]); t > 0: one scale per 128-key tile of
+    // each (sequence, KV head), [B][n_kv][t], key j in tile j / 128
+    int tile_stride;
 };
 
 // Sliding window over the cache (window 0: none): of keys 0 .. L-1 a
@@ -579,7 +582,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
              i += gridDim.x, ++n) {
             const int h0 = u.kvh * G + u.hb * GT;
             // FP8: the key scale of this KV head scales every score
-            const float su = FP8 ? scale_log2 * fs.k_scale[u.kvh] : scale_log2;
+            const bool tiles = FP8 && fs.tile_stride > 0;   // FP8: a scale per 128-key tile
+            const float su = (FP8 && !tiles) ? scale_log2 * fs.k_scale[u.kvh] : scale_log2;
+            // FP8 per-tile scales of this unit's tiles: (b, kv head) row, first tile
+            const size_t trow = tiles ? ((size_t)u.b * n_kv + u.kvh) * fs.tile_stride + u.key0 / KT : 0;
             bool ok = mbar_wait(smem_u32(&sm.s_full), n & 1, abort_flag, 0x301);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
@@ -597,8 +603,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int jj = 0; jj < 4; ++jj) {
                     const int key = (jg + jj) * KT + tid;
                     if (jg + jj < u.ntiles && key < u.nkeys && window_keeps(u.key0 + key, u.seqlen, win)) {
+                        // per-tile key scales: the maximum of the scaled scores
+                        const float kt = tiles ? __ldg(fs.k_scale + trow + jg + jj) : 1.f;
 #pragma unroll
-                        for (int h = 0; h < GT; ++h) m[h] = fmaxf(m[h], __uint_as_float(sv[jj][h]));
+                        for (int h = 0; h < GT; ++h) m[h] = fmaxf(m[h], tiles ? __uint_as_float(sv[jj][h]) * kt
+                                                                              : __uint_as_float(sv[jj][h]));
                     }
                 }
             }
@@ -627,15 +636,19 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tmem_wait_ld();
                 const int key = j * KT + tid;
                 const bool valid = key < u.nkeys && window_keeps(u.key0 + key, u.seqlen, win);
+                // per-tile scales: the key scale joins the exponent's, the value
+                // scale multiplies P (the row sums take P unscaled)
+                const float sj = tiles ? su * __ldg(fs.k_scale + trow + j) : su;
+                const float vj = tiles ? __ldg(fs.v_scale + trow + j) : 1.f;
                 uint32_t pk[NH / 2];
 #pragma unroll
                 for (int h2 = 0; h2 < NH / 2; ++h2) {
                     float p0 = 0.f, p1 = 0.f;
-                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[2 * h2]), su, -mc[2 * h2]));
-                    if (2 * h2 + 1 < GT && valid) p1 = ex2(fmaf(__uint_as_float(sv[2 * h2 + 1]), su, -mc[2 * h2 + 1]));
+                    if (2 * h2 < GT && valid) p0 = ex2(fmaf(__uint_as_float(sv[2 * h2]), sj, -mc[2 * h2]));
+                    if (2 * h2 + 1 < GT && valid) p1 = ex2(fmaf(__uint_as_float(sv[2 * h2 + 1]), sj, -mc[2 * h2 + 1]));
                     if (2 * h2 < GT) l[2 * h2] += p0;
                     if (2 * h2 + 1 < GT) l[2 * h2 + 1] += p1;
-                    pk[h2] = FP8 ? f2_to_h2_sat(p0, p1) : f2_to_bf2(p0, p1);
+                    pk[h2] = FP8 ? (tiles ? f2_to_h2_sat(p0 * vj, p1 * vj) : f2_to_h2_sat(p0, p1)) : f2_to_bf2(p0, p1);
                 }
                 // the slot is free once the P.V of the tile two before has completed
                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.p_empty[pc & 1]), ((pc >> 1) & 1) ^ 1,
@@ -663,7 +676,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             if (named_bar_or(1, NSW * 32, !ok)) break;
             const size_t row0 = (size_t)u.b * n_q + h0;
-            const float vsc = FP8 ? fs.v_scale[u.kvh] : 1.f;   // FP8: the value scale of this KV head
+            const float vsc = (FP8 && !tiles) ? fs.v_scale[u.kvh] : 1.f;   // FP8: the value scale of this KV head
 #pragma unroll
             for (int h = 0; h < GT; ++h)
                 ws_o[((row0 + h) * n_splits + u.split) * D + tid] = __uint_as_float(ov[h]) * vsc;
