@@ -452,6 +452,20 @@ def run_ours(args):
         by_f = decode_bytes(wd, seqlens, cache_elem_bytes=1)
         add("fp8_decode", "next", 2, lambda: binding.attn_decode_fp8(
             qd, k8, v8, ks8, vs8, sl_dev, wd.scale, o=of8, lse=lf8, workspace=work8, stream=stream))
+        # the same cache quantised with one scale per 128-key tile of each
+        # (sequence, KV head)
+        def to_e4m3_tiles(x):
+            Bx, nk, S, d = x.shape
+            nt = (S + 127) // 128
+            xp = torch.nn.functional.pad(x.float(), (0, 0, 0, nt * 128 - S)).view(Bx, nk, nt, 128, d)
+            sc = (xp.abs().amax(dim=(3, 4)).clamp_min(1e-6) / 448.0).float().contiguous()
+            q8 = (xp / sc[..., None, None]).view(Bx, nk, nt * 128, d)[:, :, :S].to(torch.float8_e4m3fn)
+            return q8.contiguous(), sc
+        k8t, kst = to_e4m3_tiles(kc)
+        v8t, vst = to_e4m3_tiles(vc)
+        of8t, lf8t = torch.empty_like(od), torch.empty_like(ld)
+        add("fp8_decode_tiles", "next", 2, lambda: binding.attn_decode_fp8_tiles(
+            qd, k8t, v8t, kst, vst, sl_dev, wd.scale, o=of8t, lse=lf8t, workspace=work8, stream=stream))
 
     # the Llama-3-8B prefill with its keys and values in 64-token pages placed
     # in a pool in a seeded random order (chunked-prefill serving layout)
@@ -761,6 +775,17 @@ def run_ours(args):
                                                       "decode_split_kernel_4_fp8",
                                                       "achieved over split + merge launches; traffic of the "
                                                       "split kernel")}
+    if "fp8_decode_tiles" in regimes:
+        ms_ft = mean["fp8_decode_tiles"]
+        # plus the key and value scales of the tiles below each length
+        by_ft = by_f + sum(wd.n_kv * ((int(L) + 127) // 128) * 2 * 4 for L in seqlens.tolist())
+        out["fp8_decode_tiles"] = {"workload": f"{wd.name}, e4m3 cache with one scale per 128-key tile",
+                                   "ms": ms_ft, "gbs": gbs(by_ft, ms_ft), "frac_of_peak": gbs(by_ft, ms_ft) / peak_bw,
+                                   "algorithmic_bytes": by_ft,
+                                   "kernels": "attn::dec::decode_split_kernel<4, fp8> (tile scales) + "
+                                              "decode_combine_kernel",
+                                   "roofline": hbm_roofline(by_ft, ms_ft, "attn::dec::decode_split_kernel<4, fp8>",
+                                                            None, "achieved over split + merge launches")}
     if "rope_prefill" in regimes:
         ms_rp, ms_rd = mean["rope_prefill"], mean["rope_decode"]
         out["rope_prefill"] = {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": ms_rp,
