@@ -423,27 +423,37 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         __syncwarp();
         tc_fence_after();
         const int head = hb * M + r;
+        // Each thread owns one head row of 256 output columns. Writing it
+        // straight from registers sends each warp store to 32 rows; instead the
+        // row goes to the idle ring (all of its reads completed before o_done)
+        // at a 16-byte-padded stride, so that a quarter warp's 16-byte stores
+        // fall on distinct banks, and one bulk copy per row moves it out.
+        const uint32_t stage = smem_u32(&sm.k[0][0][0]);
         if (p.n_splits > 1) {
             // partial output of this chunk for the merge kernel: unnormalised O
             // (this CTA's 256 columns) and, from rank 0, (m, l); a chunk with
             // no key writes nothing (the merge reads only the chunks below the
             // sequence's length)
             if (nt > 0) {
-                const size_t prow = ((size_t)b * p.n_q + head) * p.n_splits + split;
+                constexpr uint32_t ROW = 256 * 4 + 16;
+                const uint32_t srow = stage + r * ROW;
 #pragma unroll 1
                 for (int c = 0; c < 256 / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(trow + COL_O + 32 * c, o);
                     tmem_wait_ld();
-                    if (head < p.n_q) {
-                        float4 *dst = reinterpret_cast<float4 *>(p.ws_o + prow * DV + 256 * rank + 32 * c);
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4)
-                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
-                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
-                    }
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        sts128(srow + 128 * c + 16 * q4, make_uint4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]));
                 }
-                if (rank == 0 && head < p.n_q) p.ws_ml[prow] = make_float2(m_run, l_run);
+                if (head < p.n_q) {
+                    const size_t prow = ((size_t)b * p.n_q + head) * p.n_splits + split;
+                    fence_proxy_async_smem();
+                    bulk_store(p.ws_o + prow * DV + 256 * rank, srow, 256 * 4);
+                    tma_store_commit();
+                    if (rank == 0) p.ws_ml[prow] = make_float2(m_run, l_run);
+                    tma_store_wait_read0();
+                }
             }
         } else {
             if (head < p.n_q && nt == 0) {
@@ -451,25 +461,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int c = 0; c < 256 / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
             }
             if (nt > 0) {
+                constexpr uint32_t ROW = 256 * 2 + 16;
+                const uint32_t srow = stage + r * ROW;
                 const float inv_l = 1.f / l_run;
 #pragma unroll 1
                 for (int c = 0; c < 256 / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(trow + COL_O + 32 * c, o);
                     tmem_wait_ld();
-                    if (head < p.n_q) {
-                        uint4 *dst =
-                            reinterpret_cast<uint4 *>(p.o + ((size_t)b * p.n_q + head) * DV + 256 * rank + 32 * c);
 #pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            uint4 w;
-                            w.x = f2_to_bf2(__uint_as_float(o[8 * q8 + 0]) * inv_l, __uint_as_float(o[8 * q8 + 1]) * inv_l);
-                            w.y = f2_to_bf2(__uint_as_float(o[8 * q8 + 2]) * inv_l, __uint_as_float(o[8 * q8 + 3]) * inv_l);
-                            w.z = f2_to_bf2(__uint_as_float(o[8 * q8 + 4]) * inv_l, __uint_as_float(o[8 * q8 + 5]) * inv_l);
-                            w.w = f2_to_bf2(__uint_as_float(o[8 * q8 + 6]) * inv_l, __uint_as_float(o[8 * q8 + 7]) * inv_l);
-                            dst[q8] = w;
-                        }
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = f2_to_bf2(__uint_as_float(o[8 * q8 + 2 * e]) * inv_l,
+                                             __uint_as_float(o[8 * q8 + 2 * e + 1]) * inv_l);
+                        sts128(srow + 64 * c + 16 * q8, make_uint4(w[0], w[1], w[2], w[3]));
                     }
+                }
+                if (head < p.n_q) {
+                    // the entry point requires a 16-byte-aligned output
+                    fence_proxy_async_smem();
+                    bulk_store(p.o + ((size_t)b * p.n_q + head) * DV + 256 * rank, srow, 256 * 2);
+                    tma_store_commit();
+                    tma_store_wait_read0();
                 }
             }
             if (rank == 0 && head < p.n_q && p.lse != nullptr)
