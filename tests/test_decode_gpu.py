@@ -225,3 +225,52 @@ def test_large_batch_decode_keeps_the_largest_chunk():
     kc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
     vc = torch.randn(B, n_kv, S_max, 128, generator=g, device="cuda").to(torch.bfloat16)
     _decode_and_check(seq, q, kc, vc, 1 / math.sqrt(128), f"large-batch decode B={B}")
+
+
+def test_decode_split_ignores_workspace_contents_and_replays():
+    """The split-KV decode writes each key chunk's partial output to the
+    workspace and a second kernel merges them. Whatever the workspace holds on
+    entry (all ones, then random bytes), the result is the oracle's and
+    repeats bit for bit; a CUDA graph replays both launches with new queries,
+    each replay against the oracle. A zero-length sequence in the batch gets
+    O = 0, LSE = -inf."""
+    binding = need_gpu()
+    B, n_q, n_kv, L = 3, 32, 8, 8192
+    scale = 1 / math.sqrt(128)
+    seq = torch.tensor([8192, 0, 3000], dtype=torch.int32)
+    sl = seq.to("cuda")
+    g = torch.Generator(device="cuda").manual_seed(4242)
+    q = torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(B, n_kv, L, 128, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(B, n_kv, L, 128, generator=g, device="cuda").to(torch.bfloat16)
+    assert _planned_splits(B, n_kv, n_q // n_kv, L) > 1
+    nbytes = binding.decode_workspace_bytes(B, n_q, n_kv, 128, 128, L)
+    ws = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")
+
+    def check(o, lse, what):
+        assert torch.all(o[1] == 0) and torch.all(torch.isneginf(lse[1])), what
+        keep = [0, 2]
+        o_ref, lse_ref = oracle.sdpa(q[keep][:, :, None, :], kc[keep], vc[keep], False, scale,
+                                     seqlens=seq.numpy()[keep])
+        check_parity(o[keep], lse[keep], o_ref[:, :, 0], lse_ref[:, :, 0], what)
+
+    o1, lse1 = binding.attn_decode(q, kc, vc, sl, scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    check(o1, lse1, "workspace of all ones")
+    ws.random_(0, 256, generator=g)
+    o2, lse2 = binding.attn_decode(q, kc, vc, sl, scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(lse1, lse2)
+
+    o3, lse3 = torch.empty_like(o1), torch.empty_like(lse1)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        binding.attn_decode(q, kc, vc, sl, scale, o=o3, lse=lse3, workspace=ws)
+    for rep in range(3):
+        q.copy_(torch.randn(B, n_q, 128, generator=g, device="cuda").to(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert binding.device_status() == 0
+        check(o3, lse3, f"graph replay {rep}")
+    del graph
