@@ -20,6 +20,7 @@ Functions:
   sdpa_window(q, k, v, causal, window, n_sink, scale, seqlens=None) -> (o, lse) sliding window + sinks
   dequant_e4m3(bytes, scale)                     -> fp64      FP8 (e4m3) cache values
   dequant_e4m3_tiles(bytes, scales, tile)        -> fp64      the same with one scale per token tile
+  sdpa_fp8(q8, k8, v8, q_s, k_s, v_s, causal, scale) -> (o, lse) sdpa of per-tile dequantised e4m3 operands
   rope_tables(n_pos, d, base)                    -> (cos, sin) rotary tables [n_pos, d/2]
   rope(x, cos, sin, positions)                   -> fp64      rotary position embedding
   sdpa_rope(q, k, v, causal, scale, cos, sin)    -> (o, lse)  sdpa on rotated (bf16) queries and keys
@@ -327,6 +328,21 @@ def dequant_e4m3_tiles(raw, scales, tile: int = 128):
     S = val.shape[2]
     tok_tile = np.arange(S) // tile                      # tile of each token
     return val * sc[:, :, tok_tile][..., None]
+
+
+def sdpa_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal: bool, scale: float, tile: int = 128,
+             nthreads=None, lib=None):
+    """Attention over FP8 (e4m3) queries, keys and values with one scale per
+    tile of `tile` rows of each (sequence, head) ("Flash Attention 3 and
+    Multi-Headed Latent Attention", FP8 section: e4m3 operands with per-tile
+    scaling factors): each operand is dequantised (dequant_e4m3_tiles), then
+    the plain definition (sdpa) runs on the values. q8 [B, n_q, Sq, d],
+    k8 / v8 [B, n_kv, Skv, d] bytes; q_scale [B, n_q, ceil(Sq / tile)],
+    k_scale / v_scale [B, n_kv, ceil(Skv / tile)]."""
+    q = dequant_e4m3_tiles(q8, q_scale, tile)
+    k = dequant_e4m3_tiles(k8, k_scale, tile)
+    v = dequant_e4m3_tiles(v8, v_scale, tile)
+    return sdpa(q, k, v, causal, scale, nthreads=nthreads, lib=lib)
 
 
 def rope_tables(n_pos: int, d: int, base: float, lib=None):

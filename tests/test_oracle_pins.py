@@ -150,3 +150,34 @@ def test_round_bf16_matches_torch():
     x = torch.cat([x, ties])
     ref = x.to(torch.bfloat16).double().numpy()
     assert np.array_equal(oracle.round_bf16(x.double().numpy()), ref)
+
+
+def test_sdpa_fp8_scaling_and_tiles():
+    """The FP8 oracle mode against closed forms. Uniform power-of-two scales
+    2^a, 2^b, 2^c on q, k, v: the scores scale by 2^(a+b) (the softmax scale
+    times 2^(a+b) on the unscaled values) and the output by 2^c, exactly in
+    fp64. Per-tile scales: query rows of tile 1 and key rows of tiles 1 and
+    2 carry their own factors, which must land on rows 128.. and 256..
+    (compared with sdpa on values multiplied row by row)."""
+    rng = np.random.default_rng(9)
+    B, n_q, n_kv, Sq, Skv, d = 1, 4, 2, 200, 300, 16
+    q8 = rng.integers(0, 126, size=(B, n_q, Sq, d)).astype(np.uint8) | (rng.integers(0, 2, (B, n_q, Sq, d)) << 7).astype(np.uint8)
+    k8 = rng.integers(0, 120, size=(B, n_kv, Skv, d)).astype(np.uint8)
+    v8 = rng.integers(0, 126, size=(B, n_kv, Skv, d)).astype(np.uint8)
+    q, k, v = oracle.dequant_e4m3(q8), oracle.dequant_e4m3(k8), oracle.dequant_e4m3(v8)
+    tq, tk = (Sq + 127) // 128, (Skv + 127) // 128
+    for causal in (False, True):
+        o, lse = oracle.sdpa_fp8(q8, k8, v8, np.full((B, n_q, tq), 0.25), np.full((B, n_kv, tk), 2.0),
+                                 np.full((B, n_kv, tk), 8.0), causal, 0.1)
+        o_ref, lse_ref = oracle.sdpa(q, k, v, causal, 0.1 * 0.25 * 2.0)
+        assert np.allclose(o, 8.0 * o_ref, rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
+    qs = np.ones((B, n_q, tq)); qs[:, :, 1] = 3.0
+    ks = np.ones((B, n_kv, tk)); ks[:, :, 1] = 0.5; ks[:, :, 2] = 2.0
+    vs = np.ones((B, n_kv, tk)); vs[:, :, 2] = 4.0
+    qm = np.where(np.arange(Sq) >= 128, 3.0, 1.0)[None, None, :, None]
+    km = np.select([np.arange(Skv) >= 256, np.arange(Skv) >= 128], [2.0, 0.5], 1.0)[None, None, :, None]
+    vm = np.where(np.arange(Skv) >= 256, 4.0, 1.0)[None, None, :, None]
+    o, lse = oracle.sdpa_fp8(q8, k8, v8, qs, ks, vs, True, 0.1)
+    o_ref, lse_ref = oracle.sdpa(q * qm, k * km, v * vm, True, 0.1)
+    assert np.allclose(o, o_ref, rtol=1e-12, atol=1e-12) and np.allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
