@@ -80,6 +80,38 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
              int causal, float scale, attn_stream_t stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd on FP8 (e4m3) queries, keys and values with one
+ * scale per 128-row tile.
+ * Source: "Flash Attention 3 and Multi-Headed Latent Attention", FP8 section
+ * (e4m3 operands, largest finite 448, with scaling factors per tile).
+ *
+ *   q8  [B, n_q,  Sq,  d] e4m3 bytes, contiguous (BHSD)
+ *   k8  [B, n_kv, Skv, d] e4m3 bytes, contiguous
+ *   v8  [B, n_kv, Skv, d] e4m3 bytes, contiguous
+ *   q_scale [B, n_q,  ceil(Sq / 128)]  fp32: row i of (b, h) means
+ *           e4m3(q8[b][h][i]) * q_scale[b][h][i / 128]
+ *   k_scale, v_scale [B, n_kv, ceil(Skv / 128)] fp32, likewise for keys and
+ *           values (finite and > 0; other values give undefined results)
+ *   o, lse, causal, scale: as attn_fwd (o bf16, lse fp32 natural log)
+ *   workspace: device scratch of at least attn_fwd_fp8_workspace_bytes(...)
+ *           bytes, 256-byte aligned, contents on entry irrelevant; calls that
+ *           share it must be ordered on one stream.
+ * The result is attn_fwd of the dequantised operands. Computed as: the
+ * e4m3 values widened to f16 into the workspace (exact), then the attention
+ * kernel with f16 tensor-core operands, the query and key tile scales
+ * folded into each score tile's exponent scale and the value tile's scale
+ * into P (the row sums take P unscaled). Two launches on `stream`.
+ * Supported: d == 128, and the rest as attn_fwd.
+ * Returns ATTN_OK or an error code (nothing launched on error).
+ */
+int attn_fwd_fp8_workspace_bytes(int B, int Sq, int Skv, int n_q, int n_kv, int d, size_t *bytes);
+int attn_fwd_fp8(const void *q8, const void *k8, const void *v8,
+                 const float *q_scale, const float *k_scale, const float *v_scale,
+                 void *o, float *lse, int B, int Sq, int Skv, int n_q, int n_kv, int d,
+                 int causal, float scale, void *workspace, size_t workspace_bytes,
+                 attn_stream_t stream);
+
+/*
  * attn_fwd_window -- causal attn_fwd with a sliding window and sink keys.
  * Source: "Attention deep dive" (askaiml.pages.dev), section 6 (sliding-window
  * attention: token i attends to the last W tokens, mask (j <= i) AND

@@ -52,6 +52,10 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         L.attn_fwd.argtypes = [_vp] * 5 + [_i] * 8 + [ctypes.c_float, _vp]
         L.attn_fwd.restype = _i
+        L.attn_fwd_fp8_workspace_bytes.argtypes = [_i] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
+        L.attn_fwd_fp8_workspace_bytes.restype = _i
+        L.attn_fwd_fp8.argtypes = [_vp] * 8 + [_i] * 7 + [ctypes.c_float, _vp, ctypes.c_size_t, _vp]
+        L.attn_fwd_fp8.restype = _i
         L.attn_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 9 + [ctypes.c_float, _vp]
         L.attn_fwd_window.argtypes = [_vp] * 5 + [_i] * 9 + [ctypes.c_float, _vp]
         L.attn_fwd_window.restype = _i
@@ -135,6 +139,44 @@ def attn_fwd(q, k, v, causal: bool, scale: float, o=None, lse=None, stream=None,
     rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, n_q, n_kv, d_qk, d_v,
                         int(bool(causal)), float(scale), ctypes.c_void_p(_stream(stream)))
     _check(rc, "attn_fwd")
+    return o, lse
+
+
+def fwd_fp8_workspace_bytes(B, Sq, Skv, n_q, n_kv, d) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().attn_fwd_fp8_workspace_bytes(B, Sq, Skv, n_q, n_kv, d, ctypes.byref(out)),
+           "attn_fwd_fp8_workspace_bytes")
+    return out.value
+
+
+def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal: bool, scale: float, o=None, lse=None,
+                 workspace=None, stream=None, want_lse=True):
+    """Prefill forward on e4m3 operands with one scale per 128-row tile.
+    q8 [B,n_q,Sq,d], k8/v8 [B,n_kv,Skv,d]: contiguous one-byte CUDA tensors
+    (float8_e4m3fn or uint8 bytes); q_scale [B,n_q,ceil(Sq/128)],
+    k_scale/v_scale [B,n_kv,ceil(Skv/128)]: contiguous fp32 CUDA tensors.
+    Returns (o [B,n_q,Sq,d] bf16, lse [B,n_q,Sq] fp32 or None)."""
+    B, n_q, Sq, d = q8.shape
+    _, n_kv, Skv, _ = k8.shape
+    for t in (q8, k8, v8):
+        if t.element_size() != 1 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q8, k8, v8 must be contiguous one-byte CUDA tensors")
+    shapes = ((q_scale, (B, n_q, (Sq + 127) // 128)), (k_scale, (B, n_kv, (Skv + 127) // 128)),
+              (v_scale, (B, n_kv, (Skv + 127) // 128)))
+    for t, shp in shapes:
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shp:
+            raise ValueError(f"scales must be contiguous fp32 CUDA tensors of shape {shp}")
+    if o is None:
+        o = torch.empty((B, n_q, Sq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Sq), dtype=torch.float32, device=q8.device)
+    if workspace is None:
+        workspace = torch.empty(max(fwd_fp8_workspace_bytes(B, Sq, Skv, n_q, n_kv, d), 1), dtype=torch.uint8,
+                                device=q8.device)
+    rc = lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _ptr(o),
+                            _ptr(lse), B, Sq, Skv, n_q, n_kv, d, int(bool(causal)), float(scale), _ptr(workspace),
+                            workspace.numel(), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "attn_fwd_fp8")
     return o, lse
 
 

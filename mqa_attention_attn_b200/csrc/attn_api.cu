@@ -14,6 +14,7 @@
 #include "../../include/attn.h"
 #include "decode_gqa.cuh"
 #include "decode_mla.cuh"
+#include "fp8_widen.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -117,11 +118,24 @@ struct VarlenArgs {
     int64_t ks[3] = {0, 0, 0}, vs[3] = {0, 0, 0};   // page, token, head
 };
 
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+// Workspace of the FP8 prefill: q, k and v widened to f16, each 256-byte aligned.
+size_t fp8_prefill_ws_bytes(int B, int Sq, int Skv, int n_q, int n_kv, int d) {
+    return align256((size_t)B * n_q * Sq * d * 2) + 2 * align256((size_t)B * n_kv * Skv * d * 2);
+}
+
+// Per-tile scales of the FP8 prefill (q, k, v then hold the widened values).
+struct Fp8Args {
+    const float *q_scale, *k_scale, *v_scale;
+};
+
 template <int D>
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,
                    int n_q, int n_kv, int causal, float scale, cudaStream_t stream, const VarlenArgs *vl = nullptr,
-                   int window = 0, int n_sink = 0, const attn::rope::Tables *rope = nullptr) {
+                   int window = 0, int n_sink = 0, const attn::rope::Tables *rope = nullptr,
+                   const Fp8Args *f8 = nullptr) {
     using attn::pf::kDense;
+    using attn::pf::kFp8;
     using attn::pf::kPaged;
     using attn::pf::kRope;
     using attn::pf::kVarlen;
@@ -141,6 +155,14 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     p.window = window;
     p.n_sink = n_sink;
     if (rope) p.rope = *rope;
+    if (f8) {
+        if (D != 128 || vl || rope || window > 0) return ATTN_ERR_UNSUPPORTED;
+        p.q_scale = f8->q_scale;
+        p.k_scale = f8->k_scale;
+        p.v_scale = f8->v_scale;
+        p.q_tiles = (Sq + attn::pf::BM - 1) / attn::pf::BM;
+        p.k_tiles = (Skv + attn::pf::BN - 1) / attn::pf::BN;
+    }
     p.o = reinterpret_cast<__nv_bfloat16 *>(o);
     const int Sq_plan = vl ? vl->max_q : Sq;   // position blocks cover the longest sequence
     if (G >= 2) {
@@ -215,6 +237,10 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kPaged>, smem, attr_done_p)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kWindow>, smem, attr_done_w)) return ATTN_ERR_CUDA;
     if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kRope>, smem, attr_done_r)) return ATTN_ERR_CUDA;
+    if constexpr (D == 128) {
+        static std::atomic<uint64_t> attr_done_f{0};
+        if (!ensure_smem_attr(attn::pf::prefill_kernel<D, kFp8>, smem, attr_done_f)) return ATTN_ERR_CUDA;
+    }
     // The kernel rebalances registers between warpgroups (setmaxnreg); that is
     // only safe if it was built with exactly the register count the split
     // assumes, otherwise the increase could never be granted.
@@ -227,9 +253,15 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
         if (cudaFuncGetAttributes(&fw, attn::pf::prefill_kernel<D, kWindow>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fr, attn::pf::prefill_kernel<D, kRope>) != cudaSuccess) return ATTN_ERR_CUDA;
         if (cudaFuncGetAttributes(&fp, attn::pf::prefill_kernel<D, kPaged>) != cudaSuccess) return ATTN_ERR_CUDA;
+        bool f8_ok = true;
+        if constexpr (D == 128) {
+            cudaFuncAttributes ff;
+            if (cudaFuncGetAttributes(&ff, attn::pf::prefill_kernel<D, kFp8>) != cudaSuccess) return ATTN_ERR_CUDA;
+            f8_ok = ff.numRegs == attn::pf::kLaunchRegs;
+        }
         regs_checked.store((fa.numRegs == attn::pf::kLaunchRegs && fv.numRegs == attn::pf::kLaunchRegs &&
                             fw.numRegs == attn::pf::kLaunchRegs && fr.numRegs == attn::pf::kLaunchRegs &&
-                            fp.numRegs == attn::pf::kLaunchRegs) ? 1 : -1,
+                            fp.numRegs == attn::pf::kLaunchRegs && f8_ok) ? 1 : -1,
                            std::memory_order_release);
     }
     if (regs_checked.load(std::memory_order_acquire) < 0) return ATTN_ERR_UNSUPPORTED;
@@ -267,10 +299,14 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
             cfg.numAttrs = 1;
             if (cudaLaunchKernelEx(&cfg, attn::pf::prefill_kernel<D, kRope>, tq, tk, tv, to, p) != cudaSuccess)
                 return ATTN_ERR_CUDA;
-        } else if (window > 0)
+        } else if (window > 0) {
             attn::pf::prefill_kernel<D, kWindow><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
                                                                                                        p);
-        else
+        } else if (f8) {
+            if constexpr (D == 128)
+                attn::pf::prefill_kernel<D, kFp8><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
+                                                                                                        p);
+        } else
             attn::pf::prefill_kernel<D, kDense><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
                                                                                                       p);
     }
@@ -590,6 +626,53 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, i
         case 64: return launch_prefill<64>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
         default: return launch_prefill<128>(q, k, v, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s);
     }
+}
+
+int attn_fwd_fp8_workspace_bytes(int B, int Sq, int Skv, int n_q, int n_kv, int d, size_t *bytes) {
+    if (!bytes || B < 0 || Sq < 0 || Skv < 1 || n_q < 1 || n_kv < 1 || d < 1) return ATTN_ERR_INVALID_ARG;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    *bytes = fp8_prefill_ws_bytes(B, Sq, Skv, n_q, n_kv, d);
+    return ATTN_OK;
+}
+
+int attn_fwd_fp8(const void *q8, const void *k8, const void *v8, const float *q_scale, const float *k_scale,
+                 const float *v_scale, void *o, float *lse, int B, int Sq, int Skv, int n_q, int n_kv, int d,
+                 int causal, float scale, void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+    if (B < 0 || Sq < 0 || Skv < 1 || n_q < 1 || n_kv < 1 || d < 1) return ATTN_ERR_INVALID_ARG;
+    if (n_q % n_kv != 0) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+    if (B == 0 || Sq == 0) return ATTN_OK;
+    if (!q8 || !k8 || !v8 || !q_scale || !k_scale || !v_scale || !o) return ATTN_ERR_INVALID_ARG;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    const int G = n_q / n_kv;
+    if (!is_pow2(G) || G > 256) return ATTN_ERR_UNSUPPORTED;
+    if (causal && Sq > Skv) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)B * n_q > 0x7fffffffLL || (long long)B * n_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o)) return ATTN_ERR_MISALIGNED;
+    const size_t need = fp8_prefill_ws_bytes(B, Sq, Skv, n_q, n_kv, d);
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // widen the three operands into the workspace (f16, same layouts)
+    const size_t nq = (size_t)B * n_q * Sq * d, nk = (size_t)B * n_kv * Skv * d;
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    uint16_t *q16 = reinterpret_cast<uint16_t *>(ws);
+    uint16_t *k16 = reinterpret_cast<uint16_t *>(ws + align256(nq * 2));
+    uint16_t *v16 = reinterpret_cast<uint16_t *>(ws + align256(nq * 2) + align256(nk * 2));
+    const attn::f8::WidenSeg sq{reinterpret_cast<const uint8_t *>(q8), q16, nq / 16};
+    const attn::f8::WidenSeg sk{reinterpret_cast<const uint8_t *>(k8), k16, nk / 16};
+    const attn::f8::WidenSeg sv{reinterpret_cast<const uint8_t *>(v8), v16, nk / 16};
+    const size_t groups = (nq + 2 * nk) / 16;
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return ATTN_ERR_CUDA;
+    const size_t want = (groups + attn::f8::WIDEN_THREADS - 1) / attn::f8::WIDEN_THREADS;
+    const int grid = (int)(want < (size_t)n_sm * 8 ? want : (size_t)n_sm * 8);
+    attn::f8::widen_e4m3_kernel<<<grid, attn::f8::WIDEN_THREADS, 0, s>>>(sq, sk, sv);
+    if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    const Fp8Args f8{q_scale, k_scale, v_scale};
+    return launch_prefill<128>(q16, k16, v16, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s, nullptr, 0, 0,
+                               nullptr, &f8);
 }
 
 int attn_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Skv,

@@ -217,21 +217,6 @@ __device__ __forceinline__ bool next_unit(UnitCursor &cur, long long i, const in
     return false;
 }
 
-// Widen 8 bytes of e4m3 values (two words) to 8 f16 values (four words).
-// e4m3 -> f16 is exact (every e4m3 value is an f16 value).
-__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
-    uint4 r;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.x) : "h"((unsigned short)(lo & 0xffffu)));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.y) : "h"((unsigned short)(lo >> 16)));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.z) : "h"((unsigned short)(hi & 0xffffu)));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.w) : "h"((unsigned short)(hi >> 16)));
-    return r;
-}
-__device__ __forceinline__ uint32_t f2_to_h2_sat(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
 
 template <int GT, bool PAGED, bool FP8 = false>
 __global__ void __launch_bounds__(FP8 ? THREADS_FP8 : THREADS, (FP8 && GT >= 16) ? 1 : 2)

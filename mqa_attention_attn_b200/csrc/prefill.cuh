@@ -172,6 +172,12 @@ struct Params {
     // prefetched into L2 by this one (0: none). With one CTA per SM and the
     // grid taken in index order, that CTA starts once this wave drains.
     int l2_ahead;
+    // FP8 inputs (the FP8 kernel, BHSD as the dense one): q, k, v hold the
+    // e4m3 values widened to f16 (exact); element (b, h, i, c) means
+    // value * scale[b][h][i / 128] with q_scale [B][n_q][q_tiles] and
+    // k_scale, v_scale [B][n_kv][k_tiles].
+    const float *q_scale, *k_scale, *v_scale;
+    int q_tiles, k_tiles;
 };
 
 template <bool B>
@@ -189,8 +195,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 
 // MODE: kDense (BHSD batch), kVarlen (packed batch), kWindow (BHSD, causal
 // sliding window with sink keys), kRope (BHSD batch, queries rotated here),
-// kPaged (packed queries, keys and values in a paged cache).
-enum : int { kDense = 0, kVarlen = 1, kWindow = 2, kRope = 3, kPaged = 4 };
+// kPaged (packed queries, keys and values in a paged cache), kFp8 (BHSD
+// batch of e4m3 values widened to f16, one scale per 128-row tile: f16
+// MMAs, the query and key tile scales folded into the exponent's scale, the
+// value tile's scale into P).
+enum : int { kDense = 0, kVarlen = 1, kWindow = 2, kRope = 3, kPaged = 4, kFp8 = 5 };
 
 // One 128-key tile of a paged K or V pool into shared memory (the PAGED
 // kernel): box x of the tile holds keys key0 + x * box_rows .. + box_rows - 1,
@@ -230,6 +239,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr bool PACKED = VARLEN || PAGED;      // queries packed [total_q][n_q][D]
     constexpr bool WINDOW = MODE == kWindow;
     constexpr bool ROPE = MODE == kRope;
+    constexpr bool FP8 = MODE == kFp8;
     extern __shared__ uint8_t smem_raw[];
     Smem<D> &sm = *reinterpret_cast<Smem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -491,8 +501,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp == 1) {
         // ======================= MMA issuer =======================
         if (lane == 0) {
-            const uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0, 0);
-            const uint32_t idesc_o = umma_idesc_bf16(BM, D, 0, 1);
+            const uint32_t idesc_s = FP8 ? umma_idesc_f16(BM, BN, 0, 0) : umma_idesc_bf16(BM, BN, 0, 0);
+            const uint32_t idesc_o = FP8 ? umma_idesc_f16(BM, D, 0, 1) : umma_idesc_bf16(BM, D, 0, 1);
             bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x21);
             // Descriptors are built once per operand tile and stepped by
             // constant offsets in their 16-byte address field: for shared
@@ -612,8 +622,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             float m_run = -INFINITY, l_run = 0.f;
             bool ok = true;
             const int ntt = nt[t];
-            const float2 sl2 = make_float2(sl, sl);
+            // FP8: this row's query tile scale (rows past Sq hold no query)
+            const float qsr = (FP8 && pos < Sq)
+                                  ? __ldg(p.q_scale + ((size_t)b * p.n_q + head) * p.q_tiles + pos / BM) : 1.f;
+            const size_t kvsrow = FP8 ? ((size_t)b * p.n_kv + kvh) * p.k_tiles : 0;
             for (int j = 0; j < ntt; ++j) {
+                // FP8: key and value tile scales of tile j (loaded before the
+                // wait for its scores)
+                const float ksj = FP8 ? __ldg(p.k_scale + kvsrow + j) : 1.f;
+                const float vsj = FP8 ? __ldg(p.v_scale + kvsrow + j) : 1.f;
                 ok = warp_wait(smem_u32(&sm.s_full[t]), j & 1, abort_flag, 0x31);
                 if (!ok) break;
                 __syncwarp();
@@ -653,7 +670,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     mx3 = fmax3(mx3, __uint_as_float(x[e + 6]), __uint_as_float(x[e + 7]));
                 }
                 const float mx = fmaxf(fmax3(mx0, mx1, mx2), mx3);
-                const float m_new = fmaxf(m_run, mx * sl);
+                // scale * log2(e), times the query and key tile scales (FP8)
+                const float slj = FP8 ? sl * qsr * ksj : sl;
+                const float2 sl2 = make_float2(slj, slj);
+                const float m_new = fmaxf(m_run, mx * slj);
                 if (j == 0) {
                     m_run = m_new;
                 } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold)) {
@@ -708,7 +728,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             pe = make_float2(ex2(t2.x), ex2(t2.y));
                         }
                         rs = fadd2(rs, pe);
-                        pk[e] = f2_to_bf2(pe.x, pe.y);
+                        // FP8: P times the value tile's scale, as f16 (the
+                        // MMA's other operand); the row sum takes P unscaled
+                        pk[e] = FP8 ? f2_to_h2_sat(pe.x * vsj, pe.y * vsj) : f2_to_bf2(pe.x, pe.y);
                     }
                 };
 #pragma unroll

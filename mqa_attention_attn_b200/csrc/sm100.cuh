@@ -339,6 +339,23 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 // two fp32 -> bf16x2 word (round to nearest even), `lo` in the low half
+// Widen 8 bytes of e4m3 values (two words) to 8 f16 values (four words).
+// e4m3 -> f16 is exact (every e4m3 value is an f16 value).
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint32_t lo, uint32_t hi) {
+    uint4 r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.x) : "h"((unsigned short)(lo & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.y) : "h"((unsigned short)(lo >> 16)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.z) : "h"((unsigned short)(hi & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r.w) : "h"((unsigned short)(hi >> 16)));
+    return r;
+}
+// Two fp32 values to f16x2 (lo in the low half), round to nearest even,
+// values beyond the f16 range saturated to +-65504.
+__device__ __forceinline__ uint32_t f2_to_h2_sat(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
 __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
     __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&t);

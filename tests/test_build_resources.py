@@ -33,7 +33,8 @@ def test_no_spills_and_prefill_register_count():
     launch_regs = int(re.search(r"constexpr int kLaunchRegs = (\d+);",
                                 open(os.path.join(build.CSRC, "prefill.cuh")).read()).group(1))
     prefill = {n: v for n, v in ks.items() if "prefill_kernel" in n}
-    assert len(prefill) == 15, sorted(prefill)            # d in {32, 64, 128} x five modes
+    # d in {32, 64, 128} x five modes, and the FP8 mode at d = 128
+    assert len(prefill) == 16, sorted(prefill)
     assert any("mla_decode_kernel" in n for n in ks)
     assert sum("decode_split_kernel" in n for n in ks) >= 15
     for name, (regs, st, ld) in ks.items():
