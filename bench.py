@@ -466,6 +466,17 @@ def run_ours(args):
         of8t, lf8t = torch.empty_like(od), torch.empty_like(ld)
         add("fp8_decode_tiles", "next", 2, lambda: binding.attn_decode_fp8_tiles(
             qd, k8t, v8t, kst, vst, sl_dev, wd.scale, o=of8t, lse=lf8t, workspace=work8, stream=stream))
+        # the Llama-3-8B prefill with Q, K and V in e4m3, one scale per 128-row
+        # tile of each (sequence, head): the widening pass and the attention
+        q8p, qsp = to_e4m3_tiles(q)
+        k8p, ksp = to_e4m3_tiles(k)
+        v8p, vsp = to_e4m3_tiles(v)
+        o_f8p, lse_f8p = torch.empty_like(o), torch.empty_like(lse)
+        work_f8p = torch.empty(binding.fwd_fp8_workspace_bytes(w.B, w.Sq, w.Skv, w.n_q, w.n_kv, w.d_qk),
+                               dtype=torch.uint8, device=dev)
+        add("fp8_prefill", "next", 2, lambda: binding.attn_fwd_fp8(
+            q8p, k8p, v8p, qsp, ksp, vsp, w.causal, w.scale, o=o_f8p, lse=lse_f8p, workspace=work_f8p,
+            stream=stream))
 
     # the Llama-3-8B prefill with its keys and values in 64-token pages placed
     # in a pool in a seeded random order (chunked-prefill serving layout)
@@ -786,6 +797,15 @@ def run_ours(args):
                                               "decode_combine_kernel",
                                    "roofline": hbm_roofline(by_ft, ms_ft, "attn::dec::decode_split_kernel<4, fp8>",
                                                             None, "achieved over split + merge launches")}
+    if "fp8_prefill" in regimes:
+        ms_fp = mean["fp8_prefill"]
+        out["fp8_prefill"] = {"workload": f"{w.name}, e4m3 q, k, v with one scale per 128-row tile",
+                              "ms": ms_fp, "tflops": tf(fl_p, ms_fp), "frac_of_peak": tf(fl_p, ms_fp) / peak_tf,
+                              "kernels": "attn::f8::widen_e4m3_kernel (e4m3 -> f16 into the workspace) + "
+                                         "attn::pf::prefill_kernel<128, fp8> (f16 MMAs, tile scales folded in)",
+                              "roofline": tensor_roofline(fl_p, ms_fp, "attn::pf::prefill_kernel<128, fp8>", None,
+                                                          "achieved over both launches; f16 operands run at the "
+                                                          "bf16 rate")}
     if "rope_prefill" in regimes:
         ms_rp, ms_rd = mean["rope_prefill"], mean["rope_decode"]
         out["rope_prefill"] = {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": ms_rp,

@@ -173,7 +173,7 @@ struct Params {
     // grid taken in index order, that CTA starts once this wave drains.
     int l2_ahead;
     // FP8 inputs (the FP8 kernel, BHSD as the dense one): q, k, v hold the
-    // e4m3 values widened to f16 (exact); element (b, h, i, c) means
+    // e4m3 values widened to bf16 (exact); element (b, h, i, c) means
     // value * scale[b][h][i / 128] with q_scale [B][n_q][q_tiles] and
     // k_scale, v_scale [B][n_kv][k_tiles].
     const float *q_scale, *k_scale, *v_scale;
@@ -196,9 +196,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // MODE: kDense (BHSD batch), kVarlen (packed batch), kWindow (BHSD, causal
 // sliding window with sink keys), kRope (BHSD batch, queries rotated here),
 // kPaged (packed queries, keys and values in a paged cache), kFp8 (BHSD
-// batch of e4m3 values widened to f16, one scale per 128-row tile: f16
-// MMAs, the query and key tile scales folded into the exponent's scale, the
-// value tile's scale into P).
+// batch of e4m3 values widened to bf16, one scale per 128-row tile: the
+// query and key tile scales folded into the exponent's scale, the value
+// tile's scale into P).
 enum : int { kDense = 0, kVarlen = 1, kWindow = 2, kRope = 3, kPaged = 4, kFp8 = 5 };
 
 // One 128-key tile of a paged K or V pool into shared memory (the PAGED
@@ -501,8 +501,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp == 1) {
         // ======================= MMA issuer =======================
         if (lane == 0) {
-            const uint32_t idesc_s = FP8 ? umma_idesc_f16(BM, BN, 0, 0) : umma_idesc_bf16(BM, BN, 0, 0);
-            const uint32_t idesc_o = FP8 ? umma_idesc_f16(BM, D, 0, 1) : umma_idesc_bf16(BM, D, 0, 1);
+            const uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0, 0);
+            const uint32_t idesc_o = umma_idesc_bf16(BM, D, 0, 1);
             bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x21);
             // Descriptors are built once per operand tile and stepped by
             // constant offsets in their 16-byte address field: for shared
@@ -626,11 +626,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float qsr = (FP8 && pos < Sq)
                                   ? __ldg(p.q_scale + ((size_t)b * p.n_q + head) * p.q_tiles + pos / BM) : 1.f;
             const size_t kvsrow = FP8 ? ((size_t)b * p.n_kv + kvh) * p.k_tiles : 0;
+            // FP8: key and value tile scales, loaded one tile ahead
+            float ks_next = (FP8 && ntt > 0) ? __ldg(p.k_scale + kvsrow) : 1.f;
+            float vs_next = (FP8 && ntt > 0) ? __ldg(p.v_scale + kvsrow) : 1.f;
             for (int j = 0; j < ntt; ++j) {
-                // FP8: key and value tile scales of tile j (loaded before the
-                // wait for its scores)
-                const float ksj = FP8 ? __ldg(p.k_scale + kvsrow + j) : 1.f;
-                const float vsj = FP8 ? __ldg(p.v_scale + kvsrow + j) : 1.f;
+                const float ksj = ks_next, vsj = vs_next;
+                if (FP8 && j + 1 < ntt) {
+                    ks_next = __ldg(p.k_scale + kvsrow + j + 1);
+                    vs_next = __ldg(p.v_scale + kvsrow + j + 1);
+                }
                 ok = warp_wait(smem_u32(&sm.s_full[t]), j & 1, abort_flag, 0x31);
                 if (!ok) break;
                 __syncwarp();
@@ -708,7 +712,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // a row with no visible key yet keeps m = -inf: exponentiate
                 // against 0 instead (every p is then 0)
                 const float m_use = ((PACKED || WINDOW) && m_run == -INFINITY) ? 0.f : m_run;
-                const float2 nm2 = make_float2(-m_use, -m_use);
+                // FP8: the value tile's scale joins the exponent (P is formed
+                // already multiplied by it; the row sum divides it out per tile)
+                const float lvs = FP8 ? __log2f(vsj) : 0.f;
+                const float2 nm2 = make_float2(lvs - m_use, lvs - m_use);
                 float2 rs = make_float2(0.f, 0.f);
                 // one chunk of exponentials; which pairs take the FMA-pipe
                 // polynomial is fixed at compile time (never on masked tiles)
@@ -728,9 +735,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             pe = make_float2(ex2(t2.x), ex2(t2.y));
                         }
                         rs = fadd2(rs, pe);
-                        // FP8: P times the value tile's scale, as f16 (the
-                        // MMA's other operand); the row sum takes P unscaled
-                        pk[e] = FP8 ? f2_to_h2_sat(pe.x * vsj, pe.y * vsj) : f2_to_bf2(pe.x, pe.y);
+                        pk[e] = f2_to_bf2(pe.x, pe.y);   // FP8: times the value tile's scale
                     }
                 };
 #pragma unroll
@@ -750,7 +755,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tc_fence_before();
                     mbar_arrive(smem_u32(&sm.p_full[t][c]));
                 }
-                l_run += rs.x + rs.y;
+                l_run += FP8 ? (rs.x + rs.y) * __frcp_rn(vsj) : rs.x + rs.y;
             }
             // ---- epilogue: O / l -> bf16 -> swizzled smem -> TMA store; LSE
             if (ok && ntt > 0) ok = warp_wait(smem_u32(&sm.o_done[t]), 0, abort_flag, 0x33);

@@ -1,7 +1,7 @@
 """attn_fwd_fp8 (e4m3 Q, K, V with one scale per 128-row tile) on the GPU
 against the fp64 oracle's FP8 mode (per-tile dequantisation, then the plain
 definition). The kernel sees the same e4m3 bytes and scales; its operands
-are the exact f16 images of the bytes, so the tolerances are the bf16
+are the exact bf16 images of the bytes, so the tolerances are the bf16
 path's."""
 import math
 
