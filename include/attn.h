@@ -97,11 +97,12 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
  *           bytes, 256-byte aligned, contents on entry irrelevant; calls that
  *           share it must be ordered on one stream.
  * The result is attn_fwd of the dequantised operands. Computed as: the
- * e4m3 values widened to bf16 into the workspace (exact: every e4m3 value
- * is a bf16 value), then the attention kernel on those tiles, the query and
- * key tile scales folded into each score tile's exponent scale and the
- * value tile's scale into P (the row sums take P unscaled). Two launches
- * on `stream`.
+ * e4m3 keys and values widened to bf16 into the workspace (exact: every
+ * e4m3 value is a bf16 value), then the attention kernel, which loads the
+ * e4m3 query tiles and widens them in shared memory, folds the query and
+ * key tile scales into each score tile's exponent scale and the value
+ * tile's scale into P (the row sums take P unscaled). Two launches on
+ * `stream`.
  * Supported: d == 128, and the rest as attn_fwd.
  * Returns ATTN_OK or an error code (nothing launched on error).
  */

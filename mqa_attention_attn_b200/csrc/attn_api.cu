@@ -119,9 +119,10 @@ struct VarlenArgs {
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-// Workspace of the FP8 prefill: q, k and v widened to f16, each 256-byte aligned.
+// Workspace of the FP8 prefill: k and v widened to bf16, each 256-byte aligned.
 size_t fp8_prefill_ws_bytes(int B, int Sq, int Skv, int n_q, int n_kv, int d) {
-    return align256((size_t)B * n_q * Sq * d * 2) + 2 * align256((size_t)B * n_kv * Skv * d * 2);
+    (void)Sq, (void)n_q;
+    return 2 * align256((size_t)B * n_kv * Skv * d * 2);
 }
 
 // Per-tile scales of the FP8 prefill (q, k, v then hold the widened values).
@@ -218,7 +219,14 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
             const uint64_t dims[3] = {(uint64_t)D, (uint64_t)Sq, (uint64_t)B * n_q};
             const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)Sq * D * 2};
             const uint32_t box[3] = {(uint32_t)C::BOXD, (uint32_t)p.Pt, (uint32_t)p.Ht};
-            if (!make_map(&tq, q, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
+            if (f8) {
+                // FP8: q holds e4m3 bytes, one 128-byte row per query row
+                const uint64_t str8[2] = {(uint64_t)D, (uint64_t)Sq * D};
+                const uint32_t box8[3] = {(uint32_t)D, (uint32_t)p.Pt, (uint32_t)p.Ht};
+                if (!make_map(&tq, q, 3, dims, str8, box8, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return ATTN_ERR_CUDA;
+            } else if (!make_map(&tq, q, 3, dims, str, box, C::ROWB)) {
+                return ATTN_ERR_CUDA;
+            }
             if (!make_map(&to, o, 3, dims, str, box, C::ROWB)) return ATTN_ERR_CUDA;
         }
         {
@@ -654,24 +662,25 @@ int attn_fwd_fp8(const void *q8, const void *k8, const void *v8, const float *q_
     if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // widen the three operands into the workspace (f16, same layouts)
-    const size_t nq = (size_t)B * n_q * Sq * d, nk = (size_t)B * n_kv * Skv * d;
+    // keys and values widened into the workspace (bf16, same layouts; every
+    // CTA of a KV head reads them); the queries are widened by the attention
+    // kernel itself, each tile once, in shared memory
+    const size_t nk = (size_t)B * n_kv * Skv * d;
     uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
-    uint16_t *q16 = reinterpret_cast<uint16_t *>(ws);
-    uint16_t *k16 = reinterpret_cast<uint16_t *>(ws + align256(nq * 2));
-    uint16_t *v16 = reinterpret_cast<uint16_t *>(ws + align256(nq * 2) + align256(nk * 2));
-    const attn::f8::WidenSeg sq{reinterpret_cast<const uint8_t *>(q8), q16, nq / 16};
+    uint16_t *k16 = reinterpret_cast<uint16_t *>(ws);
+    uint16_t *v16 = reinterpret_cast<uint16_t *>(ws + align256(nk * 2));
     const attn::f8::WidenSeg sk{reinterpret_cast<const uint8_t *>(k8), k16, nk / 16};
     const attn::f8::WidenSeg sv{reinterpret_cast<const uint8_t *>(v8), v16, nk / 16};
-    const size_t groups = (nq + 2 * nk) / 16;
+    const attn::f8::WidenSeg none{nullptr, nullptr, 0};
+    const size_t groups = 2 * nk / 16;
     const int n_sm = sm_count();
     if (n_sm <= 0) return ATTN_ERR_CUDA;
     const size_t want = (groups + attn::f8::WIDEN_THREADS - 1) / attn::f8::WIDEN_THREADS;
     const int grid = (int)(want < (size_t)n_sm * 8 ? want : (size_t)n_sm * 8);
-    attn::f8::widen_e4m3_kernel<<<grid, attn::f8::WIDEN_THREADS, 0, s>>>(sq, sk, sv);
+    attn::f8::widen_e4m3_kernel<<<grid, attn::f8::WIDEN_THREADS, 0, s>>>(sk, sv, none);
     if (cudaPeekAtLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     const Fp8Args f8{q_scale, k_scale, v_scale};
-    return launch_prefill<128>(q16, k16, v16, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s, nullptr, 0, 0,
+    return launch_prefill<128>(q8, k16, v16, o, lse, B, Sq, Skv, n_q, n_kv, causal, scale, s, nullptr, 0, 0,
                                nullptr, &f8);
 }
 

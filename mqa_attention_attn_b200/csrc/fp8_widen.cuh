@@ -7,11 +7,8 @@
 // attention kernel.
 #pragma once
 
-#include <cuda_fp16.h>
-
 #include <cstddef>
 #include <cstdint>
-#include <cstring>
 
 #include "sm100.cuh"
 
@@ -28,18 +25,6 @@ struct WidenSeg {
 
 constexpr int WIDEN_THREADS = 256;
 
-// 8 e4m3 values (two words) to 8 bf16 values (four words): e4m3 -> f16 and
-// f16 -> fp32 are exact, and fp32 -> bf16 is exact for these values.
-__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint32_t lo, uint32_t hi) {
-    const uint4 h = e4m3x8_to_f16x8(lo, hi);
-    auto cv = [](uint32_t h2) {
-        __half2 v;
-        memcpy(&v, &h2, 4);
-        const float2 f = __half22float2(v);
-        return f2_to_bf2(f.x, f.y);
-    };
-    return make_uint4(cv(h.x), cv(h.y), cv(h.z), cv(h.w));
-}
 constexpr int WIDEN_UNROLL = 4;   // 16-byte loads in flight per thread
 
 // Groups i, i + stride, ... of one array: WIDEN_UNROLL independent loads

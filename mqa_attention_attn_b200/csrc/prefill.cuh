@@ -172,8 +172,9 @@ struct Params {
     // prefetched into L2 by this one (0: none). With one CTA per SM and the
     // grid taken in index order, that CTA starts once this wave drains.
     int l2_ahead;
-    // FP8 inputs (the FP8 kernel, BHSD as the dense one): q, k, v hold the
-    // e4m3 values widened to bf16 (exact); element (b, h, i, c) means
+    // FP8 inputs (the FP8 kernel, BHSD as the dense one): the q map reads
+    // the e4m3 bytes (one 128-byte box per row), k and v hold the e4m3
+    // values widened to bf16 (exact); element (b, h, i, c) means
     // value * scale[b][h][i / 128] with q_scale [B][n_q][q_tiles] and
     // k_scale, v_scale [B][n_kv][k_tiles].
     const float *q_scale, *k_scale, *v_scale;
@@ -240,6 +241,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr bool WINDOW = MODE == kWindow;
     constexpr bool ROPE = MODE == kRope;
     constexpr bool FP8 = MODE == kFp8;
+    static_assert(!FP8 || D == 128, "the FP8 mode stages one 128-byte e4m3 row per query row");
     extern __shared__ uint8_t smem_raw[];
     Smem<D> &sm = *reinterpret_cast<Smem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -326,11 +328,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tma_prefetch_desc(&tm_o);
         uint32_t qbytes = 0;
         for (int t = 0; t < 2; ++t)
-            if (nt[t] > 0) qbytes += C::QBYTES;
+            if (nt[t] > 0) qbytes += FP8 ? BM * D : C::QBYTES;
         const uint32_t qbar = smem_u32(&sm.q_full);
         mbar_arrive_expect_tx(qbar, qbytes);
         for (int t = 0; t < 2; ++t) {
             if (nt[t] == 0) continue;
+            if constexpr (FP8) {
+                // the tile's e4m3 rows (128 one-byte dims, 128-byte swizzled)
+                // into its second box, widened in place by its warpgroup
+                tma_load_3d(smem_u32(sm.q[t]) + C::QBOX, &tm_q, qbar, 0, p0[t], b * p.n_q + h0[t]);
+                continue;
+            }
             for (int bx = 0; bx < C::NBOX; ++bx)
                 if (PACKED)
                     tma_load_3d(smem_u32(sm.q[t]) + bx * C::QBOX, &tm_q, qbar, bx * C::BOXD, h0[t], q0 + p0[t]);
@@ -391,7 +399,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 int fh0, fp0;
                 tile_origin(fbh % p.n_kv, fpb, t, fh0, fp0);
                 if (fp0 >= Sq) continue;
-                for (int bx = 0; bx < C::NBOX; ++bx)
+                for (int bx = 0; bx < (FP8 ? 1 : C::NBOX); ++bx)
                     tma_prefetch_l2_3d(&tm_q, bx * C::BOXD, fp0, (fbh / p.n_kv) * p.n_q + fh0);
             }
         }
@@ -557,8 +565,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tc_fence_after();
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (nt[t] == 0) continue;
-                        // ROPE: this tile's rows have been rotated in place
-                        if (ROPE) ok = mbar_wait(smem_u32(&sm.q_rot[t]), 0, abort_flag, 0x27);
+                        // ROPE: this tile's rows have been rotated in place;
+                        // FP8: widened to bf16 in place
+                        if (ROPE || FP8) ok = mbar_wait(smem_u32(&sm.q_rot[t]), 0, abort_flag, 0x27);
                         if (!ok) break;
                         tc_fence_after();
                         issue_s(t, 0);
@@ -610,6 +619,36 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (warp_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x36)) {
                     const int pend = Sq - p0[t];   // rows at positions >= Sq hold no query
                     rt.apply(smem_u32(sm.q[t]), C::QBOX, r, [&](int row) { return (row & pmask) < pend; });
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(smem_u32(&sm.q_rot[t]));
+            }
+            if constexpr (FP8) {
+                // widen this row's e4m3 query values (staged in the tile's
+                // second box) to bf16 in the layout the score MMAs read. A
+                // row's 128 staged bytes and its 128 bf16 bytes of the second
+                // box are the same 128-byte row (the swizzle permutes chunks
+                // within a row), so each thread reads its dims 64-127 before
+                // writing them back and no thread touches another's row.
+                const uint32_t qt = smem_u32(sm.q[t]);
+                if (warp_wait(smem_u32(&sm.q_full), 0, abort_flag, 0x37)) {
+                    auto get = [&](int c) { return lds128(qt + C::QBOX + swz<3>((uint32_t)(r * 128 + c * 16))); };
+                    auto put = [&](int c, const uint4 &x) {   // e4m3 chunk c = dims 16c .. 16c + 15
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int e0 = 16 * c + 8 * hf;
+                            const int bx = e0 / C::BOXD, ci = (e0 % C::BOXD) / 8;
+                            const uint4 w = hf ? e4m3x8_to_bf16x8(x.z, x.w) : e4m3x8_to_bf16x8(x.x, x.y);
+                            sts128(qt + bx * C::QBOX + swz<C::SWB>((uint32_t)(r * C::ROWB + ci * 16)), w);
+                        }
+                    };
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) put(c, get(c));
+                    uint4 hi[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) hi[c] = get(4 + c);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) put(4 + c, hi[c]);
                     fence_proxy_async_smem();
                 }
                 mbar_arrive(smem_u32(&sm.q_rot[t]));

@@ -360,6 +360,20 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
     __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&t);
 }
+
+// 8 e4m3 values (two words) to 8 bf16 values (four words): e4m3 -> f16 and
+// f16 -> fp32 are exact, and fp32 -> bf16 is exact for these values (at most
+// 4 significant bits, exponents 2^-9 .. 2^8).
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint32_t lo, uint32_t hi) {
+    const uint4 h = e4m3x8_to_f16x8(lo, hi);
+    auto cv = [](uint32_t h2) {
+        float a, b;
+        asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+            : "=f"(a), "=f"(b) : "r"(h2));
+        return f2_to_bf2(a, b);
+    };
+    return make_uint4(cv(h.x), cv(h.y), cv(h.z), cv(h.w));
+}
 // Packed fp32 pair arithmetic (one FFMA2 / FADD2 / FMUL2 instruction each).
 // The pairs are assembled inside the asm block so no value goes through memory.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
