@@ -102,7 +102,8 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
  * e4m3 query tiles and widens them in shared memory, folds the query and
  * key tile scales into each score tile's exponent scale and the value
  * tile's scale into P (the row sums take P unscaled). Two launches on
- * `stream`.
+ * `stream`, the second a programmatic dependent of the first (its prologue
+ * and query tiles overlap the widening of the keys and values).
  * Supported: d == 128, and the rest as attn_fwd.
  * Returns ATTN_OK or an error code (nothing launched on error).
  */

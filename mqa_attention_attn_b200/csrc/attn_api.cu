@@ -311,9 +311,23 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
             attn::pf::prefill_kernel<D, kWindow><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
                                                                                                        p);
         } else if (f8) {
-            if constexpr (D == 128)
-                attn::pf::prefill_kernel<D, kFp8><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
-                                                                                                        p);
+            // a programmatic dependent of the widening pass: the prologue, the
+            // e4m3 query tiles and their widening overlap it, and only the K
+            // and V producers wait for it
+            if constexpr (D == 128) {
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3((unsigned)grid);
+                cfg.blockDim = dim3(attn::pf::THREADS);
+                cfg.dynamicSmemBytes = smem;
+                cfg.stream = stream;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                attr[0].val.programmaticStreamSerializationAllowed = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                if (cudaLaunchKernelEx(&cfg, attn::pf::prefill_kernel<D, kFp8>, tq, tk, tv, to, p) != cudaSuccess)
+                    return ATTN_ERR_CUDA;
+            }
         } else
             attn::pf::prefill_kernel<D, kDense><<<(unsigned)grid, attn::pf::THREADS, smem, stream>>>(tq, tk, tv, to,
                                                                                                       p);

@@ -55,6 +55,9 @@ __device__ __forceinline__ void widen_array(const uint8_t *src, uint16_t *dst, s
 // 16-byte loads, two 16-byte stores per load).
 __global__ void __launch_bounds__(WIDEN_THREADS) widen_e4m3_kernel(const WidenSeg a, const WidenSeg b,
                                                                     const WidenSeg c) {
+    // the attention grid launched after this one may start its prologue
+    // (it waits for this grid before it reads the widened arrays)
+    griddep_launch_dependents();
     const size_t first = (size_t)blockIdx.x * WIDEN_THREADS + threadIdx.x;
     const size_t stride = (size_t)gridDim.x * WIDEN_THREADS;
     widen_array(a.src, a.dst, a.n16, first, stride);

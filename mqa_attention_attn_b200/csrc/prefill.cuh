@@ -365,7 +365,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // K tiles issued during setup (ROPE: the rotated keys come from the grid
     // launched just before this one, so its K tiles wait in the producer;
     // PAGED: the page lookups issued here spill in the producer's registers)
-    const int k_early = (kEarlyLoads && !ROPE && !PAGED) ? min(KSTAGE, nmax) : 0;
+    const int k_early = (kEarlyLoads && !ROPE && !PAGED && !FP8) ? min(KSTAGE, nmax) : 0;
 
     // ---- setup: barriers (warp 0), TMEM (warp 1)
     if (warp == 0 && lane == 0) {
@@ -427,7 +427,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if constexpr (!kEarlyLoads) load_q();
             // K tiles (V tiles are loaded by warp 2). ROPE: the rotated keys come
             // from the grid launched just before this one
-            if (ROPE) griddep_wait();
+            // FP8: the widened keys come from the grid launched just before
+            if (ROPE || FP8) griddep_wait();
             int issued = k_early;
             for (int j = k_early; j < nmax; ++j) {
                 // K tile j - KSTAGE is free once iteration j - KSTAGE - 1 is released
@@ -451,6 +452,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int tail_tile = (PAGED && Skv % BN != 0 && (Skv - 1) / BN < nmax) ? (Skv - 1) / BN : -1;
         int issued = 0;
         if (lane == 0) {
+            if (FP8) griddep_wait();   // the widened values, likewise
             for (int j = 0; j < nmax; ++j) {
                 const int s = j % VSTAGE;
                 // V tile j - VSTAGE is free once iteration j - VSTAGE is released
