@@ -801,11 +801,13 @@ def run_ours(args):
         ms_fp = mean["fp8_prefill"]
         out["fp8_prefill"] = {"workload": f"{w.name}, e4m3 q, k, v with one scale per 128-row tile",
                               "ms": ms_fp, "tflops": tf(fl_p, ms_fp), "frac_of_peak": tf(fl_p, ms_fp) / peak_tf,
-                              "kernels": "attn::f8::widen_e4m3_kernel (e4m3 -> f16 into the workspace) + "
-                                         "attn::pf::prefill_kernel<128, fp8> (f16 MMAs, tile scales folded in)",
-                              "roofline": tensor_roofline(fl_p, ms_fp, "attn::pf::prefill_kernel<128, fp8>", None,
-                                                          "achieved over both launches; f16 operands run at the "
-                                                          "bf16 rate")}
+                              "kernels": "attn::f8::widen_e4m3_kernel (keys and values, e4m3 -> bf16) + "
+                                         "attn::pf::prefill_kernel<128, fp8> (queries widened in shared memory, "
+                                         "tile scales folded in)",
+                              "roofline": tensor_roofline(fl_p, ms_fp, "attn::pf::prefill_kernel<128, fp8>",
+                                                          "prefill_kernel_128_fp8",
+                                                          "achieved over both launches; traffic of the attention "
+                                                          "kernel")}
     if "rope_prefill" in regimes:
         ms_rp, ms_rd = mean["rope_prefill"], mean["rope_decode"]
         out["rope_prefill"] = {"workload": f"{w.name}, RoPE base {ROPE_BASE:g} on q and k", "ms": ms_rp,
