@@ -138,3 +138,34 @@ def test_window_fp8_paged_validation(lib):
     assert paged(pool=0) == -1
     assert paged(page=48) == -2
     assert paged(ws=16) == -4
+
+
+def test_fp8_prefill_validation(lib):
+    """attn_fwd_fp8 answers argument errors before any launch, and sizes its
+    workspace as the keys and values widened to bf16 (256-byte aligned)."""
+    vp = ctypes.c_void_p(256)
+    out = ctypes.c_size_t(0)
+    assert lib.attn_fwd_fp8_workspace_bytes(1, 4096, 4096, 32, 8, 128, ctypes.byref(out)) == 0
+    assert out.value == 2 * (1 * 8 * 4096 * 128 * 2)
+    assert lib.attn_fwd_fp8_workspace_bytes(2, 100, 130, 8, 2, 128, ctypes.byref(out)) == 0
+    assert out.value == 2 * ((2 * 2 * 130 * 128 * 2 + 255) // 256 * 256)
+    assert lib.attn_fwd_fp8_workspace_bytes(1, 64, 64, 4, 2, 64, ctypes.byref(out)) == -2     # d != 128
+    lib.attn_fwd_fp8_workspace_bytes(1, 256, 256, 8, 2, 128, ctypes.byref(out))
+    need = out.value
+
+    def call(q=vp, qs=vp, n_q=8, n_kv=2, d=128, Sq=256, Skv=256, causal=1, scale=0.1, ws=vp, ws_bytes=need):
+        return lib.attn_fwd_fp8(q, vp, vp, qs, vp, vp, vp, None, 1, Sq, Skv, n_q, n_kv, d, causal, scale, ws,
+                                ws_bytes, None)
+    assert call(n_q=7) == -1                      # n_q % n_kv
+    assert call(causal=2) == -1
+    assert call(scale=float("nan")) == -1
+    assert call(q=None) == -1                     # null operand
+    assert call(qs=None) == -1                    # null scales
+    assert call(d=64) == -2                       # head dim 128 only
+    assert call(n_q=12, n_kv=2) == -2             # group size not a power of two
+    assert call(Sq=300, Skv=256) == -2            # causal with Sq > Skv
+    assert call(q=ctypes.c_void_p(264)) == -3     # misaligned operand
+    assert call(ws=None) == -4                    # workspace missing
+    assert call(ws_bytes=need - 1) == -4          # workspace too small
+    assert call(ws=ctypes.c_void_p(272)) == -3    # workspace not 256-byte aligned
+    assert lib.attn_fwd_fp8(vp, vp, vp, vp, vp, vp, vp, None, 0, 256, 256, 8, 2, 128, 1, 0.1, None, 0, None) == 0
