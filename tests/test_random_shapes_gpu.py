@@ -4,11 +4,11 @@ The parametrised tests elsewhere pin chosen shapes (tile edges, ragged tails,
 head-group sizes); these draw shapes at random (a fixed, derandomised
 hypothesis search, so a run is repeatable) over the supported space: head
 group sizes, head dims, lengths on and off the 128-row/128-key tiles, causal
-and not, batches with empty sequences, and windows with sink keys.
+and not, batches with empty sequences, windows with sink keys, the MLA
+latent decode and the paged decode.
 """
 import math
 
-import numpy as np
 import pytest
 import torch
 from hypothesis import given, settings, HealthCheck
@@ -119,3 +119,55 @@ def test_window_decode_random_shapes(shape, W, n_sink, seed):
     assert binding.device_status() == 0
     o_ref, lse_ref = oracle.sdpa_window(q[:, :, None, :], kc, vc, False, W, n_sink, 0.1, seqlens=seq.numpy())
     check_parity(o, lse, o_ref[:, :, 0], lse_ref[:, :, 0], f"window decode {shape} W={W} sinks={n_sink}")
+
+
+@st.composite
+def mla_shapes(draw):
+    B = draw(st.integers(1, 3))
+    n_q = draw(st.sampled_from([128, 256]))
+    S_max = draw(st.integers(1, 2500))
+    lens = draw(st.lists(st.integers(0, S_max), min_size=B, max_size=B))
+    return B, n_q, S_max, lens
+
+
+@settings(max_examples=12, deadline=None, derandomize=True, database=None, suppress_health_check=list(HealthCheck))
+@given(mla_shapes(), st.integers(0, 2**31 - 1))
+def test_mla_decode_random_shapes(shape, seed):
+    """The absorbed MLA decode (576-wide latent rows, values = their first
+    512 columns) over random batches, lengths and one or two head blocks:
+    batches too small to fill the SMs are split over key chunks."""
+    binding = need_gpu()
+    B, n_q, S_max, lens = shape
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = torch.randn(B, n_q, 576, generator=g, device="cuda").to(torch.bfloat16)
+    cache = torch.randn(B, S_max, 576, generator=g, device="cuda").to(torch.bfloat16)
+    seq = torch.tensor(lens, dtype=torch.int32)
+    c4 = cache[:, None]
+    scale = 1.0 / math.sqrt(192)
+    o, lse = binding.attn_decode(q, c4, c4, seq.cuda(), scale, d_v=512)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    o_ref, lse_ref = oracle.sdpa(q[:, :, None, :], c4, c4, False, scale, seqlens=seq.numpy(), d_v=512)
+    check_parity(o, lse, o_ref[:, :, 0], lse_ref[:, :, 0], f"mla decode {shape}")
+
+
+@st.composite
+def paged_shapes(draw):
+    page = draw(st.sampled_from([16, 32, 64, 128, 256]))
+    n_kv = draw(st.sampled_from([1, 2, 8]))
+    G = draw(st.sampled_from([1, 2, 4, 8]))
+    B = draw(st.integers(1, 4))
+    lens = draw(st.lists(st.integers(0, 2000), min_size=B, max_size=B))
+    return B, n_kv * G, n_kv, page, lens
+
+
+@settings(max_examples=16, deadline=None, derandomize=True, database=None, suppress_health_check=list(HealthCheck))
+@given(paged_shapes(), st.integers(0, 2**31 - 1))
+def test_paged_decode_random_shapes(shape, seed):
+    """The paged decode with random page sizes, group sizes and lengths, each
+    sequence's pages drawn at random from a pool with spare pages."""
+    from test_paged_decode_gpu import _case, _check
+    B, n_q, n_kv, page, lens = shape
+    pages_per_seq = max(1, -(-max(lens) // page)) + 1
+    q, pk, pv, table, sl = _case(B, n_q, n_kv, page, pages_per_seq, lens, seed % 100000)
+    _check(q, pk, pv, table, sl, 1.0 / math.sqrt(128), f"paged decode {shape}")
