@@ -74,6 +74,15 @@ def prefill_bytes(w) -> float:
                  + 4 * w.B * w.n_q * w.Sq)
 
 
+def prefill_fp8_bytes(w) -> float:
+    """e4m3 q, k, v (one byte per element) and their fp32 tile scales, the
+    bf16 output and the fp32 LSE."""
+    tq, tk = -(-w.Sq // 128), -(-w.Skv // 128)
+    return float(w.B * w.n_q * w.Sq * w.d_qk + w.B * w.n_kv * w.Skv * (w.d_qk + w.d_v)
+                 + 4 * (w.B * w.n_q * tq + 2 * w.B * w.n_kv * tk)
+                 + 2 * w.B * w.n_q * w.Sq * w.d_v + 4 * w.B * w.n_q * w.Sq)
+
+
 def decode_bytes(w, seqlens, cache_elem_bytes=2) -> float:
     """K and V rows below each sequence's length (2 bytes per element, or 1
     for an FP8 cache), q, o (bf16) and lse (fp32)."""
@@ -801,6 +810,7 @@ def run_ours(args):
         ms_fp = mean["fp8_prefill"]
         out["fp8_prefill"] = {"workload": f"{w.name}, e4m3 q, k, v with one scale per 128-row tile",
                               "ms": ms_fp, "tflops": tf(fl_p, ms_fp), "frac_of_peak": tf(fl_p, ms_fp) / peak_tf,
+                              "algorithmic_flops": fl_p, "algorithmic_bytes": prefill_fp8_bytes(w),
                               "kernels": "attn::f8::widen_e4m3_kernel (keys and values, e4m3 -> bf16) + "
                                          "attn::pf::prefill_kernel<128, fp8> (queries widened in shared memory, "
                                          "tile scales folded in)",

@@ -56,3 +56,13 @@ def test_mla_bytes_read_each_latent_row_once():
     flops = bench.decode_flops(w, seqlens)
     assert abs(flops / 1e9 - 73.0) < 0.1
     assert math.isclose(flops, 2 * 64 * 128 * 4096 * (576 + 512))
+
+
+def test_fp8_prefill_bytes():
+    """The FP8 prefill's algorithmic bytes: one byte per q, k, v element, a
+    fp32 scale per 128-row tile of each (sequence, head), bf16 o, fp32 lse;
+    for the Llama-3-8B layout 16 + 4 + 4 MiB of e4m3 inputs, 32 MiB of o."""
+    w = inputs.WORKLOADS["llama3_8b_prefill"]
+    tiles = (w.B * w.n_q + 2 * w.B * w.n_kv) * 32
+    expect = (16 + 4 + 4 + 32) * 2 ** 20 + 4 * tiles + 4 * w.B * w.n_q * w.Sq
+    assert bench.prefill_fp8_bytes(w) == expect
